@@ -1,0 +1,252 @@
+"""CPU oracle of the KV-cache eviction + E8 lattice quantisation hot path.
+
+TEST INFRASTRUCTURE: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package.  The product path (the
+CUDA library and its binding) never calls it.
+
+The arithmetic lives in ``nq_oracle.c`` (plain C, fp32 with explicit fmaf,
+-ffp-contract=off); this module compiles it with gcc on first use and wraps it
+with numpy marshalling.  Every function cites, in the C source, the passage of
+the method description it follows:
+
+* "NexusQuant: training-free 10-33x KV cache compression" (zingnex.cn),
+  sections "Token eviction", "E8 lattice quantisation", "Implementation
+  details";
+* "Como comprimir o KV cache do seu LLM em 33x sem treino" (dev.to), section
+  "Como funciona (em 6 passos)", steps 1-5.
+
+Parity unpinned: end-to-end model quality (perplexity) -- it needs trained
+models and datasets.  Every other function is pinned by ``tests/test_oracle_*``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_SO = os.path.join(_BUILD, "liboq.so")
+_lock = threading.Lock()
+_lib = None
+
+D = 128
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile nq_oracle.c into _build/liboq.so (gcc); returns the path."""
+    os.makedirs(_BUILD, exist_ok=True)
+    stale = (not os.path.exists(_SO)) or os.path.getmtime(_SO) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+        sig = {
+            "oq_score": (None, [P, i32, i32, i32, P, P]),
+            "oq_kept_count": (i64, [i64, i64, i32]),
+            "oq_select": (i64, [P, i64, i64, i32, P]),
+            "oq_encode_unit": (i64, [P, P, i32, i64, i64, P, i64, dbl, i32, i32, P, P, P, P]),
+            "oq_decode_unit": (None, [P, P, P, P, i32, i64, P, i64, dbl, i32, i32, P, P]),
+            "oq_e8_batch": (None, [P, i64, P, P, P]),
+            "oq_fwht_batch": (None, [P, i64]),
+            "oq_f32_to_f16_batch": (None, [P, i64, P]),
+            "oq_f32_to_bf16_batch": (None, [P, i64, P]),
+            "oq_rope_batch": (None, [dbl, P, i64, P, P]),
+            "oq_rope_apply_batch": (None, [P, P, P, i64, i32]),
+            "oq_encode_batch": (i64, [P, i64, i32, P, P, i32, P, P]),
+            "oq_decode_batch": (None, [P, P, i64, i32, P, P, i32, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.asarray(a)
+    if a.dtype != np.uint16:
+        a = a.view(np.uint16) if a.dtype.itemsize == 2 else a.astype(np.uint16)
+    return np.ascontiguousarray(a)
+
+
+# ---------------------------------------------------------------- scalars
+def f32_to_f16_bits(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32).ravel()
+    out = np.empty(x.size, np.uint16)
+    _load().oq_f32_to_f16_batch(_p(x), x.size, _p(out))
+    return out
+
+
+def f32_to_bf16_bits(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32).ravel()
+    out = np.empty(x.size, np.uint16)
+    _load().oq_f32_to_bf16_batch(_p(x), x.size, _p(out))
+    return out
+
+
+def bf16_bits_to_f32(b) -> np.ndarray:
+    b = np.asarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+# ------------------------------------------------------------- transforms
+def fwht(v) -> np.ndarray:
+    """Unnormalised Sylvester FWHT of [..., 128] fp32 rows (stages h ascending)."""
+    v = np.array(v, dtype=np.float32, copy=True, order="C")
+    shp = v.shape
+    v = v.reshape(-1, D)
+    _load().oq_fwht_batch(_p(v), v.shape[0])
+    return v.reshape(shp)
+
+
+def rope_cs(theta: float, pos) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 (cos, sin) rows [n][64] for the given positions (two-level rule)."""
+    pos = np.ascontiguousarray(np.atleast_1d(pos), dtype=np.int64)
+    c = np.empty((pos.size, D // 2), np.float32)
+    s = np.empty((pos.size, D // 2), np.float32)
+    _load().oq_rope_batch(float(theta), _p(pos), pos.size, _p(c), _p(s))
+    return c, s
+
+
+def rope_apply(v, c, s, direction: int) -> np.ndarray:
+    """direction -1: undo (rotate by -angle); +1: redo.  v [n][128] fp32."""
+    v = np.array(v, dtype=np.float32, copy=True, order="C").reshape(-1, D)
+    c = np.ascontiguousarray(c, dtype=np.float32).reshape(-1, D // 2)
+    s = np.ascontiguousarray(s, dtype=np.float32).reshape(-1, D // 2)
+    _load().oq_rope_apply_batch(_p(v), _p(c), _p(s), v.shape[0], int(direction))
+    return v
+
+
+def e8_nearest(y) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Nearest E8 point of [n][8] fp32 groups.
+
+    Returns (t = 2q int32 [n][8], coset int32 [n] (1 = half-integer), fp32 distance [n])."""
+    y = np.ascontiguousarray(y, dtype=np.float32).reshape(-1, 8)
+    n = y.shape[0]
+    t = np.empty((n, 8), np.int32)
+    cs = np.empty(n, np.int32)
+    d = np.empty(n, np.float32)
+    _load().oq_e8_batch(_p(y), n, _p(t), _p(cs), _p(d))
+    return t, cs, d
+
+
+# ------------------------------------------------------ vector codec
+def words_per_vector(bits: int) -> int:
+    return 4 * bits
+
+
+def encode_vectors(x_bf16, bits: int, rope: bool = False, c=None, s=None):
+    """Encode [n][128] bf16 vectors; returns (words [n][4b] u32, meta [n] u32, clamps)."""
+    x = _u16(x_bf16).reshape(-1, D)
+    n = x.shape[0]
+    if c is None:
+        c = np.zeros((n, D // 2), np.float32)
+        s = np.zeros((n, D // 2), np.float32)
+    c = np.ascontiguousarray(c, dtype=np.float32).reshape(n, D // 2)
+    s = np.ascontiguousarray(s, dtype=np.float32).reshape(n, D // 2)
+    w = np.empty((n, 4 * bits), np.uint32)
+    m = np.empty(n, np.uint32)
+    cl = _load().oq_encode_batch(_p(x), n, int(rope), _p(c), _p(s), bits, _p(w), _p(m))
+    return w, m, int(cl)
+
+
+def decode_vectors(words, meta, bits: int, rope: bool = False, c=None, s=None):
+    """Decode [n] packed vectors to [n][128] bf16 bits (uint16)."""
+    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, 4 * bits)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32).ravel()
+    n = words.shape[0]
+    if c is None:
+        c = np.zeros((n, D // 2), np.float32)
+        s = np.zeros((n, D // 2), np.float32)
+    c = np.ascontiguousarray(c, dtype=np.float32).reshape(n, D // 2)
+    s = np.ascontiguousarray(s, dtype=np.float32).reshape(n, D // 2)
+    out = np.empty((n, D), np.uint16)
+    _load().oq_decode_batch(_p(words), _p(meta), n, int(rope), _p(c), _p(s), bits, _p(out))
+    return out
+
+
+# ------------------------------------------------------ unit level
+def score_unit(K_unit, W: int, return_mean: bool = False):
+    """Key-key proxy scores of one layer; K_unit [H][T][128] bf16."""
+    K = _u16(K_unit)
+    H, T, d = K.shape
+    assert d == D
+    out = np.empty(T, np.float64)
+    mean = np.empty((H, D), np.float32)
+    _load().oq_score(_p(K), H, T, int(W), _p(out), _p(mean))
+    return (out, mean) if return_mean else out
+
+
+def kept_count(T: int, W: int, pct: int) -> int:
+    return int(_load().oq_kept_count(int(T), int(W), int(pct)))
+
+
+def select(scores, W: int, pct: int) -> np.ndarray:
+    """Ascending kept positions of one layer (int32)."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    T = s.size
+    kept = np.empty(T, np.int32)
+    n = _load().oq_select(_p(s), T, int(W), int(pct), _p(kept))
+    return kept[:n].copy()
+
+
+def encode_unit(K_unit, V_unit, n: int, kept=None, pos_base: int = 0, theta: float = 1e4,
+                bits_k: int = 3, bits_v: int = 2):
+    """Encode one layer.  K_unit/V_unit [H][T_in][128] bf16 (or None).
+
+    Returns dict with k_codes [H][n][4bk], k_meta [H][n], v_codes, v_meta, clamps."""
+    K = _u16(K_unit) if K_unit is not None else None
+    V = _u16(V_unit) if V_unit is not None else None
+    ref = K if K is not None else V
+    H, T_in, _ = ref.shape
+    kp = None if kept is None else np.ascontiguousarray(kept, dtype=np.int32)
+    kc = np.zeros((H, n, 4 * bits_k), np.uint32) if K is not None else None
+    km = np.zeros((H, n), np.uint32) if K is not None else None
+    vc = np.zeros((H, n, 4 * bits_v), np.uint32) if V is not None else None
+    vm = np.zeros((H, n), np.uint32) if V is not None else None
+    cl = _load().oq_encode_unit(_p(K), _p(V), H, T_in, n, _p(kp), int(pos_base), float(theta),
+                                bits_k, bits_v, _p(kc), _p(km), _p(vc), _p(vm))
+    return {"k_codes": kc, "k_meta": km, "v_codes": vc, "v_meta": vm, "clamps": int(cl)}
+
+
+def decode_unit(k_codes, k_meta, v_codes, v_meta, positions=None, pos_base: int = 0,
+                theta: float = 1e4, bits_k: int = 3, bits_v: int = 2):
+    """Decode one layer to (K_out, V_out) [H][n][128] bf16 bits (or None)."""
+    kc = None if k_codes is None else np.ascontiguousarray(k_codes, dtype=np.uint32)
+    km = None if k_meta is None else np.ascontiguousarray(k_meta, dtype=np.uint32)
+    vc = None if v_codes is None else np.ascontiguousarray(v_codes, dtype=np.uint32)
+    vm = None if v_meta is None else np.ascontiguousarray(v_meta, dtype=np.uint32)
+    ref = km if km is not None else vm
+    H, n = ref.shape
+    pp = None if positions is None else np.ascontiguousarray(positions, dtype=np.int32)
+    Ko = np.empty((H, n, D), np.uint16) if kc is not None else None
+    Vo = np.empty((H, n, D), np.uint16) if vc is not None else None
+    _load().oq_decode_unit(_p(kc), _p(km), _p(vc), _p(vm), H, n, _p(pp), int(pos_base),
+                           float(theta), bits_k, bits_v, _p(Ko), _p(Vo))
+    return Ko, Vo

@@ -1,0 +1,531 @@
+/*
+ * nq_oracle.c -- plain, slow, single-threaded CPU oracle of the NexusQuant
+ * KV-cache hot path: key-key token scoring, eviction, RoPE removal, Hadamard
+ * rotation, per-vector fp16 scale, E8 lattice quantisation, bit packing and
+ * the inverse path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the CPU
+ * baseline of the benchmark may load this file.  It shares no code, header,
+ * table or constant generator with the CUDA library; every step is written
+ * out here from the method description:
+ *
+ *   - "NexusQuant: training-free 10-33x KV cache compression"
+ *     (zingnex.cn, sections "Token eviction", "E8 lattice quantisation",
+ *     "Implementation details")
+ *   - "Como comprimir o KV cache do seu LLM em 33x sem treino"
+ *     (dev.to, section "Como funciona (em 6 passos)", steps 1-5)
+ *
+ * The pages leave every formula open; the readings taken (fp32 operation
+ * order, tie rules, scale rule, packed layout) are listed in the design doc and
+ * restated next to each function below.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
+ * (no SIMD intrinsics, no OpenMP).  -ffp-contract=off matters: every fused
+ * multiply-add below is an explicit fmaf(), every other product is rounded.
+ *
+ * Parity status: every function is pinned by tests under tests/ (closed
+ * forms, brute force, library routines); end-to-end model quality is
+ * "parity unpinned" (it needs models and datasets).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OQ_D 128
+#define OQ_HALF 64
+
+/* ---------------------------------------------------------------- floats */
+
+static float oq_u2f(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t oq_f2u(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* 1/sqrt(128) rounded to fp32, and 1/(A_b * sqrt(128)) for A_3 = 3.5 and
+ * A_2 = 1.5 (the largest code magnitude of a b-bit symmetric code), each the
+ * fp32 nearest to the real number. */
+#define OQ_C_BITS 0x3DB504F3u
+#define OQ_G3_BITS 0x3CCEE116u
+#define OQ_G2_BITS 0x3D715BEFu
+
+float oq_bf16_to_f32(uint16_t h) { return oq_u2f((uint32_t)h << 16); }
+
+/* IEEE round-to-nearest-even of an fp32 value to bfloat16 (finite inputs;
+ * NaN is kept quiet). */
+uint16_t oq_f32_to_bf16(float f)
+{
+    uint32_t u = oq_f2u(f);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu))
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* IEEE binary16 round-to-nearest-even of a finite fp32 value, written from
+ * the format definition (1 sign, 5 exponent, 10 fraction bits, bias 15).
+ * Overflow gives +-inf here; the scale rule saturates separately. */
+uint16_t oq_f32_to_f16(float f)
+{
+    uint32_t u = oq_f2u(f);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    uint32_t a = u & 0x7FFFFFFFu;
+    if (a >= 0x7F800000u) /* inf / nan */
+        return (uint16_t)(sign | 0x7C00u | (a > 0x7F800000u ? 0x200u : 0u));
+    int e = (int)(a >> 23) - 127;    /* unbiased exponent */
+    uint32_t m = (a & 0x7FFFFFu);
+    if (a == 0) return sign;
+    if (e > 15) return (uint16_t)(sign | 0x7C00u);
+    uint32_t full;  /* significand with hidden bit, 24 bits */
+    int shift;      /* bits to drop */
+    uint32_t ebits;
+    if (e >= -14) { /* normal binary16 range */
+        full = m | 0x800000u;
+        shift = 13;
+        ebits = (uint32_t)(e + 15);
+    } else {        /* subnormal binary16: value = frac * 2^-24 */
+        if ((int)(a >> 23) == 0) return sign; /* fp32 subnormal: far below 2^-25 */
+        full = m | 0x800000u;
+        shift = 13 + (-14 - e);
+        if (shift > 24) return sign; /* below half of the smallest subnormal */
+        ebits = 0;
+    }
+    uint32_t keep = full >> shift;
+    uint32_t rem = full & ((1u << shift) - 1u);
+    uint32_t halfway = 1u << (shift - 1);
+    if (rem > halfway || (rem == halfway && (keep & 1u))) keep += 1u;
+    uint32_t out;
+    if (ebits) {
+        /* keep has the hidden bit at position 10; a carry to bit 11 bumps the
+         * exponent, which the addition below does by itself */
+        out = ((ebits - 1u) << 10) + keep;
+    } else {
+        out = keep; /* may round up into the smallest normal, also correct */
+    }
+    if (out >= 0x7C00u) out = 0x7C00u;
+    return (uint16_t)(sign | out);
+}
+
+float oq_f16_to_f32(uint16_t h)
+{
+    uint32_t sign = (uint32_t)(h & 0x8000u) << 16;
+    uint32_t e = (h >> 10) & 0x1Fu, m = h & 0x3FFu;
+    if (e == 0) {
+        float v = (float)m * oq_u2f(0x33800000u); /* m * 2^-24, exact */
+        return sign ? -v : v;
+    }
+    if (e == 31) return oq_u2f(sign | 0x7F800000u | (m << 13));
+    return oq_u2f(sign | ((e - 15 + 127) << 23) | (m << 13));
+}
+
+/* ------------------------------------------------------------ rope table */
+
+/* Split-half rotary embedding (pairs (i, i+64)), frequencies
+ * omega_i = theta^(-2i/D) (NexusQuant, "Supported models": standard
+ * split-half RoPE only).  The angle at position p = 256a + b is split into
+ * two exactly-known parts; each part's cos/sin is evaluated in fp64 and
+ * rounded to fp32, then combined with the angle-addition identity in fp32:
+ *   c = fmaf(cos A, cos B, -(sin A * sin B)),
+ *   s = fmaf(sin A, cos B,  (cos A * sin B)). */
+void oq_rope_cs(double theta, int64_t pos, float *c, float *s)
+{
+    int64_t a = pos >> 8, b = pos & 255;
+    for (int i = 0; i < OQ_HALF; i++) {
+        double w = pow(theta, -(double)i / 64.0);
+        double angA = (double)(256 * a) * w;
+        double angB = (double)b * w;
+        float ca = (float)cos(angA), sa = (float)sin(angA);
+        float cb = (float)cos(angB), sb = (float)sin(angB);
+        float ss = sa * sb, cs = ca * sb;
+        c[i] = fmaf(ca, cb, -ss);
+        s[i] = fmaf(sa, cb, cs);
+    }
+}
+
+/* Remove the rotation that RoPE applied at this position (rotate by -angle):
+ *   u_i    = fmaf(k_i,    c, k_{i+64} * s)
+ *   u_i+64 = fmaf(k_i+64, c, -(k_i * s))          (NexusQuant step 3) */
+void oq_rope_undo(float *v, const float *c, const float *s)
+{
+    for (int i = 0; i < OQ_HALF; i++) {
+        float a = v[i], b = v[i + OQ_HALF];
+        float bs = b * s[i], as = a * s[i];
+        v[i] = fmaf(a, c[i], bs);
+        v[i + OQ_HALF] = fmaf(b, c[i], -as);
+    }
+}
+
+/* Re-apply the rotation after reconstruction (rotate by +angle). */
+void oq_rope_redo(float *v, const float *c, const float *s)
+{
+    for (int i = 0; i < OQ_HALF; i++) {
+        float a = v[i], b = v[i + OQ_HALF];
+        float bs = b * s[i], as = a * s[i];
+        v[i] = fmaf(a, c[i], -bs);
+        v[i + OQ_HALF] = fmaf(b, c[i], as);
+    }
+}
+
+/* ----------------------------------------------------------------- FWHT */
+
+/* Unnormalised Walsh-Hadamard transform in Sylvester (natural) order:
+ * stages h = 1, 2, 4, ..., 64, each butterfly (a, b) -> (a + b, a - b).
+ * The 1/sqrt(128) normalisation is folded into the scale (NexusQuant
+ * step 4: rotate so that no outlier dominates the quantisation scale). */
+void oq_fwht128(float *v)
+{
+    for (int h = 1; h < OQ_D; h <<= 1)
+        for (int i = 0; i < OQ_D; i++)
+            if (!(i & h)) {
+                float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+}
+
+/* ------------------------------------------------------------ E8 decode */
+
+/* Nearest point of D8 + shift (shift 0: D8 = integer vectors with even sum;
+ * shift 1/2: D8 + (1/2,...,1/2)), following the Conway-Sloane decoder for
+ * D_n: round every coordinate to the nearest integer, and if the sum is odd,
+ * re-round the coordinate with the largest rounding error the other way.
+ *
+ * fp32, in this order:
+ *   u_i = y_i - shift                 (rounded; exact for shift 0)
+ *   f_i = rint(u_i)                   (nearest, ties to even)
+ *   e_i = u_i - f_i                   (exact)
+ *   d   = e_0*e_0, then d = fmaf(e_i, e_i, d) for i = 1..7
+ *   if sum(f) is odd:
+ *     k   = first index of max |e_i|
+ *     f_k += (e_k >= 0 ? 1 : -1)
+ *     d   = d + fmaf(-2, |e_k|, 1)     (= |e|^2 after the move, since
+ *                                      (1-|e_k|)^2 - e_k^2 = 1 - 2|e_k|)
+ * Output: g[i] = f_i (the point is g + shift), return value d. */
+static float oq_d8_decode(const float *y, float shift, int32_t *g)
+{
+    float u[8], e[8];
+    int32_t f[8];
+    int32_t sum = 0;
+    for (int i = 0; i < 8; i++) {
+        u[i] = y[i] - shift;
+        float r = rintf(u[i]);
+        e[i] = u[i] - r;
+        f[i] = (int32_t)r;
+        sum += f[i];
+    }
+    float d = e[0] * e[0];
+    for (int i = 1; i < 8; i++) d = fmaf(e[i], e[i], d);
+    if (sum & 1) {
+        int k = 0;
+        float m = fabsf(e[0]);
+        for (int i = 1; i < 8; i++)
+            if (fabsf(e[i]) > m) { m = fabsf(e[i]); k = i; }
+        f[k] += (e[k] >= 0.0f) ? 1 : -1;
+        d = d + fmaf(-2.0f, m, 1.0f);
+    }
+    for (int i = 0; i < 8; i++) g[i] = f[i];
+    return d;
+}
+
+/* Nearest E8 point, E8 = D8 u (D8 + 1/2) (Conway-Sloane): decode both cosets
+ * and keep the closer; a tie keeps the integer coset.  t[i] = 2*q_i (all even
+ * for the integer coset, all odd for the half coset).  Returns the coset
+ * (0 integer, 1 half) and the chosen fp32 distance in *dist. */
+int oq_e8_nearest(const float *y, int32_t *t, float *dist)
+{
+    int32_t g0[8], g1[8];
+    float d0 = oq_d8_decode(y, 0.0f, g0);
+    float d1 = oq_d8_decode(y, 0.5f, g1);
+    if (d1 < d0) {
+        for (int i = 0; i < 8; i++) t[i] = 2 * g1[i] + 1;
+        if (dist) *dist = d1;
+        return 1;
+    }
+    for (int i = 0; i < 8; i++) t[i] = 2 * g0[i];
+    if (dist) *dist = d0;
+    return 0;
+}
+
+/* Clamp 2q to the b-bit symmetric code range and return the code:
+ *   half coset (t odd):     t in [-(2^b-1), 2^b-1],  j = (t + 2^b - 1)/2
+ *   integer coset (t even): t in [-(2^b-2), 2^b-2],  j = (t + 2^b - 2)/2
+ * Sets *clamped when t had to move. */
+static uint32_t oq_code(int32_t t, int half, int bits, int *clamped)
+{
+    int32_t lim = (1 << bits) - (half ? 1 : 2);
+    int32_t tc = t < -lim ? -lim : (t > lim ? lim : t);
+    if (tc != t) *clamped += 1;
+    return (uint32_t)((tc + lim) / 2);
+}
+
+/* --------------------------------------------------------------- encode */
+
+/* Encode one 128-vector (NexusQuant steps 3-5 plus packing):
+ *  1. bf16 -> fp32; for keys, undo RoPE at this position (c, s given).
+ *  2. unnormalised FWHT-128.
+ *  3. M = max|v|; sigma = fp16(fp32(M * G_b)), saturated at 65504;
+ *     r = fp32(C / sigma) (0 when sigma is 0); y_i = fp32(v_i * r), with a
+ *     zero product taken as +0.
+ *  4. each group of 8 consecutive coordinates -> nearest E8 point -> codes.
+ *  5. pack: the b-bit code of coordinate c sits at bits [b*c, b*c + b) of the
+ *     vector's little-endian stream of 4*b 32-bit words; meta word =
+ *     coset mask (bit g = group g in the half coset) | fp16(sigma) << 16.
+ * Returns the number of clamped coordinates. */
+int oq_encode_vector(const uint16_t *x, int rope, const float *c, const float *s,
+                     int bits, uint32_t *words, uint32_t *meta)
+{
+    float v[OQ_D];
+    for (int i = 0; i < OQ_D; i++) v[i] = oq_bf16_to_f32(x[i]);
+    if (rope) oq_rope_undo(v, c, s);
+    oq_fwht128(v);
+
+    float M = 0.0f;
+    for (int i = 0; i < OQ_D; i++) M = fmaxf(M, fabsf(v[i]));
+    float G = oq_u2f(bits == 3 ? OQ_G3_BITS : OQ_G2_BITS);
+    float C = oq_u2f(OQ_C_BITS);
+    float sm = M * G;
+    if (sm > 65504.0f) sm = 65504.0f;
+    uint16_t sig16 = oq_f32_to_f16(sm);
+    float sig = oq_f16_to_f32(sig16);
+    float r = (sig == 0.0f) ? 0.0f : C / sig;
+
+    int nw = 4 * bits, clamped = 0;
+    for (int w = 0; w < nw; w++) words[w] = 0;
+    uint32_t cmask = 0;
+    for (int g = 0; g < 16; g++) {
+        float y[8];
+        for (int i = 0; i < 8; i++) {
+            float p = v[8 * g + i] * r;
+            y[i] = (p == 0.0f) ? 0.0f : p;
+        }
+        int32_t t[8];
+        int half = oq_e8_nearest(y, t, NULL);
+        if (half) cmask |= 1u << g;
+        for (int i = 0; i < 8; i++) {
+            uint32_t j = oq_code(t[i], half, bits, &clamped);
+            int bitpos = bits * (8 * g + i);
+            for (int k = 0; k < bits; k++)
+                if (j & (1u << k)) words[(bitpos + k) >> 5] |= 1u << ((bitpos + k) & 31);
+        }
+    }
+    *meta = cmask | ((uint32_t)sig16 << 16);
+    return clamped;
+}
+
+/* --------------------------------------------------------------- decode */
+
+/* Inverse of oq_encode_vector:
+ *  t_c = 2 j_c - 2^b + 2 - h_g   (h_g = coset bit of the group, t_c = 2 q_c)
+ *  w   = FWHT(t)                 (integers, |w| <= 896: exact in fp32)
+ *  kappa = fp32(fp32(sigma / 2) * C);  x_c = fp32(w_c * kappa)
+ *  keys: re-apply RoPE at this position; then bf16 round-to-nearest-even. */
+void oq_decode_vector(const uint32_t *words, uint32_t meta, int rope, const float *c,
+                      const float *s, int bits, uint16_t *out)
+{
+    float w[OQ_D];
+    for (int cidx = 0; cidx < OQ_D; cidx++) {
+        uint32_t j = 0;
+        int bitpos = bits * cidx;
+        for (int k = 0; k < bits; k++)
+            j |= ((words[(bitpos + k) >> 5] >> ((bitpos + k) & 31)) & 1u) << k;
+        int h = (meta >> (cidx >> 3)) & 1u;
+        int32_t t = 2 * (int32_t)j - (1 << bits) + 2 - h;
+        w[cidx] = (float)t;
+    }
+    oq_fwht128(w);
+    float sig = oq_f16_to_f32((uint16_t)(meta >> 16));
+    float kappa = (sig * 0.5f) * oq_u2f(OQ_C_BITS);
+    for (int i = 0; i < OQ_D; i++) w[i] = w[i] * kappa;
+    if (rope) oq_rope_redo(w, c, s);
+    for (int i = 0; i < OQ_D; i++) out[i] = oq_f32_to_bf16(w[i]);
+}
+
+/* ---------------------------------------------------------------- score */
+
+/* Key-key proxy importance (NexusQuant "Implementation details": fast
+ * key-key proxy; dev.to step 1: cross-head inner product), on the stored
+ * (RoPE'd) keys of one layer K[h][t][d] (bf16, contiguous):
+ *   m[h][d]  = fp32( (sum over t in [T-W, T) of K[h][t][d], fp64, t rising) / W )
+ *   score[t] = sum over h, then d, of (double)K[h][t][d] * (double)m[h][d] */
+void oq_score(const uint16_t *K, int H, int T, int W, double *score, float *mean_out)
+{
+    float *m = (float *)malloc(sizeof(float) * (size_t)H * OQ_D);
+    for (int h = 0; h < H; h++)
+        for (int d = 0; d < OQ_D; d++) {
+            double S = 0.0;
+            for (int t = T - W; t < T; t++)
+                S += (double)oq_bf16_to_f32(K[((size_t)h * T + t) * OQ_D + d]);
+            m[h * OQ_D + d] = (float)(S / (double)W);
+        }
+    for (int t = 0; t < T; t++) {
+        double acc = 0.0;
+        for (int h = 0; h < H; h++)
+            for (int d = 0; d < OQ_D; d++)
+                acc += (double)oq_bf16_to_f32(K[((size_t)h * T + t) * OQ_D + d]) *
+                       (double)m[h * OQ_D + d];
+        score[t] = acc;
+    }
+    if (mean_out) memcpy(mean_out, m, sizeof(float) * (size_t)H * OQ_D);
+    free(m);
+}
+
+/* --------------------------------------------------------------- select */
+
+/* Kept-token count: always BOS and the last W tokens (NexusQuant "Token
+ * eviction"); of the T-1-W middle tokens, floor(T_mid * pct / 100) are
+ * evicted.  Everything is kept when T <= 1 + W or pct == 0. */
+int64_t oq_kept_count(int64_t T, int64_t W, int pct)
+{
+    if (T <= 1 + W || pct <= 0) return T;
+    int64_t mid = T - 1 - W;
+    return T - (mid * pct) / 100;
+}
+
+typedef struct { double s; int32_t t; } oq_pair;
+
+static int oq_pair_cmp(const void *pa, const void *pb)
+{
+    const oq_pair *a = (const oq_pair *)pa, *b = (const oq_pair *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->t > b->t) - (a->t < b->t);
+}
+
+/* Kept positions in ascending order: 0, the top n_mid middle positions by
+ * (score descending, position ascending), and [T-W, T).  Returns n. */
+int64_t oq_select(const double *score, int64_t T, int64_t W, int pct, int32_t *kept)
+{
+    int64_t n = oq_kept_count(T, W, pct);
+    if (n == T) {
+        for (int64_t t = 0; t < T; t++) kept[t] = (int32_t)t;
+        return T;
+    }
+    int64_t mid = T - 1 - W, n_mid = n - 1 - W;
+    oq_pair *p = (oq_pair *)malloc(sizeof(oq_pair) * (size_t)mid);
+    for (int64_t i = 0; i < mid; i++) {
+        double s = score[1 + i];
+        p[i].s = (s == 0.0) ? 0.0 : s; /* -0 and +0 compare equal anyway */
+        p[i].t = (int32_t)(1 + i);
+    }
+    qsort(p, (size_t)mid, sizeof(oq_pair), oq_pair_cmp);
+    uint8_t *flag = (uint8_t *)calloc((size_t)T, 1);
+    flag[0] = 1;
+    for (int64_t i = 0; i < n_mid; i++) flag[p[i].t] = 1;
+    for (int64_t t = T - W; t < T; t++) flag[t] = 1;
+    int64_t k = 0;
+    for (int64_t t = 0; t < T; t++)
+        if (flag[t]) kept[k++] = (int32_t)t;
+    free(flag);
+    free(p);
+    return k;
+}
+
+/* ------------------------------------------------------ unit-level driver */
+
+/* Encode n slots of one (layer) unit.  K/V are [H][T_in][128] bf16
+ * (contiguous; either may be NULL).  Slot i reads input token
+ * src = kept ? kept[i] : i, at RoPE position pos_base + src, and writes
+ * codes[h][i][4*bits] / meta[h][i].  Returns the clamp count. */
+int64_t oq_encode_unit(const uint16_t *K, const uint16_t *V, int H, int64_t T_in, int64_t n,
+                       const int32_t *kept, int64_t pos_base, double theta, int bits_k,
+                       int bits_v, uint32_t *k_codes, uint32_t *k_meta, uint32_t *v_codes,
+                       uint32_t *v_meta)
+{
+    int64_t clamped = 0;
+    float c[OQ_HALF], s[OQ_HALF];
+    for (int64_t i = 0; i < n; i++) {
+        int64_t src = kept ? kept[i] : i;
+        if (K) oq_rope_cs(theta, pos_base + src, c, s);
+        for (int h = 0; h < H; h++) {
+            size_t vec = (size_t)h * n + (size_t)i;
+            if (K)
+                clamped += oq_encode_vector(K + ((size_t)h * T_in + src) * OQ_D, 1, c, s, bits_k,
+                                            k_codes + vec * 4 * bits_k, k_meta + vec);
+            if (V)
+                clamped += oq_encode_vector(V + ((size_t)h * T_in + src) * OQ_D, 0, c, s, bits_v,
+                                            v_codes + vec * 4 * bits_v, v_meta + vec);
+        }
+    }
+    return clamped;
+}
+
+/* Decode n slots of one unit into K_out/V_out [H][n][128] bf16; slot i is at
+ * RoPE position positions ? positions[i] : pos_base + i. */
+void oq_decode_unit(const uint32_t *k_codes, const uint32_t *k_meta, const uint32_t *v_codes,
+                    const uint32_t *v_meta, int H, int64_t n, const int32_t *positions,
+                    int64_t pos_base, double theta, int bits_k, int bits_v, uint16_t *K_out,
+                    uint16_t *V_out)
+{
+    float c[OQ_HALF], s[OQ_HALF];
+    for (int64_t i = 0; i < n; i++) {
+        int64_t pos = positions ? (int64_t)positions[i] : pos_base + i;
+        if (K_out) oq_rope_cs(theta, pos, c, s);
+        for (int h = 0; h < H; h++) {
+            size_t vec = (size_t)h * n + (size_t)i;
+            if (K_out)
+                oq_decode_vector(k_codes + vec * 4 * bits_k, k_meta[vec], 1, c, s, bits_k,
+                                 K_out + vec * OQ_D);
+            if (V_out)
+                oq_decode_vector(v_codes + vec * 4 * bits_v, v_meta[vec], 0, c, s, bits_v,
+                                 V_out + vec * OQ_D);
+        }
+    }
+}
+
+/* ------------------------------------------------ helpers for the pins */
+
+/* Batched E8 on [n][8] fp32 groups: t_out [n][8] = 2q, coset_out [n],
+ * dist_out [n]. */
+void oq_e8_batch(const float *y, int64_t n, int32_t *t_out, int32_t *coset_out, float *dist_out)
+{
+    for (int64_t i = 0; i < n; i++)
+        coset_out[i] = oq_e8_nearest(y + 8 * i, t_out + 8 * i, dist_out + i);
+}
+
+void oq_fwht_batch(float *v, int64_t n)
+{
+    for (int64_t i = 0; i < n; i++) oq_fwht128(v + OQ_D * i);
+}
+
+void oq_f32_to_f16_batch(const float *x, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = oq_f32_to_f16(x[i]);
+}
+
+void oq_f32_to_bf16_batch(const float *x, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = oq_f32_to_bf16(x[i]);
+}
+
+void oq_rope_batch(double theta, const int64_t *pos, int64_t n, float *c, float *s)
+{
+    for (int64_t i = 0; i < n; i++) oq_rope_cs(theta, pos[i], c + OQ_HALF * i, s + OQ_HALF * i);
+}
+
+/* Apply undo (dir = -1) or redo (dir = +1) to [n][128] fp32 vectors whose
+ * (c, s) rows are given [n][64]. */
+void oq_rope_apply_batch(float *v, const float *c, const float *s, int64_t n, int dir)
+{
+    for (int64_t i = 0; i < n; i++) {
+        if (dir < 0) oq_rope_undo(v + OQ_D * i, c + OQ_HALF * i, s + OQ_HALF * i);
+        else oq_rope_redo(v + OQ_D * i, c + OQ_HALF * i, s + OQ_HALF * i);
+    }
+}
+
+/* Encode a batch of vectors with per-vector positions (c, s rows given). */
+int64_t oq_encode_batch(const uint16_t *x, int64_t n, int rope, const float *c, const float *s,
+                        int bits, uint32_t *words, uint32_t *meta)
+{
+    int64_t clamped = 0;
+    for (int64_t i = 0; i < n; i++)
+        clamped += oq_encode_vector(x + OQ_D * i, rope, c + OQ_HALF * i, s + OQ_HALF * i, bits,
+                                    words + 4 * bits * i, meta + i);
+    return clamped;
+}
+
+void oq_decode_batch(const uint32_t *words, const uint32_t *meta, int64_t n, int rope,
+                     const float *c, const float *s, int bits, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        oq_decode_vector(words + 4 * bits * i, meta[i], rope, c + OQ_HALF * i, s + OQ_HALF * i,
+                         bits, out + OQ_D * i);
+}
