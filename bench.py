@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of the KV-cache eviction + E8 lattice codec hot path on B200.
+
+One step = one pass of the whole path over one synthetic KV cache held in
+HBM: key-key scores -> token selection -> E8 encode (K3V2) -> decode back to
+bf16, all layers batched into one call per stage.  Default workload: the
+Mistral-7B-shaped cache (32 layers x 8 KV heads x 32768 tokens x 128, bf16,
+theta 1e6, 60% eviction with BOS + 64-token window), inputs 4.3 GB > L2.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU runs are replicas (weak scaling):
+every rank compresses its own cache; there is no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from e8_lattice_vector_nq_b200 import synth  # noqa: E402
+
+METRIC = "KV encode+decode GB/s (bf16 in)"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mistral7b_32k")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-layers", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="override layer count (small runs)")
+    ap.add_argument("--tokens", type=int, default=0, help="override token count (small runs)")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "e8_lattice_vector_nq_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from profiles/traffic.txt, if taken on the current sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = kernel_source_hash()
+    with open(p) as f:
+        for line in f:
+            parts = line.split("#", 1)[0].split()
+            if len(parts) == 4 and parts[0] == kernel and parts[1] == workload and parts[3] == cur:
+                return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+
+            self.path = tempfile.mktemp(suffix=".csv")
+            q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_power_cap")
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 7:
+                    continue
+                try:
+                    sm.append(float(p[0]))
+                    mx.append(float(p[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[3:7]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                             timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def build_workload(args):
+    wl = synth.WORKLOADS[args.workload]
+    kw = {}
+    if args.layers:
+        kw["layers"] = args.layers
+    if args.tokens:
+        kw["tokens"] = args.tokens
+    if kw:
+        from dataclasses import replace
+
+        wl = replace(wl, **kw)
+    return wl
+
+
+def gen_cache(wl, device, layers=None):
+    L = wl.layers if layers is None else layers
+    K = torch.empty(L, wl.heads, wl.tokens, 128, dtype=torch.bfloat16, device=device)
+    V = torch.empty_like(K)
+    for l in range(L):
+        k, v = synth.gen_layer(wl, l, device)
+        K[l].copy_(k)
+        V[l].copy_(v)
+        del k, v
+    return K, V
+
+
+def algorithmic_bytes(wl, n_kept, units):
+    H, T = wl.heads, wl.tokens
+    bk = 4 * 4 * wl.bits_k + 4
+    bv = 4 * 4 * wl.bits_v + 4
+    evict = wl.evict_pct > 0 and T > 1 + wl.window
+    out = {
+        "encode": units * (n_kept * H * (256 + 256 + bk + bv) + (n_kept * 4 if evict else 0)),
+        "decode": units * (n_kept * H * (bk + bv + 256 + 256) + (n_kept * 4 if evict else 0)),
+    }
+    if evict:
+        out["score"] = units * (T * H * 256 + T * 8)
+        out["select"] = units * (T * 8 + n_kept * 4)
+    return out
+
+
+# --------------------------------------------------------------- oracle arm
+def oracle_pass(oq, Kl, Vl, wl):
+    """One layer through the CPU oracle: score, select, encode, decode."""
+    T = Kl.shape[1]
+    evict = wl.evict_pct > 0 and T > 1 + wl.window
+    kept = None
+    n = T
+    if evict:
+        s = oq.score_unit(Kl, wl.window)
+        kept = oq.select(s, wl.window, wl.evict_pct)
+        n = kept.size
+    r = oq.encode_unit(Kl, Vl, n, kept=kept, theta=wl.theta, bits_k=wl.bits_k, bits_v=wl.bits_v)
+    oq.decode_unit(r["k_codes"], r["k_meta"], r["v_codes"], r["v_meta"], positions=kept,
+                   theta=wl.theta, bits_k=wl.bits_k, bits_v=wl.bits_v)
+
+
+def host_layer(wl, layer, device):
+    k, v = synth.gen_layer(wl, layer, device)
+    u16 = lambda t: t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    return u16(k), u16(v)
+
+
+def cpu_baseline(wl, layers, device, hl=None):
+    import oracle as oq
+
+    oq.build()
+    t = 0.0
+    nbytes = 0
+    for l in range(layers):
+        Kl, Vl = hl if hl is not None else host_layer(wl, l, device)
+        t0 = time.perf_counter()
+        oracle_pass(oq, Kl, Vl, wl)
+        t += time.perf_counter() - t0
+        nbytes += Kl.nbytes + Vl.nbytes
+    return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{layers} of {wl.layers} layers ({wl.heads} heads x {wl.tokens} tokens), "
+                      f"score+select+encode+decode, single-threaded C oracle"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl = build_workload(args)
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    import oracle as oq
+
+    oq.build()
+    Kl, Vl = host_layer(wl, 0, device)
+    per = Kl.nbytes + Vl.nbytes
+    for _ in range(args.warmup):
+        oracle_pass(oq, Kl, Vl, wl)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_pass(oq, Kl, Vl, wl)
+    dt = time.perf_counter() - t0
+    val = per * args.steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "layers": wl.layers, "heads": wl.heads, "tokens": wl.tokens,
+                   "bits": f"K{wl.bits_k}V{wl.bits_v}", "evict_pct": wl.evict_pct,
+                   "window": wl.window, "theta": wl.theta,
+                   "step": "one layer of the cache per step (bounded sample)"},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"1 of {wl.layers} layers per step"},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    from e8_lattice_vector_nq_b200 import nq
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    wl = build_workload(args)
+    units = wl.layers
+    K, V = gen_cache(wl, device)
+    codec = nq.Codec(units, wl.heads, wl.tokens, wl.theta, wl.bits_k, wl.bits_v, window=wl.window,
+                     evict_pct=wl.evict_pct, device=device)
+    n = codec.n
+    Kd = torch.empty(units, wl.heads, n, 128, dtype=torch.bfloat16, device=device)
+    Vd = torch.empty_like(Kd)
+    stream = torch.cuda.current_stream(device)
+    stages = ["score", "select", "encode", "decode"] if codec.evict else ["encode", "decode"]
+
+    def step(ev=None):
+        if codec.evict:
+            if ev: ev[0].record(stream)
+            nq.nq_score(K, codec.W, codec.scores, codec.ws)
+            if ev: ev[1].record(stream)
+            nq.nq_select(codec.scores, codec.W, codec.pct, codec.kept)
+            if ev: ev[2].record(stream)
+        elif ev:
+            ev[2].record(stream)
+        nq.nq_encode(K, V, codec.k_store, codec.v_store, n, codec.rope, codec.max_pos, kept=codec.kept)
+        if ev: ev[3].record(stream)
+        nq.nq_decode(codec.k_store, codec.v_store, n, Kd, Vd, codec.rope, codec.max_pos,
+                     positions=codec.kept)
+        if ev: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    per_stage = {}
+    if codec.evict:
+        per_stage["score"] = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        per_stage["select"] = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    per_stage["encode"] = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    per_stage["decode"] = sum(e[3].elapsed_time(e[4]) for e in evs) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    assert nq.device_error() == 0, "a kernel reported a bounded-wait timeout"
+
+    in_bytes = K.numel() * 2 + V.numel() * 2
+    ms_step = ms / args.steps
+    value = world * in_bytes / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    alg = algorithmic_bytes(wl, n, units)
+    dom = max(per_stage, key=per_stage.get)
+    achieved = alg[dom] / (per_stage[dom] * 1e-3) / 1e9
+    kernel_name = {"score": "score_kernel", "select": "select_kernel", "encode": "encode_kernel",
+                   "decode": "decode_kernel"}[dom]
+    traffic = recorded_traffic(kernel_name, wl.name)
+
+    enc_ms = sum(per_stage[s] for s in stages if s != "decode")
+    out_bytes = Kd.numel() * 2 + Vd.numel() * 2
+    packed_bits = codec.packed_bytes * 8
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "layers": wl.layers, "heads": wl.heads, "tokens": wl.tokens,
+                   "head_dim": 128, "bits": f"K{wl.bits_k}V{wl.bits_v}",
+                   "evict_pct": wl.evict_pct, "window": wl.window, "theta": wl.theta,
+                   "kept_per_layer": n, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world}"},
+        "stages_ms": {k: round(v, 4) for k, v in per_stage.items()},
+        "encode_gbs": in_bytes / (enc_ms * 1e-3) / 1e9,
+        "decode_gbs": out_bytes / (per_stage["decode"] * 1e-3) / 1e9,
+        "tokens_layers_per_s": world * wl.tokens * wl.layers / (ms_step * 1e-3),
+        "bits_per_elem": packed_bits / (K.numel() + V.numel()),
+        "hbm_frac_of_step": (sum(alg.values()) / (ms_step * 1e-3) / 1e9) / peak,
+        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes": alg[dom]},
+        "gpu_launches": args.steps * (5 if codec.evict else 2),
+    }
+    clocks = clk.summary()
+    if clocks:
+        line["clocks"] = clocks
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes)
+    if not args.no_cpu_baseline and rank == 0:
+        del Kd, Vd
+        hl = (K[0].cpu().view(torch.int16).numpy().view(np.uint16),
+              V[0].cpu().view(torch.int16).numpy().view(np.uint16))
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_layers, device, hl=hl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
+    """Same metric through the public API with HOST buffers: pinned H2D of the
+    inputs, the four calls, D2H of the reconstructed cache, every step."""
+    from e8_lattice_vector_nq_b200 import nq
+
+    Kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
+    Vh = torch.empty(V.shape, dtype=V.dtype, pin_memory=True)
+    Kh.copy_(K)
+    Vh.copy_(V)
+    Koh = torch.empty(Kd.shape, dtype=Kd.dtype, pin_memory=True)
+    Voh = torch.empty(Vd.shape, dtype=Vd.dtype, pin_memory=True)
+
+    def step():
+        K.copy_(Kh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        codec.encode(K, V)
+        codec.decode(Kd, Vd)
+        Koh.copy_(Kd, non_blocking=True)
+        Voh.copy_(Vd, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([ms], device=K.device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * in_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": Kd.numel() * 2 + Vd.numel() * 2,
+            "ms_per_step": ms, "steps": args.e2e_steps}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,258 @@
+// nq_abi.cu -- the extern "C" boundary of libnq: argument validation, RoPE
+// table construction on the host, status codes and error messages.  Every
+// compute entry point validates all sizes, strides and alignments on the host
+// and launches nothing when they are wrong.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "nq_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+
+nq_status fail(nq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+nq_status cuda_status(cudaError_t err, const char* what) {
+  if (err == cudaSuccess) return NQ_OK;
+  return fail(NQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nq_status check_kv(const void* p, nq_kv_strides s, const char* name) {
+  if (!p) return fail(NQ_ERR_INVALID, "%s is NULL", name);
+  if (!aligned(p, 16)) return fail(NQ_ERR_INVALID, "%s must be 16-byte aligned", name);
+  if (s.unit < 0 || s.head < 0 || s.token < 0 || s.unit % 8 || s.head % 8 || s.token % 8)
+    return fail(NQ_ERR_INVALID, "%s strides must be non-negative multiples of 8 elements", name);
+  return NQ_OK;
+}
+
+nq_status check_packed(const nq_packed* p, const char* name) {
+  if (!p) return fail(NQ_ERR_INVALID, "%s descriptor is NULL", name);
+  if (p->bits != 2 && p->bits != 3)
+    return fail(NQ_ERR_INVALID, "%s.bits must be 2 or 3 (got %d)", name, p->bits);
+  if (!p->codes || !p->meta) return fail(NQ_ERR_INVALID, "%s codes/meta is NULL", name);
+  if (!aligned(p->codes, 16)) return fail(NQ_ERR_INVALID, "%s.codes must be 16-byte aligned", name);
+  if (!aligned(p->meta, 4)) return fail(NQ_ERR_INVALID, "%s.meta must be 4-byte aligned", name);
+  if (p->unit_stride < 0 || p->head_stride < 0)
+    return fail(NQ_ERR_INVALID, "%s strides must be non-negative", name);
+  return NQ_OK;
+}
+
+nq_status check_rope(const float* tab, int64_t max_pos) {
+  if (!tab) return fail(NQ_ERR_INVALID, "rope_tab is NULL (required for keys)");
+  if (!aligned(tab, 8)) return fail(NQ_ERR_INVALID, "rope_tab must be 8-byte aligned");
+  if (max_pos < 1) return fail(NQ_ERR_INVALID, "rope_max_pos must be >= 1");
+  return NQ_OK;
+}
+
+constexpr int64_t kMaxSelectT = int64_t(1) << 20;
+
+}  // namespace
+
+extern "C" {
+
+const char* nq_last_error(void) { return g_last_error.c_str(); }
+
+int nq_version(void) { return 1; }
+
+int64_t nq_packed_bytes_per_vector(int bits) {
+  if (bits != 2 && bits != 3) return -1;
+  return 4 * (4 * bits) + 4;
+}
+
+size_t nq_rope_tables_bytes(int64_t max_pos) {
+  if (max_pos < 1) return 0;
+  const int64_t na = (max_pos + 255) / 256;
+  return static_cast<size_t>(na + 256) * nq::kHalf * 2 * sizeof(float);
+}
+
+nq_status nq_rope_tables_fill_host(double theta, int64_t max_pos, void* host_buf, size_t bytes) {
+  if (!(theta > 1.0) || !std::isfinite(theta)) return fail(NQ_ERR_INVALID, "theta must be > 1");
+  if (max_pos < 1) return fail(NQ_ERR_INVALID, "max_pos must be >= 1");
+  if (!host_buf) return fail(NQ_ERR_INVALID, "host_buf is NULL");
+  if (bytes < nq_rope_tables_bytes(max_pos))
+    return fail(NQ_ERR_WORKSPACE, "rope table buffer too small: %zu < %zu", bytes,
+                nq_rope_tables_bytes(max_pos));
+  float* t = static_cast<float*>(host_buf);
+  const int64_t na = (max_pos + 255) / 256;
+  for (int i = 0; i < nq::kHalf; ++i) {
+    // w_i = theta^(-2i/D) with D = 128
+    const double w = std::pow(theta, -static_cast<double>(i) / 64.0);
+    for (int64_t a = 0; a < na; ++a) {
+      const double ang = static_cast<double>(256 * a) * w;
+      t[2 * (a * nq::kHalf + i)] = static_cast<float>(std::cos(ang));
+      t[2 * (a * nq::kHalf + i) + 1] = static_cast<float>(std::sin(ang));
+    }
+    for (int64_t b = 0; b < 256; ++b) {
+      const double ang = static_cast<double>(b) * w;
+      t[2 * ((na + b) * nq::kHalf + i)] = static_cast<float>(std::cos(ang));
+      t[2 * ((na + b) * nq::kHalf + i) + 1] = static_cast<float>(std::sin(ang));
+    }
+  }
+  return NQ_OK;
+}
+
+size_t nq_score_workspace_bytes(int units, int heads) {
+  if (units < 0 || heads < 0) return 0;
+  return static_cast<size_t>(units) * heads * nq::kD * sizeof(float);
+}
+
+nq_status nq_score(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
+                   double* scores, void* ws, size_t ws_bytes, nq_stream_t stream) {
+  if (units < 0 || heads < 1 || heads > 1024)
+    return fail(NQ_ERR_INVALID, "need units >= 0 and 1 <= heads <= 1024");
+  if (T < 1 || W < 1 || W > T) return fail(NQ_ERR_INVALID, "need 1 <= W <= T");
+  if (heads > 256) return fail(NQ_ERR_UNSUPPORTED, "nq_score supports at most 256 heads");
+  if (units == 0) return NQ_OK;
+  if (nq_status st = check_kv(K, ks, "K")) return st;
+  if (!scores || !aligned(scores, 8)) return fail(NQ_ERR_INVALID, "scores NULL or misaligned");
+  if (!ws || !aligned(ws, 16)) return fail(NQ_ERR_INVALID, "workspace NULL or not 16-byte aligned");
+  if (ws_bytes < nq_score_workspace_bytes(units, heads))
+    return fail(NQ_ERR_WORKSPACE, "score workspace too small: %zu < %zu", ws_bytes,
+                nq_score_workspace_bytes(units, heads));
+  if (static_cast<int64_t>(units) * ((T + 63) / 64) > 0x7FFFFFFF)
+    return fail(NQ_ERR_UNSUPPORTED, "units * T too large for one launch");
+  return cuda_status(nq::launch_score(K, ks, units, heads, T, W, scores, static_cast<float*>(ws),
+                                      reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_score launch");
+}
+
+int64_t nq_kept_count(int64_t T, int64_t W, int evict_pct) {
+  if (T < 0 || W < 0) return -1;
+  if (T <= 1 + W || evict_pct <= 0) return T;
+  const int64_t mid = T - 1 - W;
+  const int pct = evict_pct > 100 ? 100 : evict_pct;
+  return T - (mid * pct) / 100;
+}
+
+nq_status nq_select(const double* scores, int units, int64_t T, int W, int evict_pct,
+                    int32_t* kept, int64_t kept_stride, nq_stream_t stream) {
+  if (units < 0 || T < 1 || W < 0 || W > T)
+    return fail(NQ_ERR_INVALID, "need units >= 0, T >= 1, 0 <= W <= T");
+  if (evict_pct < 0 || evict_pct > 100) return fail(NQ_ERR_INVALID, "evict_pct must be in [0, 100]");
+  if (T > kMaxSelectT)
+    return fail(NQ_ERR_UNSUPPORTED, "T = %lld exceeds the selection limit %lld",
+                static_cast<long long>(T), static_cast<long long>(kMaxSelectT));
+  if (units == 0) return NQ_OK;
+  if (!scores || !aligned(scores, 8)) return fail(NQ_ERR_INVALID, "scores NULL or misaligned");
+  if (!kept || !aligned(kept, 4)) return fail(NQ_ERR_INVALID, "kept NULL or misaligned");
+  const int64_t n = nq_kept_count(T, W, evict_pct);
+  if (kept_stride < n)
+    return fail(NQ_ERR_INVALID, "kept_stride %lld < kept count %lld",
+                static_cast<long long>(kept_stride), static_cast<long long>(n));
+  return cuda_status(nq::launch_select(scores, units, T, W, evict_pct, n, kept, kept_stride,
+                                       reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_select launch");
+}
+
+nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_strides vs, int units,
+                    int heads, int64_t T_in, int64_t n, const int32_t* kept, int64_t kept_stride,
+                    int64_t pos_base, const float* rope_tab, int64_t rope_max_pos,
+                    const nq_packed* k_out, const nq_packed* v_out, int64_t slot0,
+                    nq_stream_t stream) {
+  if (!K && !V) return fail(NQ_ERR_INVALID, "K and V are both NULL");
+  if (units < 0 || heads < 1 || heads > 1024 || n < 0 || slot0 < 0 || pos_base < 0)
+    return fail(NQ_ERR_INVALID, "need units >= 0, 1 <= heads <= 1024, n >= 0, slot0 >= 0, pos_base >= 0");
+  if (units == 0 || n == 0) return NQ_OK;
+  if (T_in < 1) return fail(NQ_ERR_INVALID, "T_in must be >= 1");
+  if (kept) {
+    if (!aligned(kept, 4)) return fail(NQ_ERR_INVALID, "kept misaligned");
+    if (kept_stride < n) return fail(NQ_ERR_INVALID, "kept_stride < n");
+  } else if (n > T_in) {
+    return fail(NQ_ERR_INVALID, "n > T_in without a kept list");
+  }
+  if (K) {
+    if (nq_status st = check_kv(K, ks, "K")) return st;
+    if (nq_status st = check_packed(k_out, "k_out")) return st;
+    if (nq_status st = check_rope(rope_tab, rope_max_pos)) return st;
+    if (!kept && pos_base + n > rope_max_pos)
+      return fail(NQ_ERR_INVALID, "positions up to %lld exceed rope_max_pos %lld",
+                  static_cast<long long>(pos_base + n - 1), static_cast<long long>(rope_max_pos));
+  }
+  if (V) {
+    if (nq_status st = check_kv(V, vs, "V")) return st;
+    if (nq_status st = check_packed(v_out, "v_out")) return st;
+  }
+  nq::EncodeLaunch L{};
+  L.K = K;
+  L.ks = ks;
+  L.V = V;
+  L.vs = vs;
+  L.units = units;
+  L.heads = heads;
+  L.T_in = T_in;
+  L.n = n;
+  L.kept = kept;
+  L.kept_stride = kept_stride;
+  L.pos_base = pos_base;
+  L.rope_tab = rope_tab;
+  L.rope_max_pos = rope_max_pos;
+  if (K) L.k_out = *k_out;
+  if (V) L.v_out = *v_out;
+  L.slot0 = slot0;
+  return cuda_status(nq::launch_encode(L, reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_encode launch");
+}
+
+nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int heads,
+                    int64_t n, int64_t slot0, const int32_t* positions, int64_t pos_stride,
+                    int64_t pos_base, const float* rope_tab, int64_t rope_max_pos, void* K_out,
+                    nq_kv_strides kos, void* V_out, nq_kv_strides vos, nq_stream_t stream) {
+  if (!K_out && !V_out) return fail(NQ_ERR_INVALID, "K_out and V_out are both NULL");
+  if (units < 0 || heads < 1 || heads > 1024 || n < 0 || slot0 < 0 || pos_base < 0)
+    return fail(NQ_ERR_INVALID, "need units >= 0, 1 <= heads <= 1024, n >= 0, slot0 >= 0, pos_base >= 0");
+  if (units == 0 || n == 0) return NQ_OK;
+  if (positions) {
+    if (!aligned(positions, 4)) return fail(NQ_ERR_INVALID, "positions misaligned");
+    if (pos_stride < n) return fail(NQ_ERR_INVALID, "pos_stride < n");
+  }
+  if (K_out) {
+    if (nq_status st = check_kv(K_out, kos, "K_out")) return st;
+    if (nq_status st = check_packed(k_in, "k_in")) return st;
+    if (nq_status st = check_rope(rope_tab, rope_max_pos)) return st;
+    if (!positions && pos_base + n > rope_max_pos)
+      return fail(NQ_ERR_INVALID, "positions up to %lld exceed rope_max_pos %lld",
+                  static_cast<long long>(pos_base + n - 1), static_cast<long long>(rope_max_pos));
+  }
+  if (V_out) {
+    if (nq_status st = check_kv(V_out, vos, "V_out")) return st;
+    if (nq_status st = check_packed(v_in, "v_in")) return st;
+  }
+  nq::DecodeLaunch L{};
+  if (K_out) L.k_in = *k_in;
+  if (V_out) L.v_in = *v_in;
+  L.units = units;
+  L.heads = heads;
+  L.n = n;
+  L.slot0 = slot0;
+  L.positions = positions;
+  L.pos_stride = pos_stride;
+  L.pos_base = pos_base;
+  L.rope_tab = rope_tab;
+  L.rope_max_pos = rope_max_pos;
+  L.K_out = K_out;
+  L.kos = kos;
+  L.V_out = V_out;
+  L.vos = vos;
+  return cuda_status(nq::launch_decode(L, reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_decode launch");
+}
+
+nq_status nq_device_error(uint32_t* flags_out) {
+  if (!flags_out) return fail(NQ_ERR_INVALID, "flags_out is NULL");
+  return cuda_status(nq::codec_read_clear_error(flags_out), "nq_device_error");
+}
+
+}  // extern "C"

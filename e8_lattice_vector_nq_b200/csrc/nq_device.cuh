@@ -1,0 +1,168 @@
+// nq_device.cuh -- device-side helpers shared by the libnq kernels (sm_100a):
+// bulk-copy (TMA, non-tensor) and mbarrier wrappers in inline PTX, bounded
+// waits, bf16 unpacking, packed fp32x2 arithmetic and the shared error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nq {
+
+constexpr int kD = 128;
+constexpr int kHalf = 64;
+constexpr int kRowPad = 272;  // smem bytes per staged 128 x bf16 row (256 + 16: conflict-free)
+constexpr int kTileSlots = 32;
+
+// fp32 constants of the scale rule: C = 1/sqrt(128), G_b = 1/(A_b sqrt(128))
+// with A_3 = 3.5, A_2 = 1.5, each the fp32 nearest to the real number.
+constexpr uint32_t kCBits = 0x3DB504F3u;
+constexpr uint32_t kG3Bits = 0x3CCEE116u;
+constexpr uint32_t kG2Bits = 0x3D715BEFu;
+constexpr float kMagicRound = 12582912.0f;  // 1.5 * 2^23: x + M - M = rint(x) for |x| < 2^22
+constexpr float kTwo23 = 8388608.0f;        // 2^23: bits(2^23 + j) = 0x4B000000 | j
+
+// Device error word of this translation unit: bit 0 = a bounded wait on a
+// bulk copy gave up.  Read and cleared through the ABI (nq_device_error).
+static __device__ unsigned int g_nq_error;
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; give up after about
+// one second, set the device error word and return false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > 1000000000ull) {
+      atomicOr(&g_nq_error, 1u);
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------- bulk async copies
+// global -> shared, completion counted on an mbarrier (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// shared -> global, tracked by this thread's bulk groups.
+__device__ __forceinline__ void bulk_s2g(void* gmem_dst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's committed bulk stores have finished READING smem.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until this thread's committed bulk stores are complete (globally visible).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Make this thread's generic-proxy smem writes visible to the async proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------- conversions
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float4 lds128f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// ----------------------------------------------------- packed fp32 pairs
+// IEEE round-to-nearest per lane (sm_100 f32x2 instructions).
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  // a - b == fma(b, -1, a): one rounding of the exact difference.
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// ------------------------------------------------------------- RoPE table
+// Combine the two-level table for position pos and frequency pair index i:
+// c = fmaf(cA, cB, -(sA*sB)), s = fmaf(sA, cB, cA*sB).
+__device__ __forceinline__ float2 rope_cs(const float2* __restrict__ tab, int64_t n_a, int64_t pos,
+                                          int i) {
+  int64_t a = pos >> 8;
+  a = a < 0 ? 0 : (a >= n_a ? n_a - 1 : a);  // out-of-contract positions stay in bounds
+  const int b = static_cast<int>(pos & 255);
+  const float2 A = __ldg(tab + a * kHalf + i);
+  const float2 B = __ldg(tab + (n_a + b) * kHalf + i);
+  const float ss = __fmul_rn(A.y, B.y);
+  const float cs = __fmul_rn(A.x, B.y);
+  return make_float2(__fmaf_rn(A.x, B.x, -ss), __fmaf_rn(A.y, B.x, cs));
+}
+
+}  // namespace nq

@@ -1,0 +1,247 @@
+// nq_evict.cu -- key-key proxy scoring and token selection for sm_100a.
+//
+// Method: NexusQuant ("NexusQuant: training-free 10-33x KV cache
+// compression", zingnex.cn, sections "Token eviction" and "Implementation
+// details": a fast key-key proxy score; always keep BOS and a recent sliding
+// window, drop the low scorers; "Como comprimir o KV cache...", dev.to,
+// "Como funciona", steps 1-2: rank tokens by a cross-head inner product).
+//
+//   window_mean_kernel: m[u][h][d] = fp32(fp64 sum of the last W keys / W)
+//   score_kernel:       scores[u][t] = sum_h sum_d K[u][h][t][d] * m[u][h][d]
+//                       in fp64 (one coalesced pass over K)
+//   select_kernel:      per unit, an 8-pass MSD radix select of the
+//                       (score desc, position asc) threshold on
+//                       order-preserving 64-bit keys, then an ordered
+//                       compaction with warp ballots.
+#include "nq_internal.h"
+
+namespace nq {
+
+// ----------------------------------------------------------- window mean
+__global__ void window_mean_kernel(const uint16_t* __restrict__ K, nq_kv_strides ks, int heads,
+                                   int64_t T, int W, float* __restrict__ mean) {
+  const int u = blockIdx.x / heads, h = blockIdx.x % heads, d = threadIdx.x;
+  const uint16_t* p = K + u * ks.unit + h * ks.head + d;
+  double S = 0.0;  // every partial sum of bf16 values is exact in fp64 here
+  for (int64_t t = T - W; t < T; ++t) S += static_cast<double>(bf16lo(__ldg(p + t * ks.token)));
+  mean[(static_cast<int64_t>(u) * heads + h) * kD + d] = static_cast<float>(S / W);
+}
+
+// ---------------------------------------------------------------- score
+constexpr int kScoreTok = 64;      // tokens per CTA
+constexpr int kScoreThreads = 256;
+
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __restrict__ K,
+                                                              nq_kv_strides ks, int heads,
+                                                              int64_t T,
+                                                              const float* __restrict__ mean,
+                                                              double* __restrict__ scores) {
+  extern __shared__ double part[];  // [heads][kScoreTok]
+  const int64_t tiles = (T + kScoreTok - 1) / kScoreTok;
+  const int u = static_cast<int>(blockIdx.x / tiles);
+  const int64_t t0 = (blockIdx.x % tiles) * kScoreTok;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4, chunk = lane & 15;
+  const int nwarps = kScoreThreads / 32;
+
+  for (int h = warp; h < heads; h += nwarps) {
+    const float* mh = mean + (static_cast<int64_t>(u) * heads + h) * kD + chunk * 8;
+    double m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = static_cast<double>(__ldg(mh + i));
+    const uint16_t* base = K + u * ks.unit + h * ks.head + chunk * 8;
+#pragma unroll 4
+    for (int it = 0; it < kScoreTok / 2; ++it) {
+      const int tl = 2 * it + half;
+      const int64_t t = t0 + tl;
+      double acc = 0.0;
+      if (t < T) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(base + t * ks.token));
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc = fma(static_cast<double>(bf16lo(w[k])), m[2 * k], acc);
+          acc = fma(static_cast<double>(bf16hi(w[k])), m[2 * k + 1], acc);
+        }
+      }
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (chunk == 0) part[h * kScoreTok + tl] = acc;
+    }
+  }
+  __syncthreads();
+  for (int tl = threadIdx.x; tl < kScoreTok; tl += blockDim.x) {
+    const int64_t t = t0 + tl;
+    if (t < T) {
+      double s = 0.0;
+      for (int h = 0; h < heads; ++h) s += part[h * kScoreTok + tl];
+      scores[static_cast<int64_t>(u) * T + t] = s;
+    }
+  }
+}
+
+// --------------------------------------------------------------- select
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+
+// Order-preserving map of a finite double to uint64 (larger score -> larger
+// key); -0 is folded onto +0 so that the two compare equal.
+__device__ __forceinline__ uint64_t score_key(double x) {
+  if (x == 0.0) x = 0.0;
+  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x));
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ void block_exclusive_scan32(int* vals /*[32] smem*/) {
+  // small serial scan by one thread: 32 warps
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+      const int c = vals[w];
+      vals[w] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __restrict__ scores,
+                                                             int64_t T, int W, int64_t n_kept,
+                                                             int32_t* __restrict__ kept,
+                                                             int64_t kept_stride) {
+  extern __shared__ uint32_t flagbits[];  // ceil(T/32) words
+  __shared__ unsigned int hist[256];
+  __shared__ uint64_t s_prefix;
+  __shared__ int64_t s_k;
+  __shared__ int warp_cnt[kSelWarps];
+
+  const int u = blockIdx.x;
+  const double* s = scores + static_cast<int64_t>(u) * T;
+  int32_t* out = kept + static_cast<int64_t>(u) * kept_stride;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (n_kept >= T) {
+    for (int64_t t = tid; t < T; t += blockDim.x) out[t] = static_cast<int32_t>(t);
+    return;
+  }
+  const int64_t lo = 1, hi = T - W;  // middle range [lo, hi)
+  const int64_t n_mid = n_kept - 1 - W;
+
+  // --- radix select: the n_mid-th largest key among the middle tokens
+  uint64_t prefix = 0, pmask = 0;
+  int64_t k = n_mid;
+  if (n_mid > 0) {
+    for (int pass = 0; pass < 8; ++pass) {
+      const int shift = 56 - 8 * pass;
+      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      for (int64_t t = lo + tid; t < hi; t += blockDim.x) {
+        const uint64_t key = score_key(__ldg(s + t));
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int64_t cum = 0;
+        int sel = 0;
+        for (int d = 255; d >= 0; --d) {
+          if (cum + hist[d] >= k) {
+            sel = d;
+            break;
+          }
+          cum += hist[d];
+        }
+        s_k = k - cum;
+        s_prefix = prefix | (static_cast<uint64_t>(sel) << shift);
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      k = s_k;
+      pmask |= 0xFFull << shift;
+      __syncthreads();
+    }
+  }
+  const uint64_t kstar = prefix;  // threshold key
+  const int64_t need_eq = k;      // how many keys equal to kstar are taken, lowest positions first
+
+  // --- ordered compaction: each warp owns a contiguous segment of positions
+  const int64_t seg = ((T + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
+  const int64_t s0 = warp * seg, s1 = min64(T, s0 + seg);
+
+  // pass A: keys equal to the threshold, per warp
+  int eq = 0;
+  if (n_mid > 0) {
+    for (int64_t b = s0; b < s1; b += 32) {
+      const int64_t t = b + lane;
+      const bool is_eq = (t < s1) && (t >= lo) && (t < hi) && score_key(__ldg(s + t)) == kstar;
+      eq += __popc(__ballot_sync(0xffffffffu, is_eq));
+    }
+  }
+  if (lane == 0) warp_cnt[warp] = eq;
+  __syncthreads();
+  block_exclusive_scan32(warp_cnt);
+  int64_t eq_rank = warp_cnt[warp];
+  __syncthreads();
+
+  // pass B: keep flags (bitmask in smem) and per-warp kept counts
+  int cnt = 0;
+  for (int64_t b = s0; b < s1; b += 32) {
+    const int64_t t = b + lane;
+    const bool in_range = t < s1;
+    const bool mid = in_range && t >= lo && t < hi;
+    const uint64_t key = mid ? score_key(__ldg(s + t)) : 0ull;
+    const bool is_eq = mid && n_mid > 0 && key == kstar;
+    const uint32_t eqb = __ballot_sync(0xffffffffu, is_eq);
+    const int64_t r = eq_rank + __popc(eqb & ((1u << lane) - 1u));
+    const bool keep =
+        in_range && (!mid || (n_mid > 0 && (key > kstar || (is_eq && r < need_eq))));
+    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+    eq_rank += __popc(eqb);
+    if (lane == 0) flagbits[b >> 5] = kb;
+    cnt += __popc(kb);
+  }
+  if (lane == 0) warp_cnt[warp] = cnt;
+  __syncthreads();
+  block_exclusive_scan32(warp_cnt);
+
+  // pass C: write kept positions in ascending order
+  int64_t o = warp_cnt[warp];
+  for (int64_t b = s0; b < s1; b += 32) {
+    const uint32_t kb = flagbits[b >> 5];
+    const int64_t idx = o + __popc(kb & ((1u << lane) - 1u));
+    if (((kb >> lane) & 1u) && idx < n_kept) out[idx] = static_cast<int32_t>(b + lane);
+    o += __popc(kb);
+  }
+}
+
+// ---------------------------------------------------------------- launch
+cudaError_t launch_score(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
+                         double* scores, float* mean_ws, cudaStream_t stream) {
+  window_mean_kernel<<<units * heads, kD, 0, stream>>>(static_cast<const uint16_t*>(K), ks, heads,
+                                                       T, W, mean_ws);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t tiles = (T + kScoreTok - 1) / kScoreTok;
+  const size_t smem = static_cast<size_t>(heads) * kScoreTok * sizeof(double);
+  if (smem > 48 * 1024) {
+    err = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+  }
+  score_kernel<<<static_cast<unsigned>(units * tiles), kScoreThreads, smem, stream>>>(
+      static_cast<const uint16_t*>(K), ks, heads, T, mean_ws, scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const double* scores, int units, int64_t T, int W, int evict_pct,
+                          int64_t n_kept, int32_t* kept, int64_t kept_stride,
+                          cudaStream_t stream) {
+  (void)evict_pct;
+  const size_t smem = static_cast<size_t>((T + 31) / 32 + kSelWarps) * sizeof(uint32_t);
+  cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  select_kernel<<<units, kSelThreads, smem, stream>>>(scores, T, W, n_kept, kept, kept_stride);
+  return cudaGetLastError();
+}
+
+}  // namespace nq

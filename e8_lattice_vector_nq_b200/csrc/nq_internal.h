@@ -1,0 +1,56 @@
+// nq_internal.h -- launch descriptors shared by the C ABI layer (nq_abi.cu)
+// and the kernel files.  Arguments are validated by the ABI layer before any
+// launcher below is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nq.h"
+#include "nq_device.cuh"
+
+namespace nq {
+
+struct EncodeLaunch {
+  const void* K;
+  nq_kv_strides ks;
+  const void* V;
+  nq_kv_strides vs;
+  int units, heads;
+  int64_t T_in, n;
+  const int32_t* kept;
+  int64_t kept_stride;
+  int64_t pos_base;
+  const float* rope_tab;
+  int64_t rope_max_pos;
+  nq_packed k_out, v_out;
+  int64_t slot0;
+};
+
+struct DecodeLaunch {
+  nq_packed k_in, v_in;
+  int units, heads;
+  int64_t n, slot0;
+  const int32_t* positions;
+  int64_t pos_stride;
+  int64_t pos_base;
+  const float* rope_tab;
+  int64_t rope_max_pos;
+  void* K_out;
+  nq_kv_strides kos;
+  void* V_out;
+  nq_kv_strides vos;
+};
+
+cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
+
+cudaError_t codec_read_clear_error(uint32_t* flags);
+
+cudaError_t launch_score(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
+                         double* scores, float* mean_ws, cudaStream_t stream);
+cudaError_t launch_select(const double* scores, int units, int64_t T, int W, int evict_pct,
+                          int64_t n_kept, int32_t* kept, int64_t kept_stride,
+                          cudaStream_t stream);
+
+}  // namespace nq

@@ -1,0 +1,290 @@
+"""Python binding of libnq (include/nq.h): argument marshalling only.
+
+Every step of the path runs in the CUDA library; this module turns torch
+tensors into pointers, strides and the current CUDA stream, and raises when a
+call returns a non-OK status.  There is no fallback: if libnq.so is missing
+or the device is not CUDA, the calls fail loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SO_PATH = os.path.join(HERE, "libnq.so")
+D = 128
+
+NQ_OK, NQ_ERR_INVALID, NQ_ERR_WORKSPACE, NQ_ERR_CUDA, NQ_ERR_UNSUPPORTED = range(5)
+
+
+class NQError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libnq status {status}: {msg}")
+        self.status = status
+
+
+class KVStrides(ctypes.Structure):
+    _fields_ = [("unit", ctypes.c_int64), ("head", ctypes.c_int64), ("token", ctypes.c_int64)]
+
+
+class Packed(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p),
+                ("unit_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64),
+                ("bits", ctypes.c_int32)]
+
+
+_lib = None
+
+EXPORTS = (
+    "nq_last_error", "nq_version", "nq_packed_bytes_per_vector", "nq_rope_tables_bytes",
+    "nq_rope_tables_fill_host", "nq_score_workspace_bytes", "nq_score", "nq_kept_count",
+    "nq_select", "nq_encode", "nq_decode", "nq_device_error",
+)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnq.so from the package directory (built by build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(SO_PATH):
+        raise ImportError(f"libnq.so not built at {SO_PATH}; run python -m e8_lattice_vector_nq_b200.build")
+    L = ctypes.CDLL(SO_PATH)
+    P, i64, i32, sz, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_double
+    PK = ctypes.POINTER(Packed)
+    sig = {
+        "nq_last_error": (ctypes.c_char_p, []),
+        "nq_version": (i32, []),
+        "nq_packed_bytes_per_vector": (i64, [i32]),
+        "nq_rope_tables_bytes": (sz, [i64]),
+        "nq_rope_tables_fill_host": (i32, [dbl, i64, P, sz]),
+        "nq_score_workspace_bytes": (sz, [i32, i32]),
+        "nq_score": (i32, [P, KVStrides, i32, i32, i64, i32, P, P, sz, P]),
+        "nq_kept_count": (i64, [i64, i64, i32]),
+        "nq_select": (i32, [P, i32, i64, i32, i32, P, i64, P]),
+        "nq_encode": (i32, [P, KVStrides, P, KVStrides, i32, i32, i64, i64, P, i64, i64, P, i64,
+                            PK, PK, i64, P]),
+        "nq_decode": (i32, [PK, PK, i32, i32, i64, i64, P, i64, i64, P, i64, P, KVStrides, P,
+                            KVStrides, P]),
+        "nq_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != NQ_OK:
+        raise NQError(status, lib().nq_last_error().decode())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libnq works on CUDA tensors only (no CPU path)")
+
+
+def kv_strides(t: torch.Tensor) -> KVStrides:
+    """Strides of a [units][heads][tokens][128] bf16 tensor (last dim contiguous)."""
+    if t.dim() != 4 or t.shape[-1] != D or t.stride(-1) != 1 or t.dtype != torch.bfloat16:
+        raise ValueError("expected bf16 [units, heads, tokens, 128] with a contiguous last dim")
+    return KVStrides(t.stride(0), t.stride(1), t.stride(2))
+
+
+# ------------------------------------------------------------ packed store
+@dataclass
+class PackedStore:
+    """Device arrays of one packed K or V store: codes [units][heads][cap][4*bits]
+    (uint32 words held in an int32 tensor) and meta [units][heads][cap]."""
+
+    codes: torch.Tensor
+    meta: torch.Tensor
+    bits: int
+
+    @classmethod
+    def empty(cls, units: int, heads: int, cap: int, bits: int, device="cuda") -> "PackedStore":
+        codes = torch.empty(units, heads, cap, 4 * bits, dtype=torch.int32, device=device)
+        meta = torch.empty(units, heads, cap, dtype=torch.int32, device=device)
+        return cls(codes, meta, bits)
+
+    def select_units(self, sl) -> "PackedStore":
+        return PackedStore(self.codes[sl], self.meta[sl], self.bits)
+
+    def desc(self) -> Packed:
+        assert self.codes.stride(1) == self.meta.stride(1) * 4 * self.bits
+        assert self.codes.stride(0) == self.meta.stride(0) * 4 * self.bits
+        return Packed(self.codes.data_ptr(), self.meta.data_ptr(), self.meta.stride(0),
+                      self.meta.stride(1), self.bits)
+
+    @property
+    def nbytes(self) -> int:
+        return self.codes.numel() * 4 + self.meta.numel() * 4
+
+
+# -------------------------------------------------------------- RoPE tables
+def rope_tables(theta: float, max_pos: int, device="cuda") -> torch.Tensor:
+    """Two-level fp32 cos/sin tables built on the host by the library, copied to the device."""
+    L = lib()
+    nbytes = L.nq_rope_tables_bytes(int(max_pos))
+    host = torch.empty(nbytes // 4, dtype=torch.float32)
+    _check(L.nq_rope_tables_fill_host(float(theta), int(max_pos), _ptr(host), nbytes))
+    return host.to(device)
+
+
+# --------------------------------------------------------------- the calls
+def kept_count(T: int, W: int, evict_pct: int) -> int:
+    return int(lib().nq_kept_count(int(T), int(W), int(evict_pct)))
+
+
+def score_workspace(units: int, heads: int, device="cuda") -> torch.Tensor:
+    n = lib().nq_score_workspace_bytes(int(units), int(heads))
+    return torch.empty(max(n, 16) // 4, dtype=torch.float32, device=device)
+
+
+def nq_score(K: torch.Tensor, W: int, scores: torch.Tensor | None = None,
+             ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """scores[u][t] (fp64) of K [units][heads][T][128] (see nq.h, nq_score)."""
+    _require_cuda(K)
+    units, heads, T, _ = K.shape
+    if scores is None:
+        scores = torch.empty(units, T, dtype=torch.float64, device=K.device)
+    if ws is None:
+        ws = score_workspace(units, heads, K.device)
+    assert scores.is_contiguous() and scores.dtype == torch.float64
+    _check(lib().nq_score(_ptr(K), kv_strides(K), units, heads, T, int(W), _ptr(scores), _ptr(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)))
+    return scores
+
+
+def nq_select(scores: torch.Tensor, W: int, evict_pct: int, kept: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """kept [units][n] int32 ascending positions (see nq.h, nq_select)."""
+    _require_cuda(scores)
+    units, T = scores.shape
+    n = kept_count(T, W, evict_pct)
+    if kept is None:
+        kept = torch.empty(units, n, dtype=torch.int32, device=scores.device)
+    assert kept.dtype == torch.int32 and kept.stride(1) == 1
+    _check(lib().nq_select(_ptr(scores), units, T, int(W), int(evict_pct), _ptr(kept),
+                           kept.stride(0), _stream(stream)))
+    return kept
+
+
+def nq_encode(K: torch.Tensor | None, V: torch.Tensor | None, k_out: PackedStore | None,
+              v_out: PackedStore | None, n: int, rope_tab: torch.Tensor | None = None,
+              rope_max_pos: int = 0, kept: torch.Tensor | None = None, pos_base: int = 0,
+              slot0: int = 0, stream=None):
+    """Encode n slots of every (unit, head) into the packed stores (see nq.h, nq_encode)."""
+    _require_cuda(K, V, kept, rope_tab)
+    ref = K if K is not None else V
+    units, heads, T_in, _ = ref.shape
+    kd = k_out.desc() if K is not None else None
+    vd = v_out.desc() if V is not None else None
+    ks = kv_strides(K) if K is not None else KVStrides(0, 0, 0)
+    vs = kv_strides(V) if V is not None else KVStrides(0, 0, 0)
+    if kept is not None:
+        assert kept.dtype == torch.int32 and kept.stride(-1) == 1
+    for st in (k_out if K is not None else None, v_out if V is not None else None):
+        if st is not None and (st.meta.shape[0] < units or st.meta.shape[1] < heads
+                               or st.meta.shape[2] < slot0 + n):
+            raise ValueError("packed store too small for units x heads x (slot0 + n)")
+    _check(lib().nq_encode(_ptr(K), ks, _ptr(V), vs, units, heads, T_in, int(n), _ptr(kept),
+                           kept.stride(0) if kept is not None else 0, int(pos_base),
+                           _ptr(rope_tab), int(rope_max_pos),
+                           ctypes.byref(kd) if kd is not None else None,
+                           ctypes.byref(vd) if vd is not None else None, int(slot0),
+                           _stream(stream)))
+
+
+def nq_decode(k_in: PackedStore | None, v_in: PackedStore | None, n: int,
+              K_out: torch.Tensor | None, V_out: torch.Tensor | None,
+              rope_tab: torch.Tensor | None = None, rope_max_pos: int = 0,
+              positions: torch.Tensor | None = None, pos_base: int = 0, slot0: int = 0,
+              stream=None):
+    """Decode n slots of every (unit, head) into bf16 outputs (see nq.h, nq_decode)."""
+    _require_cuda(K_out, V_out, positions, rope_tab)
+    ref = K_out if K_out is not None else V_out
+    units, heads = ref.shape[0], ref.shape[1]
+    kd = k_in.desc() if K_out is not None else None
+    vd = v_in.desc() if V_out is not None else None
+    kos = kv_strides(K_out) if K_out is not None else KVStrides(0, 0, 0)
+    vos = kv_strides(V_out) if V_out is not None else KVStrides(0, 0, 0)
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.stride(-1) == 1
+    for st in (k_in if K_out is not None else None, v_in if V_out is not None else None):
+        if st is not None and (st.meta.shape[0] < units or st.meta.shape[1] < heads
+                               or st.meta.shape[2] < slot0 + n):
+            raise ValueError("packed store too small for units x heads x (slot0 + n)")
+    for o in (K_out, V_out):
+        if o is not None and o.shape[2] < n:
+            raise ValueError("output has fewer than n tokens")
+    _check(lib().nq_decode(ctypes.byref(kd) if kd is not None else None,
+                           ctypes.byref(vd) if vd is not None else None, units, heads, int(n),
+                           int(slot0), _ptr(positions),
+                           positions.stride(0) if positions is not None else 0, int(pos_base),
+                           _ptr(rope_tab), int(rope_max_pos), _ptr(K_out), kos, _ptr(V_out),
+                           vos, _stream(stream)))
+
+
+def device_error() -> int:
+    v = ctypes.c_uint32(0)
+    _check(lib().nq_device_error(ctypes.byref(v)))
+    return int(v.value)
+
+
+# ------------------------------------------------------- whole-cache helper
+class Codec:
+    """One layer-batched compression pass (score -> select -> encode) and its
+    inverse, all through the C ABI.  Buffers are allocated once per shape."""
+
+    def __init__(self, units: int, heads: int, T: int, theta: float, bits_k: int = 3,
+                 bits_v: int = 2, window: int = 64, evict_pct: int = 0, device="cuda",
+                 max_pos: int | None = None):
+        self.units, self.heads, self.T = units, heads, T
+        self.W, self.pct = window, evict_pct
+        self.bits_k, self.bits_v = bits_k, bits_v
+        self.evict = evict_pct > 0 and T > 1 + window
+        self.n = kept_count(T, window, evict_pct) if self.evict else T
+        self.max_pos = max_pos or T
+        self.rope = rope_tables(theta, self.max_pos, device)
+        self.k_store = PackedStore.empty(units, heads, self.n, bits_k, device)
+        self.v_store = PackedStore.empty(units, heads, self.n, bits_v, device)
+        if self.evict:
+            self.scores = torch.empty(units, T, dtype=torch.float64, device=device)
+            self.ws = score_workspace(units, heads, device)
+            self.kept = torch.empty(units, self.n, dtype=torch.int32, device=device)
+        else:
+            self.kept = None
+
+    def encode(self, K: torch.Tensor, V: torch.Tensor, stream=None):
+        if self.evict:
+            nq_score(K, self.W, self.scores, self.ws, stream)
+            nq_select(self.scores, self.W, self.pct, self.kept, stream)
+        nq_encode(K, V, self.k_store, self.v_store, self.n, self.rope, self.max_pos,
+                  kept=self.kept, stream=stream)
+
+    def decode(self, K_out: torch.Tensor, V_out: torch.Tensor, stream=None):
+        nq_decode(self.k_store, self.v_store, self.n, K_out, V_out, self.rope, self.max_pos,
+                  positions=self.kept, stream=stream)
+
+    @property
+    def packed_bytes(self) -> int:
+        b = self.k_store.nbytes + self.v_store.nbytes
+        if self.kept is not None:
+            b += self.kept.numel() * 4
+        return b

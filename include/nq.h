@@ -1,0 +1,192 @@
+/*
+ * nq.h -- C ABI of libnq: B200 (sm_100a) kernels for training-free KV-cache
+ * compression by token eviction plus E8 lattice vector quantisation.
+ *
+ * The method follows two descriptions of NexusQuant:
+ *   [NQ-zh]  "NexusQuant: training-free 10-33x KV cache compression"
+ *            (zingnex.cn), sections "Token eviction", "E8 lattice
+ *            quantisation", "Implementation details";
+ *   [NQ-pt]  "Como comprimir o KV cache do seu LLM em 33x sem treino"
+ *            (dev.to), section "Como funciona (em 6 passos)", steps 1-5.
+ * The pages give no formulas or code; the concrete arithmetic below (fp32
+ * operation order, tie rules, scale rule, packed layout) is this library's
+ * reading and is restated next to each call.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every tensor pointer is a DEVICE pointer that the caller allocates and
+ *   owns; the library never allocates, frees or retains memory, except
+ *   nq_rope_tables_fill_host, which writes a caller-owned HOST buffer.
+ * - Every compute call is asynchronous on the caller's CUDA stream and
+ *   returns as soon as its kernels are queued.  Nothing synchronises.
+ * - Return value: nq_status.  NQ_ERR_INVALID for bad arguments (checked on the
+ *   host before anything is launched; nothing is launched then),
+ *   NQ_ERR_WORKSPACE for a workspace smaller than required, NQ_ERR_CUDA when a
+ *   launch reports an error.  nq_last_error() gives a message for the calling
+ *   thread.  No C++ exception, exit() or device trap crosses the ABI.
+ * - A KV tensor (bf16) holds, for each (unit, head, token), one vector of 128
+ *   contiguous bf16 coordinates.  Its three strides are in ELEMENTS and must
+ *   be multiples of 8, and the base pointer 16-byte aligned (16-byte vector
+ *   loads).  A "unit" is one layer of one sequence.
+ * - Inputs must be finite with |x| <= 2^32; other values are out of
+ *   contract (no fault: the kernels stay within their buffers, the codes of
+ *   such a vector are unspecified).
+ * - Kernels with bounded waits (mbarrier completion of bulk copies) give up
+ *   after about one second and set a device error word that
+ *   nq_device_error() reads; they never spin forever.
+ */
+#ifndef NQ_H
+#define NQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nq_stream_t; /* = cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    NQ_OK = 0,
+    NQ_ERR_INVALID = 1,
+    NQ_ERR_WORKSPACE = 2,
+    NQ_ERR_CUDA = 3,
+    NQ_ERR_UNSUPPORTED = 4
+} nq_status;
+
+#define NQ_HEAD_DIM 128
+
+/* Strides, in bf16 elements, of a [units][heads][tokens][128] KV tensor. */
+typedef struct {
+    int64_t unit;
+    int64_t head;
+    int64_t token;
+} nq_kv_strides;
+
+/* A packed store of E8 codes for one of K or V.
+ *   codes: uint32 words, 4*bits words per vector.  The b-bit code of
+ *          coordinate c (0..127) of a vector sits at bits [b*c, b*c + b) of
+ *          the vector's little-endian stream of words (b = 3: 12 words,
+ *          b = 2: 8 words).
+ *   meta:  one uint32 per vector: bits 0..15 = coset mask (bit g set when
+ *          group g, coordinates 8g..8g+7, lies in the half-integer coset
+ *          D8 + 1/2), bits 16..31 = the vector's fp16 scale sigma.
+ *   Vector (unit u, head h, slot i) is at index u*unit_stride + h*head_stride
+ *   + i (in vectors) of both arrays.  16-byte aligned codes pointer. */
+typedef struct {
+    uint32_t *codes;
+    uint32_t *meta;
+    int64_t unit_stride;
+    int64_t head_stride;
+    int32_t bits; /* 2 or 3 */
+} nq_packed;
+
+/* Thread-local message for the last non-OK status (never NULL). */
+const char *nq_last_error(void);
+
+/* ABI version, bumped on incompatible changes. */
+int nq_version(void);
+
+/* Bytes of raw packed storage per vector: 4*(4*bits) + 4 (52 for K3, 36 for V2). */
+int64_t nq_packed_bytes_per_vector(int bits);
+
+/* ----------------------------------------------------------- RoPE tables
+ * Split-half rotary embedding ([NQ-zh] "Supported models": split-half RoPE
+ * only; interleaved RoPE is not supported), pairs (i, i+64), frequencies
+ * w_i = theta^(-i/64).  For position p = 256a + b the tables hold fp32
+ * roundings of fp64 cos/sin:
+ *   A[a][i] = (cos(256a*w_i), sin(256a*w_i)),  a < ceil(max_pos/256)
+ *   B[b][i] = (cos(b*w_i),    sin(b*w_i)),     b < 256
+ * as float2 pairs, A first then B.  The kernels combine them in fp32:
+ *   c = fmaf(cA, cB, -(sA*sB)),  s = fmaf(sA, cB, cA*sB).
+ * The caller copies the filled host buffer to device memory once per theta
+ * and passes that device pointer with the same max_pos. */
+size_t nq_rope_tables_bytes(int64_t max_pos);
+nq_status nq_rope_tables_fill_host(double theta, int64_t max_pos, void *host_buf, size_t bytes);
+
+/* ----------------------------------------------------------------- score
+ * Key-key proxy importance ([NQ-zh] "Implementation details": fast key-key
+ * proxy; [NQ-pt] step 1: cross-head inner product), on the stored, rotated
+ * keys:
+ *   m[u][h][d]   = fp32( (sum over t in [T-W, T) of K[u][h][t][d], fp64) / W )
+ *   scores[u][t] = sum over h, d of (double)K[u][h][t][d] * (double)m[u][h][d]
+ * (fp64 accumulation; products are exact, summation order is the kernel's).
+ * K: bf16 [units][heads][T][128] with strides ks.  scores: fp64
+ * [units][T], row-contiguous.  ws: device workspace of at least
+ * nq_score_workspace_bytes(units, heads) bytes (holds m).  1 <= W <= T. */
+size_t nq_score_workspace_bytes(int units, int heads);
+nq_status nq_score(const void *K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
+                   double *scores, void *ws, size_t ws_bytes, nq_stream_t stream);
+
+/* ---------------------------------------------------------------- select
+ * Token eviction ([NQ-zh] "Token eviction": always keep BOS and a recent
+ * sliding window, drop the low scorers; [NQ-pt] step 2).  Per unit:
+ *   mid = T - 1 - W, n_evict = floor(mid * evict_pct / 100),
+ *   kept = {0} u top (mid - n_evict) of positions [1, T-W) by
+ *          (score descending, position ascending) u [T-W, T),
+ * written in ascending order to kept[u*kept_stride + 0 .. n-1], n =
+ * nq_kept_count(T, W, evict_pct) (every unit keeps the same count).
+ * T <= 1 + W or evict_pct == 0 keeps everything.  scores: fp64 [units][T]
+ * row-contiguous (as written by nq_score); kept_stride >= n. */
+int64_t nq_kept_count(int64_t T, int64_t W, int evict_pct);
+nq_status nq_select(const double *scores, int units, int64_t T, int W, int evict_pct,
+                    int32_t *kept, int64_t kept_stride, nq_stream_t stream);
+
+/* ---------------------------------------------------------------- encode
+ * RoPE removal, Hadamard rotation and E8 quantisation ([NQ-zh] "E8 lattice
+ * quantisation", "Implementation details"; [NQ-pt] steps 3-5).  For slot i
+ * (0 <= i < n) of every (unit u, head h):
+ *   src = kept ? kept[u*kept_stride + i] : i      (input token, < T_in)
+ *   pos = pos_base + src                          (RoPE position)
+ *   keys:   v = RoPE^-1(K[u][h][src]) at pos:
+ *             v_i    = fmaf(k_i,    c, k_{i+64}*s)
+ *             v_i+64 = fmaf(k_i+64, c, -(k_i*s))
+ *   values: v = V[u][h][src]
+ *   v <- unnormalised Walsh-Hadamard (Sylvester order, stages 1, 2, ..., 64,
+ *        butterfly (a, b) -> (a+b, a-b), fp32)
+ *   sigma = fp16(min(fp32(max|v| * G_b), 65504)), G_b = fp32(1/(A_b*sqrt(128))),
+ *           A_3 = 3.5, A_2 = 1.5;  r = fp32(C/sigma) (0 if sigma == 0),
+ *           C = fp32(1/sqrt(128));  y = fp32(v * r)
+ *   each group of 8 coordinates of y -> nearest E8 point (Conway-Sloane:
+ *           decode D8 and D8 + 1/2 in fp32 -- round to nearest even, fix an
+ *           odd sum on the first largest-error coordinate, fp32 squared
+ *           distance, ties to the integer coset)
+ *   2q clamped to the b-bit symmetric range (half coset |2q| <= 2^b-1,
+ *           integer coset |2q| <= 2^b-2), code = (2q + lim)/2,
+ *   written to slot slot0 + i of k_out / v_out.
+ * K and/or V may be NULL (then its k_out/v_out is ignored).  bits: K and V
+ * may differ (K3V2).  rope_tab: device tables from nq_rope_tables_fill_host
+ * (required when K != NULL), positions must be < rope_max_pos. */
+nq_status nq_encode(const void *K, nq_kv_strides ks, const void *V, nq_kv_strides vs, int units,
+                    int heads, int64_t T_in, int64_t n, const int32_t *kept, int64_t kept_stride,
+                    int64_t pos_base, const float *rope_tab, int64_t rope_max_pos,
+                    const nq_packed *k_out, const nq_packed *v_out, int64_t slot0,
+                    nq_stream_t stream);
+
+/* ---------------------------------------------------------------- decode
+ * Inverse path: for slot slot0 + i (0 <= i < n) of every (unit, head):
+ *   t_c   = 2 j_c - 2^b + 2 - h_g       (= 2q, h_g the group's coset bit)
+ *   w     = Walsh-Hadamard(t)           (integers, exact in fp32)
+ *   x_c   = fp32(w_c * kappa),  kappa = fp32(fp32(sigma/2) * C)
+ *   keys: re-apply RoPE at pos = pos_base + (positions ?
+ *         positions[u*pos_stride + i] : i) ([NQ-zh] "Implementation
+ *         details": RoPE restored after quantisation):
+ *           o_i = fmaf(x_i, c, -(x_{i+64}*s)),  o_i+64 = fmaf(x_i+64, c, x_i*s)
+ *   bf16 round-to-nearest-even into K_out/V_out[u][h][i] (strides kos/vos).
+ * k_in/v_in may be NULL (that output is skipped). */
+nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int heads,
+                    int64_t n, int64_t slot0, const int32_t *positions, int64_t pos_stride,
+                    int64_t pos_base, const float *rope_tab, int64_t rope_max_pos, void *K_out,
+                    nq_kv_strides kos, void *V_out, nq_kv_strides vos, nq_stream_t stream);
+
+/* -------------------------------------------------------------- status
+ * Reads and clears the device error word that kernels set when a bounded
+ * wait gave up (bit 0: bulk-copy completion timed out).  Synchronises the
+ * current device.  Returns NQ_ERR_CUDA if the read itself failed. */
+nq_status nq_device_error(uint32_t *flags_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NQ_H */

@@ -449,7 +449,7 @@ int64_t oq_encode_unit(const uint16_t *K, const uint16_t *V, int H, int64_t T_in
 }
 
 /* Decode n slots of one unit into K_out/V_out [H][n][128] bf16; slot i is at
- * RoPE position positions ? positions[i] : pos_base + i. */
+ * RoPE position pos_base + (positions ? positions[i] : i). */
 void oq_decode_unit(const uint32_t *k_codes, const uint32_t *k_meta, const uint32_t *v_codes,
                     const uint32_t *v_meta, int H, int64_t n, const int32_t *positions,
                     int64_t pos_base, double theta, int bits_k, int bits_v, uint16_t *K_out,
@@ -457,7 +457,7 @@ void oq_decode_unit(const uint32_t *k_codes, const uint32_t *k_meta, const uint3
 {
     float c[OQ_HALF], s[OQ_HALF];
     for (int64_t i = 0; i < n; i++) {
-        int64_t pos = positions ? (int64_t)positions[i] : pos_base + i;
+        int64_t pos = pos_base + (positions ? (int64_t)positions[i] : i);
         if (K_out) oq_rope_cs(theta, pos, c, s);
         for (int h = 0; h < H; h++) {
             size_t vec = (size_t)h * n + (size_t)i;
