@@ -268,16 +268,17 @@ template <int BITS, bool ROPE>
 __device__ __forceinline__ void decode_vector(const uint32_t (&w)[4 * BITS], uint32_t meta,
                                               uint32_t cs_addr, uint32_t out_addr) {
   float2 v[64];
-  constexpr float kBase = -16777216.0f - static_cast<float>((1 << BITS) - 2);  // -2^24 - (2^b - 2)
+  // x = 2^22 + j (the fp32 spacing at 2^22 is 1/2, so the mantissa holds 2j);
+  // t = 2x - 2^23 - (2^b - 2) - h, every constant below 2^24: exact.
+  constexpr float kBase = -8388608.0f - static_cast<float>((1 << BITS) - 2);
 #pragma unroll
   for (int g = 0; g < 16; ++g) {
     const float kg = kBase - static_cast<float>((meta >> g) & 1u);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int c = 8 * g + 2 * k;
-      const float x0 = __uint_as_float(0x4B000000u | code_at<BITS>(w, c));
-      const float x1 = __uint_as_float(0x4B000000u | code_at<BITS>(w, c + 1));
-      // t = 2 (2^23 + j) - 2^24 - (2^b - 2) - h  (exact small integer)
+      const float x0 = __uint_as_float(0x4A800000u | (code_at<BITS>(w, c) << 1));
+      const float x1 = __uint_as_float(0x4A800000u | (code_at<BITS>(w, c + 1) << 1));
       v[4 * g + k] = fma2(make_float2(x0, x1), make_float2(2.0f, 2.0f), make_float2(kg, kg));
     }
   }
