@@ -129,6 +129,26 @@ nq_status nq_score(const void* K, nq_kv_strides ks, int units, int heads, int64_
                      "nq_score launch");
 }
 
+nq_status nq_score_static(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
+                          double* scores, nq_stream_t stream) {
+  if (units < 0 || heads < 1 || heads > 256)
+    return fail(NQ_ERR_INVALID, "need units >= 0 and 1 <= heads <= 256");
+  if (T < 1 || W < 1 || W > T) return fail(NQ_ERR_INVALID, "need 1 <= W <= T");
+  if (static_cast<int64_t>(units) * heads > NQ_SCORE_STATIC_MAX_VECTORS)
+    return fail(NQ_ERR_UNSUPPORTED,
+                "nq_score_static: units * heads = %lld exceeds its fixed scratch of %d "
+                "(unit, head) window means; use nq_score with a caller workspace",
+                static_cast<long long>(units) * heads, NQ_SCORE_STATIC_MAX_VECTORS);
+  if (units == 0) return NQ_OK;
+  if (nq_status st = check_kv(K, ks, "K")) return st;
+  if (!scores || !aligned(scores, 8)) return fail(NQ_ERR_INVALID, "scores NULL or misaligned");
+  if (static_cast<int64_t>(units) * ((T + 63) / 64) > 0x7FFFFFFF)
+    return fail(NQ_ERR_UNSUPPORTED, "units * T too large for one launch");
+  return cuda_status(nq::launch_score_static(K, ks, units, heads, T, W, scores,
+                                             reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_score_static");
+}
+
 int64_t nq_kept_count(int64_t T, int64_t W, int evict_pct) {
   if (T < 0 || W < 0) return -1;
   if (T <= 1 + W || evict_pct <= 0) return T;

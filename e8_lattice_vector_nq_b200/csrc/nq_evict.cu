@@ -13,6 +13,8 @@
 //                       (score desc, position asc) threshold on
 //                       order-preserving 64-bit keys, then an ordered
 //                       compaction with warp ballots.
+#include <mutex>
+
 #include "nq_internal.h"
 
 namespace nq {
@@ -230,6 +232,48 @@ cudaError_t launch_score(const void* K, nq_kv_strides ks, int units, int heads, 
   score_kernel<<<static_cast<unsigned>(units * tiles), kScoreThreads, smem, stream>>>(
       static_cast<const uint16_t*>(K), ks, heads, T, mean_ws, scores);
   return cudaGetLastError();
+}
+
+// ------------------------------------------ score without any allocation
+// Scratch for the window means of nq_score_static: a fixed array in the
+// library's own device memory, present on every GPU that loads the library
+// until the process exits.  All calls share it and it keeps the last call's
+// contents; the window-mean kernel overwrites every entry a call reads, so
+// nothing has to be cleared.  Two calls whose kernels overlap on a GPU race
+// on it.
+static __device__ __align__(256) float g_score_scratch[NQ_SCORE_STATIC_MAX_VECTORS * kD];
+
+namespace {
+constexpr int kMaxDevices = 256;
+std::mutex g_scratch_mu;
+float* g_scratch_addr[kMaxDevices] = {};
+}  // namespace
+
+// Device address of g_score_scratch on the current device.  Host code only
+// sees a host-side stand-in under the array's name, so the address is looked
+// up once per device, with that device current, and cached.
+static cudaError_t score_scratch_address(float** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_score_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_score_static(const void* K, nq_kv_strides ks, int units, int heads, int64_t T,
+                                int W, double* scores, cudaStream_t stream) {
+  float* mean = nullptr;
+  cudaError_t err = score_scratch_address(&mean);
+  if (err != cudaSuccess) return err;
+  return launch_score(K, ks, units, heads, T, W, scores, mean, stream);
 }
 
 cudaError_t launch_select(const double* scores, int units, int64_t T, int W, int evict_pct,

@@ -49,6 +49,8 @@ cudaError_t codec_read_clear_error(uint32_t* flags);
 
 cudaError_t launch_score(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
                          double* scores, float* mean_ws, cudaStream_t stream);
+cudaError_t launch_score_static(const void* K, nq_kv_strides ks, int units, int heads, int64_t T,
+                                int W, double* scores, cudaStream_t stream);
 cudaError_t launch_select(const double* scores, int units, int64_t T, int W, int evict_pct,
                           int64_t n_kept, int32_t* kept, int64_t kept_stride,
                           cudaStream_t stream);

@@ -40,7 +40,8 @@ _lib = None
 
 EXPORTS = (
     "nq_last_error", "nq_version", "nq_packed_bytes_per_vector", "nq_rope_tables_bytes",
-    "nq_rope_tables_fill_host", "nq_score_workspace_bytes", "nq_score", "nq_kept_count",
+    "nq_rope_tables_fill_host", "nq_score_workspace_bytes", "nq_score", "nq_score_static",
+    "nq_kept_count",
     "nq_select", "nq_encode", "nq_decode", "nq_device_error",
 )
 
@@ -63,6 +64,7 @@ def lib() -> ctypes.CDLL:
         "nq_rope_tables_fill_host": (i32, [dbl, i64, P, sz]),
         "nq_score_workspace_bytes": (sz, [i32, i32]),
         "nq_score": (i32, [P, KVStrides, i32, i32, i64, i32, P, P, sz, P]),
+        "nq_score_static": (i32, [P, KVStrides, i32, i32, i64, i32, P, P]),
         "nq_kept_count": (i64, [i64, i64, i32]),
         "nq_select": (i32, [P, i32, i64, i32, i32, P, i64, P]),
         "nq_encode": (i32, [P, KVStrides, P, KVStrides, i32, i32, i64, i64, P, i64, i64, P, i64,
@@ -168,6 +170,21 @@ def nq_score(K: torch.Tensor, W: int, scores: torch.Tensor | None = None,
     assert scores.is_contiguous() and scores.dtype == torch.float64
     _check(lib().nq_score(_ptr(K), kv_strides(K), units, heads, T, int(W), _ptr(scores), _ptr(ws),
                           ws.numel() * ws.element_size(), _stream(stream)))
+    return scores
+
+
+def nq_score_static(K: torch.Tensor, W: int, scores: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Same scores as nq_score without a caller workspace: for callers that
+    cannot allocate device memory (see nq.h, nq_score_static).  Calls that
+    overlap on one GPU race on the library's shared scratch."""
+    _require_cuda(K)
+    units, heads, T, _ = K.shape
+    if scores is None:
+        scores = torch.empty(units, T, dtype=torch.float64, device=K.device)
+    assert scores.is_contiguous() and scores.dtype == torch.float64
+    _check(lib().nq_score_static(_ptr(K), kv_strides(K), units, heads, T, int(W), _ptr(scores),
+                                 _stream(stream)))
     return scores
 
 

@@ -119,6 +119,33 @@ size_t nq_score_workspace_bytes(int units, int heads);
 nq_status nq_score(const void *K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
                    double *scores, void *ws, size_t ws_bytes, nq_stream_t stream);
 
+/* ------------------------------------------- score with no allocation
+ * This entry point has no counterpart in the method description; it exists
+ * for callers of this library that cannot allocate device memory: code
+ * embedded in a host framework that owns every byte of the GPU (a serving
+ * engine whose memory planner reserved all of HBM for its KV pool up front),
+ * or a latency-critical loop where a cudaMalloc/cudaFree would block or
+ * synchronise the device.  Such callers cannot provide nq_score's workspace.
+ *
+ * nq_score_static computes exactly what nq_score computes, with the same
+ * arguments minus the workspace.  The window means live instead in a fixed
+ * array inside the library's own device memory, sized for at most
+ * NQ_SCORE_STATIC_MAX_VECTORS (unit, head) pairs (1 MiB); every GPU that
+ * loads the library holds that array until the process exits.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   - units * heads above the maximum: NQ_ERR_UNSUPPORTED, nothing launched.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture.
+ *   - All calls share the array and it keeps the last call's contents (each
+ *     call overwrites every entry it reads, so nothing needs clearing).
+ *     Calls whose kernels overlap on the same GPU (different streams, or
+ *     different host threads) race on it and give undefined scores:
+ *     serialise them. */
+#define NQ_SCORE_STATIC_MAX_VECTORS 2048
+nq_status nq_score_static(const void *K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
+                          double *scores, nq_stream_t stream);
+
 /* ---------------------------------------------------------------- select
  * Token eviction ([NQ-zh] "Token eviction": always keep BOS and a recent
  * sliding window, drop the low scorers; [NQ-pt] step 2).  Per unit:
