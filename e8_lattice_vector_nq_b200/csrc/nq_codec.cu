@@ -9,38 +9,39 @@
 // point (Conway-Sloane, D8 u D8+1/2), clamp to b-bit codes and pack; decode
 // inverts the chain and writes bf16.
 //
-// Design (B200): one thread owns one 128-coordinate vector in registers
-// (64 packed fp32 pairs), so the Hadamard butterflies, the RoPE pairs
-// (i, i+64) and the 8-coordinate E8 groups need no shuffles.  A persistent
-// CTA of HG warps walks tiles of 32 slots x HG heads; every thread stages its
-// own 256-byte row with a bulk async copy (TMA engine, mbarrier completion)
-// into a padded shared-memory row, double buffered, so that HBM reads of the
-// next tiles overlap the arithmetic of the current one.  The per-position
-// RoPE (cos, sin) pairs of a tile are combined once per CTA and shared by the
-// HG heads.  Decode writes each reconstructed row to shared memory and
-// stores it with a bulk async copy.
+// Design (B200).  Two threads own one 128-coordinate vector: half h holds
+// the coordinate pairs (i, i+64) for i in [32h, 32h+32) as packed fp32x2
+// registers.  With that layout the RoPE pairs, the Hadamard stages 1..16 and
+// 64, and the E8 groups all stay inside a thread; only Hadamard stage 32
+// crosses to the partner lane (lane ^ 16, one shuffle per coordinate).  The
+// two lanes of an fp32x2 register hold groups g and g+8, so the E8 search
+// runs two groups per packed instruction (__fadd2_rn / __ffma2_rn /
+// __fmul2_rn: per-lane IEEE round-to-nearest, the same bits as scalar code).
+// A persistent CTA of HG warps (HG heads) walks tiles of 16 slots x HG heads.
+// Encode stages every input row with a 256-byte bulk async copy (TMA engine,
+// mbarrier completion) into a padded shared-memory row, double buffered, so
+// the loads of tile k+2 overlap the arithmetic of tile k; the RoPE (cos, sin)
+// pairs of a tile are combined once per CTA and shared by its heads.  Decode
+// loads the next tile's codes one tile ahead and writes each reconstructed
+// row through shared memory with a 256-byte bulk async store.  Every
+// (bits, RoPE) variant is its own kernel: keys and values are two launches.
 #include "nq_internal.h"
 
 namespace nq {
 
-// ------------------------------------------------------------- tile map
-struct KindParams {
-  const uint16_t* src;   // encode: bf16 input; decode: bf16 output (as uint16_t*)
-  int64_t su, sh, st;    // element strides of the bf16 tensor
-  uint32_t* codes;
-  uint32_t* meta;
-  int64_t pu, ph;        // vector strides of the packed store
-  int bits;
-  int rope;
-};
+constexpr int kSlots = 16;                  // slots per tile: one warp = 16 slots x 2 halves
+constexpr int kCsBytes = 32 * kSlots * 16;  // float4 cs[32][16]
 
 struct CodecArgs {
-  KindParams kind[2];
-  int nkinds;
+  const uint16_t* kv;  // encode: bf16 input; decode: bf16 output
+  int64_t su, sh, st;  // element strides of the bf16 tensor
+  uint32_t* codes;
+  uint32_t* meta;
+  int64_t pu, ph;      // vector strides of the packed store
   int heads, hg, ngroups;
-  int64_t T_in;          // encode: input tokens per (unit, head)
+  int64_t T_in;        // encode: input tokens per (unit, head)
   int64_t n, slot0, pos_base;
-  const int32_t* idx;    // encode: kept (source tokens); decode: positions
+  const int32_t* idx;  // encode: kept (source tokens); decode: positions
   int64_t idx_stride;
   const float2* tab;
   int64_t n_a;
@@ -48,14 +49,12 @@ struct CodecArgs {
 };
 
 struct Tile {
-  int kind, group, unit;
+  int group, unit;
   int64_t stile;
 };
 
 __device__ __forceinline__ Tile tile_of(const CodecArgs& a, int64_t t) {
   Tile r;
-  r.kind = static_cast<int>(t % a.nkinds);
-  t /= a.nkinds;
   r.group = static_cast<int>(t % a.ngroups);
   t /= a.ngroups;
   r.stile = t % a.slot_tiles;
@@ -63,263 +62,234 @@ __device__ __forceinline__ Tile tile_of(const CodecArgs& a, int64_t t) {
   return r;
 }
 
-// cs table of one tile in shared memory: float4 cs[32 pair-pairs][32 slots],
-// entry (j, slot) = (c_2j, c_2j+1, s_2j, s_2j+1) at that slot's position.
-constexpr int kCsBytes = 32 * kTileSlots * 16;
-
-__device__ __forceinline__ void fill_cs(const CodecArgs& a, const Tile& tl, bool use_idx,
-                                        float4* cs, int tid, int nthreads) {
-  for (int e = tid; e < 32 * kTileSlots; e += nthreads) {
-    const int slot_l = e % kTileSlots;
-    const int j = e / kTileSlots;
-    const int64_t slot = tl.stile * kTileSlots + slot_l;
-    float4 v = make_float4(1.f, 1.f, 0.f, 0.f);
+// cs table of one tile: float4 cs[j][slot] = (c_2j, s_2j, c_2j+1, s_2j+1) at
+// that slot's RoPE position; a thread of half h reads j in [16h, 16h+16).
+__device__ __forceinline__ void fill_cs(const CodecArgs& a, const Tile& tl, float4* cs, int tid,
+                                        int nthreads) {
+  for (int e = tid; e < 32 * kSlots; e += nthreads) {
+    const int slot_l = e % kSlots;
+    const int j = e / kSlots;
+    const int64_t slot = tl.stile * kSlots + slot_l;
+    float4 v = make_float4(1.f, 0.f, 1.f, 0.f);
     if (slot < a.n) {
       int64_t p = slot;
-      if (use_idx && a.idx) p = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot);
+      if (a.idx) p = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot);
       p += a.pos_base;
       const float2 c0 = rope_cs(a.tab, a.n_a, p, 2 * j);
       const float2 c1 = rope_cs(a.tab, a.n_a, p, 2 * j + 1);
-      v = make_float4(c0.x, c1.x, c0.y, c1.y);
+      v = make_float4(c0.x, c0.y, c1.x, c1.y);
     }
-    cs[j * kTileSlots + slot_l] = v;
+    cs[j * kSlots + slot_l] = v;
   }
 }
 
-// --------------------------------------------------------- Hadamard (fp32)
-// Unnormalised Sylvester transform on 128 coordinates held as 64 pairs
-// v[j] = (x_2j, x_2j+1); stage order h = 1, 2, ..., 64 as in the reference
-// definition.  Every output is the IEEE fp32 sum / difference of the same
-// two operands as in the scalar butterfly network.
-__device__ __forceinline__ void fwht128(float2 (&v)[64]) {
+// ------------------------------------------------------ Hadamard (fp32)
+// Unnormalised Sylvester transform, stages h = 1, 2, ..., 64 in this order.
+// v[j] = (x_{32h+j}, x_{32h+j+64}); stage 32 pairs this thread's j with the
+// partner's j (x_i with x_{i+32}); stage 64 is the pair's own butterfly.
+// Every output is the IEEE fp32 sum / difference of the same two operands as
+// the scalar butterfly network.
+__device__ __forceinline__ void fwht_half(float2 (&v)[32], int half) {
 #pragma unroll
-  for (int j = 0; j < 64; ++j) {
+  for (int s = 1; s < 32; s <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (!(j & s)) {
+        const float2 A = v[j], B = v[j + s];
+        v[j] = add2(A, B);
+        v[j + s] = sub2(A, B);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[j].x, 16),
+                                 __shfl_xor_sync(0xffffffffu, v[j].y, 16));
+    // half 0 holds x_i (a), half 1 holds x_{i+32} (b): a+b and a-b
+    v[j] = half ? sub2(o, v[j]) : add2(v[j], o);
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
     const float a = v[j].x, b = v[j].y;
     v[j] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
   }
+}
+
+// ---------------------------------------------------------- E8 (fp32x2)
+// Nearest E8 point of two groups at once (lane x: group g, lane y: group
+// g+8), Conway-Sloane: per coset (shift 0 and 1/2) u = y - shift, f = rint(u)
+// (ties to even via the 1.5*2^23 trick), e = u - f, d = e0^2 then an fma
+// chain, an odd sum of f adds 1 - 2 max|e| (moving the first largest-error
+// coordinate toward u); the half coset wins only when strictly closer.
+// Returns the clamped b-bit codes of each lane packed as code i at bits
+// [BITS*i, BITS*i + BITS), and the coset bit of each lane.
+template <int BITS>
+__device__ __forceinline__ void e8_pair(const float2 (&y)[8], uint32_t& gx, uint32_t& gy,
+                                        uint32_t& hx, uint32_t& hy) {
+  const float2 M2 = make_float2(kMagicRound, kMagicRound);
+  const float2 H2 = make_float2(0.5f, 0.5f);
+  float2 e0[8], e1[8];
+  float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
+  uint32_t p0x = 0, p0y = 0, p1x = 0, p1y = 0;
+  float m0x = 0.f, m0y = 0.f, m1x = 0.f, m1y = 0.f;
 #pragma unroll
-  for (int hp = 1; hp < 64; hp <<= 1) {
+  for (int i = 0; i < 8; ++i) {
+    const float2 r0 = add2(y[i], M2);
+    e0[i] = sub2(y[i], sub2(r0, M2));
+    const float2 u = sub2(y[i], H2);
+    const float2 r1 = add2(u, M2);
+    e1[i] = sub2(u, sub2(r1, M2));
+    p0x ^= __float_as_uint(r0.x);
+    p0y ^= __float_as_uint(r0.y);
+    p1x ^= __float_as_uint(r1.x);
+    p1y ^= __float_as_uint(r1.y);
+    d0 = i == 0 ? mul2(e0[i], e0[i]) : fma2(e0[i], e0[i], d0);
+    d1 = i == 0 ? mul2(e1[i], e1[i]) : fma2(e1[i], e1[i], d1);
+    m0x = fmaxf(m0x, fabsf(e0[i].x));
+    m0y = fmaxf(m0y, fabsf(e0[i].y));
+    m1x = fmaxf(m1x, fabsf(e1[i].x));
+    m1y = fmaxf(m1y, fabsf(e1[i].y));
+  }
+  const float2 m0 = make_float2(m0x, m0y), m1 = make_float2(m1x, m1y);
+  const float2 fix0 = add2(d0, fma2(make_float2(-2.f, -2.f), m0, make_float2(1.f, 1.f)));
+  const float2 fix1 = add2(d1, fma2(make_float2(-2.f, -2.f), m1, make_float2(1.f, 1.f)));
+  const bool o0x = p0x & 1u, o0y = p0y & 1u, o1x = p1x & 1u, o1y = p1y & 1u;
+  const float D0x = o0x ? fix0.x : d0.x, D0y = o0y ? fix0.y : d0.y;
+  const float D1x = o1x ? fix1.x : d1.x, D1y = o1y ? fix1.y : d1.y;
+  const bool halfx = D1x < D0x, halfy = D1y < D0y;
+  hx = halfx;
+  hy = halfy;
+
+  // chosen coset per lane: residual E, shifted input U, rounded F = U - E
+  const float2 hh = make_float2(halfx ? 1.f : 0.f, halfy ? 1.f : 0.f);
+  const float mx = halfx ? m1x : m0x, my = halfy ? m1y : m0y;
+  bool fx = !(halfx ? o1x : o0x), fy = !(halfy ? o1y : o0y);  // "fix done" flags
+  constexpr float kOffH = static_cast<float>(1 << (BITS - 1)) + kTwo23;
+  constexpr float kOffI = static_cast<float>((1 << (BITS - 1)) - 1) + kTwo23;
+  constexpr float kLoH = -static_cast<float>(1 << (BITS - 1));
+  constexpr float kHiH = static_cast<float>((1 << (BITS - 1)) - 1);
+  constexpr float kLoI = -static_cast<float>((1 << (BITS - 1)) - 1);
+  constexpr float kHiI = static_cast<float>((1 << (BITS - 1)) - 1);
+  const float2 off = make_float2(halfx ? kOffH : kOffI, halfy ? kOffH : kOffI);
+  const float lox = halfx ? kLoH : kLoI, loy = halfy ? kLoH : kLoI;
+  const float hix = halfx ? kHiH : kHiI, hiy = halfy ? kHiH : kHiI;
+  uint32_t ax = 0, ay = 0;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      if (!(j & hp)) {
-        const float2 A = v[j], B = v[j + hp];
-        v[j] = add2(A, B);
-        v[j + hp] = sub2(A, B);
+  for (int i = 0; i < 8; ++i) {
+    const float2 E = make_float2(halfx ? e1[i].x : e0[i].x, halfy ? e1[i].y : e0[i].y);
+    const float2 U = fma2(hh, make_float2(-0.5f, -0.5f), y[i]);
+    float2 F = sub2(U, E);
+    const bool hitx = !fx && fabsf(E.x) == mx;
+    const bool hity = !fy && fabsf(E.y) == my;
+    fx = fx || hitx;
+    fy = fy || hity;
+    if (hitx) F.x = __fadd_rn(F.x, E.x >= 0.f ? 1.f : -1.f);
+    if (hity) F.y = __fadd_rn(F.y, E.y >= 0.f ? 1.f : -1.f);
+    F = make_float2(fminf(fmaxf(F.x, lox), hix), fminf(fmaxf(F.y, loy), hiy));
+    const float2 J = add2(F, off);  // 2^23 + code: the code sits in the low mantissa bits
+    ax += __float_as_uint(J.x) << (BITS * i);
+    ay += __float_as_uint(J.y) << (BITS * i);
+  }
+  gx = ax & ((1u << (8 * BITS)) - 1u);
+  gy = ay & ((1u << (8 * BITS)) - 1u);
+}
+
+// --------------------------------------------------------------- encode
+// Staged bf16 row -> this half's 64 coordinates; keys: RoPE removed.
+template <bool ROPE>
+__device__ __forceinline__ void load_half(float2 (&v)[32], uint32_t row, uint32_t csa, int half) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 A = lds128(row + 16 * (4 * half + q));      // x_{32h+8q .. +7}
+    const uint4 B = lds128(row + 16 * (8 + 4 * half + q));  // x_{64+32h+8q .. +7}
+    const uint32_t a[4] = {A.x, A.y, A.z, A.w}, b[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      v[8 * q + 2 * t] = make_float2(bf16lo(a[t]), bf16lo(b[t]));
+      v[8 * q + 2 * t + 1] = make_float2(bf16hi(a[t]), bf16hi(b[t]));
+    }
+  }
+  if (ROPE) {
+    // u_i = fmaf(k_i, c, k_{i+64} s),  u_{i+64} = fmaf(k_{i+64}, c, -(k_i s))
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const float4 t = lds128f(csa + jj * (kSlots * 16));
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const float c = w ? t.z : t.x, s = w ? t.w : t.y;
+        const float2 P = v[2 * jj + w];
+        const float2 Q = mul2(P, make_float2(s, s));
+        v[2 * jj + w] = make_float2(__fmaf_rn(P.x, c, Q.y), __fmaf_rn(P.y, c, -Q.x));
       }
     }
   }
 }
 
-// ------------------------------------------------------------ E8 (fp32)
-// One D8 + shift decode (shift 0 or 1/2), Conway-Sloane:
-//   u = y - shift; f = rint(u) (ties to even, via the 1.5*2^23 round trick);
-//   e = u - f; d = e0^2 then fma chain; parity = sum f mod 2 (LSB of the
-//   rounded float's bits); m = max |e|.
-struct D8 {
-  float f[8], e[8];
-  float d, m;
-  uint32_t par;
-};
-
-__device__ __forceinline__ void d8_decode(const float (&y)[8], float shift, D8& o) {
-  uint32_t par = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float u = __fsub_rn(y[i], shift);
-    const float rr = __fadd_rn(u, kMagicRound);
-    o.f[i] = __fsub_rn(rr, kMagicRound);
-    o.e[i] = __fsub_rn(u, o.f[i]);
-    par ^= __float_as_uint(rr);
-  }
-  float d = __fmul_rn(o.e[0], o.e[0]);
-#pragma unroll
-  for (int i = 1; i < 8; ++i) d = __fmaf_rn(o.e[i], o.e[i], d);
-  float m = fabsf(o.e[0]);
-#pragma unroll
-  for (int i = 1; i < 8; ++i) m = fmaxf(m, fabsf(o.e[i]));
-  o.par = par & 1u;
-  // an odd sum re-rounds the worst coordinate: |e|^2 grows by 1 - 2|e_k|
-  o.d = o.par ? __fadd_rn(d, __fmaf_rn(-2.0f, m, 1.0f)) : d;
-  o.m = m;
-}
-
-// Nearest E8 point of y and its b-bit codes, packed as BITS*8 bits
-// (code i at bits [BITS*i, BITS*i + BITS)); returns the coset (1 = half).
 template <int BITS>
-__device__ __forceinline__ uint32_t e8_codes(const float (&y)[8], uint32_t& half_out) {
-  D8 c0, c1;
-  d8_decode(y, 0.0f, c0);
-  d8_decode(y, 0.5f, c1);
-  const bool half = c1.d < c0.d;
-  const float m = half ? c1.m : c0.m;
-  bool found = !(half ? c1.par : c0.par);  // even sum: nothing to fix
-  constexpr float kOffHalf = static_cast<float>(1 << (BITS - 1));
-  constexpr float kOffInt = static_cast<float>((1 << (BITS - 1)) - 1);
-  constexpr float kMaxHalf = static_cast<float>((1 << BITS) - 1);
-  constexpr float kMaxInt = static_cast<float>((1 << BITS) - 2);
-  const float off = half ? kOffHalf : kOffInt;
-  const float jmax = half ? kMaxHalf : kMaxInt;
-  uint32_t acc = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float e = half ? c1.e[i] : c0.e[i];
-    float f = half ? c1.f[i] : c0.f[i];
-    const bool hit = !found && (fabsf(e) == m);
-    found = found || hit;
-    if (hit) f = __fadd_rn(f, e >= 0.0f ? 1.0f : -1.0f);
-    const float jf = fminf(fmaxf(__fadd_rn(f, off), 0.0f), jmax);
-    acc += __float_as_uint(__fadd_rn(jf, kTwo23)) << (BITS * i);
-  }
-  half_out = half ? 1u : 0u;
-  return acc & ((1u << (8 * BITS)) - 1u);
-}
-
-// ----------------------------------------------------------- encode core
-// Staged bf16 row -> fp32 pairs; keys: RoPE removed at the slot's position.
-template <bool ROPE>
-__device__ __forceinline__ void load_row(float2 (&v)[64], uint32_t row_addr, uint32_t cs_addr) {
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint4 q = lds128(row_addr + 16 * c);
-    v[4 * c + 0] = make_float2(bf16lo(q.x), bf16hi(q.x));
-    v[4 * c + 1] = make_float2(bf16lo(q.y), bf16hi(q.y));
-    v[4 * c + 2] = make_float2(bf16lo(q.z), bf16hi(q.z));
-    v[4 * c + 3] = make_float2(bf16lo(q.w), bf16hi(q.w));
-  }
-  if (ROPE) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float4 t = lds128f(cs_addr + j * (kTileSlots * 16));
-      const float2 c2 = make_float2(t.x, t.y), s2 = make_float2(t.z, t.w);
-      const float2 A = v[j], B = v[j + 32];
-      const float2 bs = mul2(B, s2);
-      const float2 as = mul2(A, s2);
-      v[j] = fma2(A, c2, bs);
-      v[j + 32] = fma2(B, c2, make_float2(-as.x, -as.y));
-    }
-  }
-}
-
-// Rotate, scale, E8-quantise and pack one vector.
-template <int BITS>
-__device__ __forceinline__ void quantise(float2 (&v)[64], uint32_t* codes, uint32_t* meta) {
-  fwht128(v);
+__device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool valid,
+                                              uint32_t* codes, uint32_t* meta) {
+  fwht_half(v, half);
   float M = 0.0f;
 #pragma unroll
-  for (int j = 0; j < 64; ++j) M = fmaxf(M, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
+  for (int j = 0; j < 32; ++j) M = fmaxf(M, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
+  M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
   const float G = __uint_as_float(BITS == 3 ? kG3Bits : kG2Bits);
   const float C = __uint_as_float(kCBits);
-  const float sm = fminf(__fmul_rn(M, G), 65504.0f);
-  const __half sh = __float2half_rn(sm);
+  const __half sh = __float2half_rn(fminf(__fmul_rn(M, G), 65504.0f));
   const float sig = __half2float(sh);
   const float r = (sig == 0.0f) ? 0.0f : __fdiv_rn(C, sig);
   const float2 r2 = make_float2(r, r);
 
-  uint32_t gw[16];
-  uint32_t cmask = 0;
+  uint32_t gx[4], gy[4];
+  uint32_t cm = 0;
 #pragma unroll
-  for (int g = 0; g < 16; ++g) {
-    const float2 p0 = mul2(v[4 * g + 0], r2), p1 = mul2(v[4 * g + 1], r2);
-    const float2 p2 = mul2(v[4 * g + 2], r2), p3 = mul2(v[4 * g + 3], r2);
-    const float y[8] = {p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y};
-    uint32_t half;
-    gw[g] = e8_codes<BITS>(y, half);
-    cmask |= half << g;
+  for (int q = 0; q < 4; ++q) {
+    float2 y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = mul2(v[8 * q + i], r2);
+    uint32_t hx, hy;
+    e8_pair<BITS>(y, gx[q], gy[q], hx, hy);
+    cm |= (hx << (4 * half + q)) | (hy << (8 + 4 * half + q));
   }
-  uint4* dst = reinterpret_cast<uint4*>(codes);
+  cm |= __shfl_xor_sync(0xffffffffu, cm, 16);
+  if (!valid) return;
   if (BITS == 3) {
-    // three words per 32 coordinates (four 24-bit groups)
-    uint32_t w[12];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t g0 = gw[4 * q], g1 = gw[4 * q + 1], g2 = gw[4 * q + 2], g3 = gw[4 * q + 3];
-      w[3 * q + 0] = g0 | (g1 << 24);
-      w[3 * q + 1] = (g1 >> 8) | (g2 << 16);
-      w[3 * q + 2] = (g2 >> 16) | (g3 << 8);
+    // groups 4h..4h+3 -> words 3h..3h+2; groups 8+4h.. -> words 6+3h..
+    const uint32_t a0 = gx[0] | (gx[1] << 24), a1 = (gx[1] >> 8) | (gx[2] << 16),
+                   a2 = (gx[2] >> 16) | (gx[3] << 8);
+    const uint32_t b0 = gy[0] | (gy[1] << 24), b1 = (gy[1] >> 8) | (gy[2] << 16),
+                   b2 = (gy[2] >> 16) | (gy[3] << 8);
+    if (half == 0) {
+      *reinterpret_cast<uint2*>(codes + 0) = make_uint2(a0, a1);
+      codes[2] = a2;
+      *reinterpret_cast<uint2*>(codes + 6) = make_uint2(b0, b1);
+      codes[8] = b2;
+    } else {
+      codes[3] = a0;
+      *reinterpret_cast<uint2*>(codes + 4) = make_uint2(a1, a2);
+      codes[9] = b0;
+      *reinterpret_cast<uint2*>(codes + 10) = make_uint2(b1, b2);
     }
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
   } else {
-    uint32_t w[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) w[q] = gw[2 * q] | (gw[2 * q + 1] << 16);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    // groups 4h..4h+3 -> words 2h, 2h+1; groups 8+4h.. -> words 4+2h, 5+2h
+    *reinterpret_cast<uint2*>(codes + 2 * half) =
+        make_uint2(gx[0] | (gx[1] << 16), gx[2] | (gx[3] << 16));
+    *reinterpret_cast<uint2*>(codes + 4 + 2 * half) =
+        make_uint2(gy[0] | (gy[1] << 16), gy[2] | (gy[3] << 16));
   }
-  *meta = cmask | (static_cast<uint32_t>(__half_as_ushort(sh)) << 16);
-}
-
-// ----------------------------------------------------------- decode core
-template <int BITS>
-__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[4 * BITS], int c) {
-  const int p = BITS * c;
-  const int wi = p >> 5, off = p & 31;
-  uint32_t x;
-  if (off + BITS <= 32) {
-    x = w[wi] >> off;
-  } else {
-    x = __funnelshift_r(w[wi], w[wi + 1], off);
-  }
-  return x & ((1u << BITS) - 1u);
+  if (half == 0) *meta = cm | (static_cast<uint32_t>(__half_as_ushort(sh)) << 16);
 }
 
 template <int BITS, bool ROPE>
-__device__ __forceinline__ void decode_vector(const uint32_t (&w)[4 * BITS], uint32_t meta,
-                                              uint32_t cs_addr, uint32_t out_addr) {
-  float2 v[64];
-  // x = 2^22 + j (the fp32 spacing at 2^22 is 1/2, so the mantissa holds 2j);
-  // t = 2x - 2^23 - (2^b - 2) - h, every constant below 2^24: exact.
-  constexpr float kBase = -8388608.0f - static_cast<float>((1 << BITS) - 2);
-#pragma unroll
-  for (int g = 0; g < 16; ++g) {
-    const float kg = kBase - static_cast<float>((meta >> g) & 1u);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int c = 8 * g + 2 * k;
-      const float x0 = __uint_as_float(0x4A800000u | (code_at<BITS>(w, c) << 1));
-      const float x1 = __uint_as_float(0x4A800000u | (code_at<BITS>(w, c + 1) << 1));
-      v[4 * g + k] = fma2(make_float2(x0, x1), make_float2(2.0f, 2.0f), make_float2(kg, kg));
-    }
-  }
-  fwht128(v);
-  const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(meta >> 16)));
-  const float kappa = __fmul_rn(__fmul_rn(sig, 0.5f), __uint_as_float(kCBits));
-  const float2 k2 = make_float2(kappa, kappa);
-#pragma unroll
-  for (int j = 0; j < 64; ++j) v[j] = mul2(v[j], k2);
-  if (ROPE) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float4 t = lds128f(cs_addr + j * (kTileSlots * 16));
-      const float2 c2 = make_float2(t.x, t.y), s2 = make_float2(t.z, t.w);
-      const float2 A = v[j], B = v[j + 32];
-      const float2 bs = mul2(B, s2);
-      const float2 as = mul2(A, s2);
-      v[j] = fma2(A, c2, make_float2(-bs.x, -bs.y));
-      v[j + 32] = fma2(B, c2, as);
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    uint32_t q[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const __nv_bfloat162 b = __floats2bfloat162_rn(v[4 * c + k].x, v[4 * c + k].y);
-      q[k] = *reinterpret_cast<const uint32_t*>(&b);
-    }
-    sts128(out_addr + 16 * c, make_uint4(q[0], q[1], q[2], q[3]));
-  }
-}
-
-// ------------------------------------------------------------- encode
-__global__ void __launch_bounds__(256, 1) encode_kernel(const CodecArgs a) {
+__global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int nthreads = blockDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rows_bytes = nthreads * kRowPad;
-  const int stage_bytes = rows_bytes + kCsBytes;
+  const int slot_l = lane & 15, half = lane >> 4;
+  const int rows_bytes = (nthreads / 2) * kRowPad;
+  const int stage_bytes = rows_bytes + (ROPE ? kCsBytes : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * stage_bytes);
+  const int row_idx = warp * kSlots + slot_l;  // this vector's staged row
 
   const int64_t first = blockIdx.x, step = gridDim.x;
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
@@ -332,20 +302,19 @@ __global__ void __launch_bounds__(256, 1) encode_kernel(const CodecArgs a) {
 
   auto issue = [&](int64_t k, int s) {
     const Tile tl = tile_of(a, first + k * step);
-    const KindParams& kp = a.kind[tl.kind];
     unsigned char* st = smem + s * stage_bytes;
     const int h = tl.group * a.hg + warp;
-    const int64_t slot = tl.stile * kTileSlots + lane;
-    const int64_t valid = min64(kTileSlots, a.n - tl.stile * kTileSlots);
+    const int64_t slot = tl.stile * kSlots + slot_l;
+    const int64_t valid = min64(kSlots, a.n - tl.stile * kSlots);
     if (tid == 0) mbar_arrive_expect_tx(&bars[s], static_cast<uint32_t>(valid * a.hg * 256));
-    if (slot < a.n) {
+    if (half == 0 && slot < a.n) {
       int64_t src = slot;
       if (a.idx) src = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot);
       src = src < 0 ? 0 : (src >= a.T_in ? a.T_in - 1 : src);
-      const uint16_t* g = kp.src + tl.unit * kp.su + h * kp.sh + src * kp.st;
-      bulk_g2s(st + tid * kRowPad, g, 256, &bars[s]);
+      const uint16_t* g = a.kv + tl.unit * a.su + h * a.sh + src * a.st;
+      bulk_g2s(st + row_idx * kRowPad, g, 256, &bars[s]);
     }
-    if (kp.rope) fill_cs(a, tl, true, reinterpret_cast<float4*>(st + rows_bytes), tid, nthreads);
+    if (ROPE) fill_cs(a, tl, reinterpret_cast<float4*>(st + rows_bytes), tid, nthreads);
   };
 
   if (my_tiles > 0) issue(0, 0);
@@ -359,100 +328,170 @@ __global__ void __launch_bounds__(256, 1) encode_kernel(const CodecArgs a) {
     if (!__syncthreads_and(ok)) return;  // a copy never landed: error word set, stop
 
     const Tile tl = tile_of(a, first + k * step);
-    const KindParams& kp = a.kind[tl.kind];
     const int h = tl.group * a.hg + warp;
-    const int64_t slot = tl.stile * kTileSlots + lane;
-    unsigned char* st = smem + s * stage_bytes;
-    const uint32_t row = smem_u32(st + tid * kRowPad);
-    const uint32_t csa = smem_u32(st + rows_bytes) + lane * 16;
+    const int64_t slot = tl.stile * kSlots + slot_l;
     const bool valid = slot < a.n;
-    // The staged row (and its RoPE pairs) moves to registers, then the stage
-    // is refilled with tile k+2 while this tile is quantised.
-    float2 v[64];
+    unsigned char* st = smem + s * stage_bytes;
+    float2 v[32];
     if (valid) {
-      if (kp.rope) load_row<true>(v, row, csa);
-      else load_row<false>(v, row, csa);
+      load_half<ROPE>(v, smem_u32(st + row_idx * kRowPad),
+                      smem_u32(st + rows_bytes) + (16 * half * kSlots + slot_l) * 16, half);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = make_float2(0.f, 0.f);
     }
     __syncthreads();  // everyone is done with stage s
     if (k + 2 < my_tiles) issue(k + 2, s);
-    if (valid) {
-      const int64_t vec = tl.unit * kp.pu + h * kp.ph + a.slot0 + slot;
-      uint32_t* codes = kp.codes + vec * (4 * kp.bits);
-      uint32_t* meta = kp.meta + vec;
-      if (kp.bits == 3) quantise<3>(v, codes, meta);
-      else quantise<2>(v, codes, meta);
-    }
+    const int64_t vec = tl.unit * a.pu + h * a.ph + a.slot0 + slot;
+    quantise_half<BITS>(v, half, valid, a.codes + vec * (4 * BITS), a.meta + vec);
   }
 }
 
-// ------------------------------------------------------------- decode
-__global__ void __launch_bounds__(256, 1) decode_kernel(const CodecArgs a) {
+// --------------------------------------------------------------- decode
+// Code of coordinate c of a 32-coordinate block held in BITS words
+// (code c at bits [BITS*c, BITS*c + BITS) of the block's little-endian words).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[BITS], int c) {
+  const int p = BITS * c;
+  const int wi = p >> 5, off = p & 31;
+  const int wn = wi + 1 < BITS ? wi + 1 : wi;  // never read past the block
+  const uint32_t x = (off + BITS <= 32) ? (w[wi] >> off) : __funnelshift_r(w[wi], w[wn], off);
+  return x & ((1u << BITS) - 1u);
+}
+
+template <int BITS, bool ROPE>
+__device__ __forceinline__ void decode_half(const uint32_t (&w)[4 * BITS], uint32_t meta,
+                                            uint32_t csa, uint32_t row, int half) {
+  // This half's blocks: coordinates [32h, 32h+32) and [64+32h, 96+32h), each
+  // BITS words starting at word BITS*h and BITS*(2+h).
+  uint32_t wa[BITS], wb[BITS];
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) {
+    wa[k] = half ? w[BITS + k] : w[k];
+    wb[k] = half ? w[3 * BITS + k] : w[2 * BITS + k];
+  }
+  float2 v[32];
+  // x = 2^22 + j (the fp32 spacing at 2^22 is 1/2, so the mantissa holds 2j);
+  // t = 2x - 2^23 - (2^b - 2) - h, every constant below 2^24: exact.
+  constexpr float kBase = -8388608.0f - static_cast<float>((1 << BITS) - 2);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int ga = 4 * half + q, gb = 8 + 4 * half + q;
+    const float2 kg = make_float2(kBase - static_cast<float>((meta >> ga) & 1u),
+                                  kBase - static_cast<float>((meta >> gb) & 1u));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float xa = __uint_as_float(0x4A800000u | (code_at<BITS>(wa, 8 * q + i) << 1));
+      const float xb = __uint_as_float(0x4A800000u | (code_at<BITS>(wb, 8 * q + i) << 1));
+      v[8 * q + i] = fma2(make_float2(xa, xb), make_float2(2.0f, 2.0f), kg);
+    }
+  }
+  fwht_half(v, half);
+  const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(meta >> 16)));
+  const float kappa = __fmul_rn(__fmul_rn(sig, 0.5f), __uint_as_float(kCBits));
+  const float2 k2 = make_float2(kappa, kappa);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = mul2(v[j], k2);
+  if (ROPE) {
+    // o_i = fmaf(x_i, c, -(x_{i+64} s)),  o_{i+64} = fmaf(x_{i+64}, c, x_i s)
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const float4 t = lds128f(csa + jj * (kSlots * 16));
+#pragma unroll
+      for (int ww = 0; ww < 2; ++ww) {
+        const float c = ww ? t.z : t.x, s = ww ? t.w : t.y;
+        const float2 P = v[2 * jj + ww];
+        const float2 Q = mul2(P, make_float2(s, s));
+        v[2 * jj + ww] = make_float2(__fmaf_rn(P.x, c, -Q.y), __fmaf_rn(P.y, c, Q.x));
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t A[4], B[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const __nv_bfloat162 pa = __floats2bfloat162_rn(v[8 * q + 2 * t].x, v[8 * q + 2 * t + 1].x);
+      const __nv_bfloat162 pb = __floats2bfloat162_rn(v[8 * q + 2 * t].y, v[8 * q + 2 * t + 1].y);
+      A[t] = *reinterpret_cast<const uint32_t*>(&pa);
+      B[t] = *reinterpret_cast<const uint32_t*>(&pb);
+    }
+    sts128(row + 16 * (4 * half + q), make_uint4(A[0], A[1], A[2], A[3]));
+    sts128(row + 16 * (8 + 4 * half + q), make_uint4(B[0], B[1], B[2], B[3]));
+  }
+}
+
+// Codes and meta of this thread's vector in tile t (registers, one tile ahead).
+template <int BITS>
+__device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int warp, int slot_l,
+                                           uint32_t (&w)[4 * BITS], uint32_t& meta) {
+  const Tile tl = tile_of(a, t);
+  const int h = tl.group * a.hg + warp;
+  const int64_t slot = tl.stile * kSlots + slot_l;
+  if (slot < a.n) {
+    const int64_t vec = tl.unit * a.pu + h * a.ph + a.slot0 + slot;
+    const uint4* src = reinterpret_cast<const uint4*>(a.codes + vec * (4 * BITS));
+#pragma unroll
+    for (int c = 0; c < BITS; ++c) {
+      const uint4 q = __ldg(src + c);
+      w[4 * c] = q.x;
+      w[4 * c + 1] = q.y;
+      w[4 * c + 2] = q.z;
+      w[4 * c + 3] = q.w;
+    }
+    meta = __ldg(a.meta + vec);
+  }
+}
+
+template <int BITS, bool ROPE>
+__global__ void __launch_bounds__(256, 2) decode_kernel(const CodecArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int nthreads = blockDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int slot_l = lane & 15, half = lane >> 4;
   unsigned char* out_rows = smem;
-  float4* cs_buf[2] = {reinterpret_cast<float4*>(smem + nthreads * kRowPad),
-                       reinterpret_cast<float4*>(smem + nthreads * kRowPad + kCsBytes)};
-  const uint32_t row = smem_u32(out_rows + tid * kRowPad);
+  unsigned char* cs_base = smem + (nthreads / 2) * kRowPad;  // two cs buffers, kCsBytes each
+  const int row_idx = warp * kSlots + slot_l;
+  const uint32_t row = smem_u32(out_rows + row_idx * kRowPad);
 
   const int64_t first = blockIdx.x, step = gridDim.x;
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
 
-  uint32_t w[12];
+  uint32_t w[4 * BITS];
   uint32_t meta = 0;
-  auto load_in = [&](int64_t k) {
-    const Tile tl = tile_of(a, first + k * step);
-    const KindParams& kp = a.kind[tl.kind];
-    const int h = tl.group * a.hg + warp;
-    const int64_t slot = tl.stile * kTileSlots + lane;
-    if (slot < a.n) {
-      const int64_t vec = tl.unit * kp.pu + h * kp.ph + a.slot0 + slot;
-      const uint4* src = reinterpret_cast<const uint4*>(kp.codes + vec * (4 * kp.bits));
-      const uint4 q0 = __ldg(src), q1 = __ldg(src + 1);
-      w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
-      w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
-      if (kp.bits == 3) {
-        const uint4 q2 = __ldg(src + 2);
-        w[8] = q2.x; w[9] = q2.y; w[10] = q2.z; w[11] = q2.w;
-      }
-      meta = __ldg(kp.meta + vec);
-    }
-  };
+#pragma unroll
+  for (int i = 0; i < 4 * BITS; ++i) w[i] = 0;
   auto prep_cs = [&](int64_t k, int b) {
-    const Tile tl = tile_of(a, first + k * step);
-    if (a.kind[tl.kind].rope) fill_cs(a, tl, true, cs_buf[b], tid, nthreads);
+    if (ROPE)
+      fill_cs(a, tile_of(a, first + k * step), reinterpret_cast<float4*>(cs_base + b * kCsBytes),
+              tid, nthreads);
   };
 
   if (my_tiles > 0) {
     prep_cs(0, 0);
-    load_in(0);
+    load_codes<BITS>(a, first, warp, slot_l, w, meta);
   }
   __syncthreads();
   for (int64_t k = 0; k < my_tiles; ++k) {
     const Tile tl = tile_of(a, first + k * step);
-    const KindParams& kp = a.kind[tl.kind];
     const int h = tl.group * a.hg + warp;
-    const int64_t slot = tl.stile * kTileSlots + lane;
-    uint32_t wc[12];
+    const int64_t slot = tl.stile * kSlots + slot_l;
+    uint32_t wc[4 * BITS];
 #pragma unroll
-    for (int i = 0; i < 12; ++i) wc[i] = w[i];
+    for (int i = 0; i < 4 * BITS; ++i) wc[i] = w[i];
     const uint32_t mc = meta;
-    if (k + 1 < my_tiles) load_in(k + 1);  // next tile's codes in flight during this one
-    if (slot < a.n) {
-      const uint32_t csa = smem_u32(cs_buf[k & 1]) + lane * 16;
-      bulk_wait_read_all();  // this thread's previous row store has left smem
-      if (kp.bits == 3) {
-        const uint32_t(&w3)[12] = wc;
-        if (kp.rope) decode_vector<3, true>(w3, mc, csa, row);
-        else decode_vector<3, false>(w3, mc, csa, row);
-      } else {
-        const uint32_t(&w2)[8] = *reinterpret_cast<const uint32_t(*)[8]>(wc);
-        if (kp.rope) decode_vector<2, true>(w2, mc, csa, row);
-        else decode_vector<2, false>(w2, mc, csa, row);
-      }
-      fence_proxy_async_smem();
-      uint16_t* dst = const_cast<uint16_t*>(kp.src) + tl.unit * kp.su + h * kp.sh + slot * kp.st;
-      bulk_s2g(dst, out_rows + tid * kRowPad, 256);
+    if (k + 1 < my_tiles) load_codes<BITS>(a, first + (k + 1) * step, warp, slot_l, w, meta);
+    const bool valid = slot < a.n;
+    // the row's previous bulk store (issued by half 0) has finished reading smem
+    if (half == 0) bulk_wait_read_all();
+    __syncwarp();
+    const uint32_t csa = smem_u32(cs_base + (k & 1) * kCsBytes) + (16 * half * kSlots + slot_l) * 16;
+    decode_half<BITS, ROPE>(wc, mc, csa, row, half);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (valid && half == 0) {
+      uint16_t* dst = const_cast<uint16_t*>(a.kv) + tl.unit * a.su + h * a.sh + slot * a.st;
+      bulk_s2g(dst, out_rows + row_idx * kRowPad, 256);
       bulk_commit();
     }
     if (k + 1 < my_tiles) prep_cs(k + 1, static_cast<int>((k + 1) & 1));
@@ -468,21 +507,23 @@ static int pick_head_group(int heads) {
   return 1;
 }
 
-static cudaError_t launch_codec(bool decode, CodecArgs& a, int units, cudaStream_t stream) {
+template <int BITS, bool ROPE>
+static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t stream) {
   a.hg = pick_head_group(a.heads);
   a.ngroups = a.heads / a.hg;
-  a.slot_tiles = (a.n + kTileSlots - 1) / kTileSlots;
-  a.num_tiles = static_cast<int64_t>(units) * a.slot_tiles * a.ngroups * a.nkinds;
+  a.slot_tiles = (a.n + kSlots - 1) / kSlots;
+  a.num_tiles = static_cast<int64_t>(units) * a.slot_tiles * a.ngroups;
   if (a.num_tiles == 0) return cudaSuccess;
   const int threads = 32 * a.hg;
+  const int rows_bytes = (threads / 2) * kRowPad;
   size_t smem;
   const void* fn;
   if (decode) {
-    smem = static_cast<size_t>(threads) * kRowPad + 2 * kCsBytes;
-    fn = reinterpret_cast<const void*>(decode_kernel);
+    smem = static_cast<size_t>(rows_bytes) + (ROPE ? 2 * kCsBytes : 0);
+    fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE>);
   } else {
-    smem = 2 * (static_cast<size_t>(threads) * kRowPad + kCsBytes) + 16;
-    fn = reinterpret_cast<const void*>(encode_kernel);
+    smem = 2 * (static_cast<size_t>(rows_bytes) + (ROPE ? kCsBytes : 0)) + 16;
+    fn = reinterpret_cast<const void*>(encode_kernel<BITS, ROPE>);
   }
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -497,10 +538,19 @@ static cudaError_t launch_codec(bool decode, CodecArgs& a, int units, cudaStream
   if (per_sm < 1) per_sm = 1;
   const int64_t grid = min64(a.num_tiles, static_cast<int64_t>(sms) * per_sm);
   if (decode)
-    decode_kernel<<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
+    decode_kernel<BITS, ROPE><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
   else
-    encode_kernel<<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
+    encode_kernel<BITS, ROPE><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+static cudaError_t launch_kind(bool decode, const CodecArgs& a, int bits, bool rope, int units,
+                               cudaStream_t stream) {
+  if (bits == 3)
+    return rope ? launch_one<3, true>(decode, a, units, stream)
+                : launch_one<3, false>(decode, a, units, stream);
+  return rope ? launch_one<2, true>(decode, a, units, stream)
+              : launch_one<2, false>(decode, a, units, stream);
 }
 
 cudaError_t codec_read_clear_error(uint32_t* flags) {
@@ -513,56 +563,82 @@ cudaError_t codec_read_clear_error(uint32_t* flags) {
   return cudaSuccess;
 }
 
-cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream) {
+static CodecArgs common_args(int heads, int64_t n, int64_t slot0, int64_t pos_base,
+                             const int32_t* idx, int64_t idx_stride, const float* tab,
+                             int64_t max_pos) {
   CodecArgs a{};
-  int nk = 0;
+  a.heads = heads;
+  a.n = n;
+  a.slot0 = slot0;
+  a.pos_base = pos_base;
+  a.idx = idx;
+  a.idx_stride = idx_stride;
+  a.tab = reinterpret_cast<const float2*>(tab);
+  a.n_a = (max_pos + 255) / 256;
+  return a;
+}
+
+cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream) {
+  CodecArgs a = common_args(L.heads, L.n, L.slot0, L.pos_base, L.kept, L.kept_stride, L.rope_tab,
+                            L.rope_max_pos);
+  a.T_in = L.T_in;
   if (L.K) {
-    a.kind[nk++] = KindParams{static_cast<const uint16_t*>(L.K), L.ks.unit, L.ks.head, L.ks.token,
-                              L.k_out.codes, L.k_out.meta, L.k_out.unit_stride,
-                              L.k_out.head_stride, L.k_out.bits, 1};
+    CodecArgs k = a;
+    k.kv = static_cast<const uint16_t*>(L.K);
+    k.su = L.ks.unit;
+    k.sh = L.ks.head;
+    k.st = L.ks.token;
+    k.codes = L.k_out.codes;
+    k.meta = L.k_out.meta;
+    k.pu = L.k_out.unit_stride;
+    k.ph = L.k_out.head_stride;
+    cudaError_t err = launch_kind(false, k, L.k_out.bits, true, L.units, stream);
+    if (err != cudaSuccess) return err;
   }
   if (L.V) {
-    a.kind[nk++] = KindParams{static_cast<const uint16_t*>(L.V), L.vs.unit, L.vs.head, L.vs.token,
-                              L.v_out.codes, L.v_out.meta, L.v_out.unit_stride,
-                              L.v_out.head_stride, L.v_out.bits, 0};
+    CodecArgs v = a;
+    v.kv = static_cast<const uint16_t*>(L.V);
+    v.su = L.vs.unit;
+    v.sh = L.vs.head;
+    v.st = L.vs.token;
+    v.codes = L.v_out.codes;
+    v.meta = L.v_out.meta;
+    v.pu = L.v_out.unit_stride;
+    v.ph = L.v_out.head_stride;
+    return launch_kind(false, v, L.v_out.bits, false, L.units, stream);
   }
-  a.nkinds = nk;
-  a.heads = L.heads;
-  a.T_in = L.T_in;
-  a.n = L.n;
-  a.slot0 = L.slot0;
-  a.pos_base = L.pos_base;
-  a.idx = L.kept;
-  a.idx_stride = L.kept_stride;
-  a.tab = reinterpret_cast<const float2*>(L.rope_tab);
-  a.n_a = (L.rope_max_pos + 255) / 256;
-  return launch_codec(false, a, L.units, stream);
+  return cudaSuccess;
 }
 
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
-  CodecArgs a{};
-  int nk = 0;
+  CodecArgs a = common_args(L.heads, L.n, L.slot0, L.pos_base, L.positions, L.pos_stride,
+                            L.rope_tab, L.rope_max_pos);
   if (L.K_out) {
-    a.kind[nk++] = KindParams{static_cast<const uint16_t*>(L.K_out), L.kos.unit, L.kos.head,
-                              L.kos.token, L.k_in.codes, L.k_in.meta, L.k_in.unit_stride,
-                              L.k_in.head_stride, L.k_in.bits, 1};
+    CodecArgs k = a;
+    k.kv = static_cast<const uint16_t*>(L.K_out);
+    k.su = L.kos.unit;
+    k.sh = L.kos.head;
+    k.st = L.kos.token;
+    k.codes = L.k_in.codes;
+    k.meta = L.k_in.meta;
+    k.pu = L.k_in.unit_stride;
+    k.ph = L.k_in.head_stride;
+    cudaError_t err = launch_kind(true, k, L.k_in.bits, true, L.units, stream);
+    if (err != cudaSuccess) return err;
   }
   if (L.V_out) {
-    a.kind[nk++] = KindParams{static_cast<const uint16_t*>(L.V_out), L.vos.unit, L.vos.head,
-                              L.vos.token, L.v_in.codes, L.v_in.meta, L.v_in.unit_stride,
-                              L.v_in.head_stride, L.v_in.bits, 0};
+    CodecArgs v = a;
+    v.kv = static_cast<const uint16_t*>(L.V_out);
+    v.su = L.vos.unit;
+    v.sh = L.vos.head;
+    v.st = L.vos.token;
+    v.codes = L.v_in.codes;
+    v.meta = L.v_in.meta;
+    v.pu = L.v_in.unit_stride;
+    v.ph = L.v_in.head_stride;
+    return launch_kind(true, v, L.v_in.bits, false, L.units, stream);
   }
-  a.nkinds = nk;
-  a.heads = L.heads;
-  a.T_in = 0;
-  a.n = L.n;
-  a.slot0 = L.slot0;
-  a.pos_base = L.pos_base;
-  a.idx = L.positions;
-  a.idx_stride = L.pos_stride;
-  a.tab = reinterpret_cast<const float2*>(L.rope_tab);
-  a.n_a = (L.rope_max_pos + 255) / 256;
-  return launch_codec(true, a, L.units, stream);
+  return cudaSuccess;
 }
 
 }  // namespace nq
