@@ -52,7 +52,7 @@ nq_status check_packed(const nq_packed* p, const char* name) {
 
 nq_status check_rope(const float* tab, int64_t max_pos) {
   if (!tab) return fail(NQ_ERR_INVALID, "rope_tab is NULL (required for keys)");
-  if (!aligned(tab, 8)) return fail(NQ_ERR_INVALID, "rope_tab must be 8-byte aligned");
+  if (!aligned(tab, 16)) return fail(NQ_ERR_INVALID, "rope_tab must be 16-byte aligned");
   if (max_pos < 1) return fail(NQ_ERR_INVALID, "rope_max_pos must be >= 1");
   return NQ_OK;
 }

@@ -32,6 +32,28 @@ namespace nq {
 constexpr int kSlots = 16;                  // slots per tile: one warp = 16 slots x 2 halves
 constexpr int kCsBytes = 32 * kSlots * 16;  // float4 cs[32][16]
 
+// Division by a fixed divisor for numerators below 2^31 (round-up method of
+// Granlund and Montgomery): q = (n * m) >> (31 + l), l = ceil(log2 d),
+// m = floor(2^(31+l) / d) + 1.
+struct FastDiv {
+  uint64_t m;
+  uint32_t d, shift;
+};
+
+static FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  FastDiv f;
+  f.d = d;
+  f.shift = 31 + l;
+  f.m = ((1ull << f.shift) / d) + 1;
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return static_cast<uint32_t>((static_cast<uint64_t>(n) * f.m) >> f.shift);
+}
+
 struct CodecArgs {
   const uint16_t* kv;  // encode: bf16 input; decode: bf16 output
   int64_t su, sh, st;  // element strides of the bf16 tensor
@@ -46,6 +68,7 @@ struct CodecArgs {
   const float2* tab;
   int64_t n_a;
   int64_t slot_tiles, num_tiles;
+  FastDiv div_groups, div_stiles;
 };
 
 struct Tile {
@@ -53,31 +76,47 @@ struct Tile {
   int64_t stile;
 };
 
-__device__ __forceinline__ Tile tile_of(const CodecArgs& a, int64_t t) {
+// Tile index -> (unit, slot tile, head group); tile counts stay below 2^31.
+__device__ __forceinline__ Tile tile_of(const CodecArgs& a, int64_t t64) {
+  const uint32_t t = static_cast<uint32_t>(t64);
+  const uint32_t q = fdiv(t, a.div_groups);
+  const uint32_t u = fdiv(q, a.div_stiles);
   Tile r;
-  r.group = static_cast<int>(t % a.ngroups);
-  t /= a.ngroups;
-  r.stile = t % a.slot_tiles;
-  r.unit = static_cast<int>(t / a.slot_tiles);
+  r.group = static_cast<int>(t - q * a.div_groups.d);
+  r.stile = static_cast<int64_t>(q - u * a.div_stiles.d);
+  r.unit = static_cast<int>(u);
   return r;
 }
 
 // cs table of one tile: float4 cs[j][slot] = (c_2j, s_2j, c_2j+1, s_2j+1) at
 // that slot's RoPE position; a thread of half h reads j in [16h, 16h+16).
+// Thread t fills slot t % 16 for j = t/16, t/16 + nthreads/16, ... : one
+// position lookup, then two table rows read at consecutive frequencies.
 __device__ __forceinline__ void fill_cs(const CodecArgs& a, const Tile& tl, float4* cs, int tid,
                                         int nthreads) {
-  for (int e = tid; e < 32 * kSlots; e += nthreads) {
-    const int slot_l = e % kSlots;
-    const int j = e / kSlots;
-    const int64_t slot = tl.stile * kSlots + slot_l;
+  const int slot_l = tid % kSlots;
+  const int64_t slot = tl.stile * kSlots + slot_l;
+  const float2* rowA = a.tab;
+  const float2* rowB = a.tab + a.n_a * kHalf;
+  if (slot < a.n) {
+    int64_t p = slot;
+    if (a.idx) p = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot);
+    p += a.pos_base;
+    int64_t hi = p >> 8;
+    hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
+    rowA = a.tab + hi * kHalf;
+    rowB = a.tab + (a.n_a + (p & 255)) * kHalf;
+  }
+  for (int j = tid / kSlots; j < 32; j += nthreads / kSlots) {
     float4 v = make_float4(1.f, 0.f, 1.f, 0.f);
     if (slot < a.n) {
-      int64_t p = slot;
-      if (a.idx) p = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot);
-      p += a.pos_base;
-      const float2 c0 = rope_cs(a.tab, a.n_a, p, 2 * j);
-      const float2 c1 = rope_cs(a.tab, a.n_a, p, 2 * j + 1);
-      v = make_float4(c0.x, c0.y, c1.x, c1.y);
+      const float4 A = __ldg(reinterpret_cast<const float4*>(rowA + 2 * j));
+      const float4 B = __ldg(reinterpret_cast<const float4*>(rowB + 2 * j));
+      // c = fmaf(cA, cB, -(sA sB)),  s = fmaf(sA, cB, cA sB)
+      v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
+      v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
+      v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
+      v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
     }
     cs[j * kSlots + slot_l] = v;
   }
@@ -101,12 +140,15 @@ __device__ __forceinline__ void fwht_half(float2 (&v)[32], int half) {
       }
     }
   }
+  // half 0 holds x_i (a), half 1 holds x_{i+32} (b): a+b = fma(a, 1, b) and
+  // a-b = fma(b, -1, a), each one rounding of the exact sum or difference
+  const float sg = half ? -1.0f : 1.0f;
+  const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[j].x, 16),
                                  __shfl_xor_sync(0xffffffffu, v[j].y, 16));
-    // half 0 holds x_i (a), half 1 holds x_{i+32} (b): a+b and a-b
-    v[j] = half ? sub2(o, v[j]) : add2(v[j], o);
+    v[j] = fma2(v[j], sg2, o);
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
@@ -130,19 +172,17 @@ __device__ __forceinline__ void e8_pair(const float2 (&y)[8], uint32_t& gx, uint
   const float2 H2 = make_float2(0.5f, 0.5f);
   float2 e0[8], e1[8];
   float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
-  uint32_t p0x = 0, p0y = 0, p1x = 0, p1y = 0;
+  float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);  // sums of f (exact)
   float m0x = 0.f, m0y = 0.f, m1x = 0.f, m1y = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float2 r0 = add2(y[i], M2);
-    e0[i] = sub2(y[i], sub2(r0, M2));
+    const float2 f0 = sub2(add2(y[i], M2), M2);
+    e0[i] = sub2(y[i], f0);
     const float2 u = sub2(y[i], H2);
-    const float2 r1 = add2(u, M2);
-    e1[i] = sub2(u, sub2(r1, M2));
-    p0x ^= __float_as_uint(r0.x);
-    p0y ^= __float_as_uint(r0.y);
-    p1x ^= __float_as_uint(r1.x);
-    p1y ^= __float_as_uint(r1.y);
+    const float2 f1 = sub2(add2(u, M2), M2);
+    e1[i] = sub2(u, f1);
+    s0 = add2(s0, f0);
+    s1 = add2(s1, f1);
     d0 = i == 0 ? mul2(e0[i], e0[i]) : fma2(e0[i], e0[i], d0);
     d1 = i == 0 ? mul2(e1[i], e1[i]) : fma2(e1[i], e1[i], d1);
     m0x = fmaxf(m0x, fabsf(e0[i].x));
@@ -150,10 +190,13 @@ __device__ __forceinline__ void e8_pair(const float2 (&y)[8], uint32_t& gx, uint
     m1x = fmaxf(m1x, fabsf(e1[i].x));
     m1y = fmaxf(m1y, fabsf(e1[i].y));
   }
+  // parity of an integer-valued sum: the LSB of its 1.5*2^23-biased bits
+  const float2 b0 = add2(s0, M2), b1 = add2(s1, M2);
+  const bool o0x = __float_as_uint(b0.x) & 1u, o0y = __float_as_uint(b0.y) & 1u;
+  const bool o1x = __float_as_uint(b1.x) & 1u, o1y = __float_as_uint(b1.y) & 1u;
   const float2 m0 = make_float2(m0x, m0y), m1 = make_float2(m1x, m1y);
   const float2 fix0 = add2(d0, fma2(make_float2(-2.f, -2.f), m0, make_float2(1.f, 1.f)));
   const float2 fix1 = add2(d1, fma2(make_float2(-2.f, -2.f), m1, make_float2(1.f, 1.f)));
-  const bool o0x = p0x & 1u, o0y = p0y & 1u, o1x = p1x & 1u, o1y = p1y & 1u;
   const float D0x = o0x ? fix0.x : d0.x, D0y = o0y ? fix0.y : d0.y;
   const float D1x = o1x ? fix1.x : d1.x, D1y = o1y ? fix1.y : d1.y;
   const bool halfx = D1x < D0x, halfy = D1y < D0y;
@@ -183,8 +226,9 @@ __device__ __forceinline__ void e8_pair(const float2 (&y)[8], uint32_t& gx, uint
     const bool hity = !fy && fabsf(E.y) == my;
     fx = fx || hitx;
     fy = fy || hity;
-    if (hitx) F.x = __fadd_rn(F.x, E.x >= 0.f ? 1.f : -1.f);
-    if (hity) F.y = __fadd_rn(F.y, E.y >= 0.f ? 1.f : -1.f);
+    // E is never -0 (y carries no -0), so its sign bit decides the direction
+    if (hitx) F.x = __fadd_rn(F.x, copysignf(1.0f, E.x));
+    if (hity) F.y = __fadd_rn(F.y, copysignf(1.0f, E.y));
     F = make_float2(fminf(fmaxf(F.x, lox), hix), fminf(fmaxf(F.y, loy), hiy));
     const float2 J = add2(F, off);  // 2^23 + code: the code sits in the low mantissa bits
     ax += __float_as_uint(J.x) << (BITS * i);
@@ -246,7 +290,7 @@ __device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool va
   for (int q = 0; q < 4; ++q) {
     float2 y[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = mul2(v[8 * q + i], r2);
+    for (int i = 0; i < 8; ++i) y[i] = add2(mul2(v[8 * q + i], r2), make_float2(0.f, 0.f));
     uint32_t hx, hy;
     e8_pair<BITS>(y, gx[q], gy[q], hx, hy);
     cm |= (hx << (4 * half + q)) | (hy << (8 + 4 * half + q));
@@ -348,15 +392,24 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
 }
 
 // --------------------------------------------------------------- decode
-// Code of coordinate c of a 32-coordinate block held in BITS words
-// (code c at bits [BITS*c, BITS*c + BITS) of the block's little-endian words).
+// 2^22 + j as an fp32 bit pattern for the code j of coordinate c of a
+// 32-coordinate block held in BITS words (code c at bits [BITS*c, BITS*c +
+// BITS) of the block's little-endian words): the code is moved to bit 1 with
+// one (funnel) shift and masked into the mantissa of 2^22 with one LOP3.
 template <int BITS>
-__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[BITS], int c) {
+__device__ __forceinline__ float code_as_float(const uint32_t (&w)[BITS], int c) {
   const int p = BITS * c;
   const int wi = p >> 5, off = p & 31;
   const int wn = wi + 1 < BITS ? wi + 1 : wi;  // never read past the block
-  const uint32_t x = (off + BITS <= 32) ? (w[wi] >> off) : __funnelshift_r(w[wi], w[wn], off);
-  return x & ((1u << BITS) - 1u);
+  uint32_t x;
+  if (off == 0) {
+    x = w[wi] << 1;
+  } else if (off + BITS <= 32) {
+    x = w[wi] >> (off - 1);
+  } else {
+    x = __funnelshift_r(w[wi], w[wn], off - 1);
+  }
+  return __uint_as_float((x & (((1u << BITS) - 1u) << 1)) | 0x4A800000u);
 }
 
 template <int BITS, bool ROPE>
@@ -381,8 +434,8 @@ __device__ __forceinline__ void decode_half(const uint32_t (&w)[4 * BITS], uint3
                                   kBase - static_cast<float>((meta >> gb) & 1u));
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float xa = __uint_as_float(0x4A800000u | (code_at<BITS>(wa, 8 * q + i) << 1));
-      const float xb = __uint_as_float(0x4A800000u | (code_at<BITS>(wb, 8 * q + i) << 1));
+      const float xa = code_as_float<BITS>(wa, 8 * q + i);
+      const float xb = code_as_float<BITS>(wb, 8 * q + i);
       v[8 * q + i] = fma2(make_float2(xa, xb), make_float2(2.0f, 2.0f), kg);
     }
   }
@@ -514,6 +567,9 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   a.slot_tiles = (a.n + kSlots - 1) / kSlots;
   a.num_tiles = static_cast<int64_t>(units) * a.slot_tiles * a.ngroups;
   if (a.num_tiles == 0) return cudaSuccess;
+  if (a.num_tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  a.div_groups = make_fastdiv(static_cast<uint32_t>(a.ngroups));
+  a.div_stiles = make_fastdiv(static_cast<uint32_t>(a.slot_tiles));
   const int threads = 32 * a.hg;
   const int rows_bytes = (threads / 2) * kRowPad;
   size_t smem;

@@ -150,19 +150,4 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-// ------------------------------------------------------------- RoPE table
-// Combine the two-level table for position pos and frequency pair index i:
-// c = fmaf(cA, cB, -(sA*sB)), s = fmaf(sA, cB, cA*sB).
-__device__ __forceinline__ float2 rope_cs(const float2* __restrict__ tab, int64_t n_a, int64_t pos,
-                                          int i) {
-  int64_t a = pos >> 8;
-  a = a < 0 ? 0 : (a >= n_a ? n_a - 1 : a);  // out-of-contract positions stay in bounds
-  const int b = static_cast<int>(pos & 255);
-  const float2 A = __ldg(tab + a * kHalf + i);
-  const float2 B = __ldg(tab + (n_a + b) * kHalf + i);
-  const float ss = __fmul_rn(A.y, B.y);
-  const float cs = __fmul_rn(A.x, B.y);
-  return make_float2(__fmaf_rn(A.x, B.x, -ss), __fmaf_rn(A.y, B.x, cs));
-}
-
 }  // namespace nq

@@ -52,23 +52,30 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = static_cast<double>(__ldg(mh + i));
     const uint16_t* base = K + u * ks.unit + h * ks.head + chunk * 8;
-#pragma unroll 4
-    for (int it = 0; it < kScoreTok / 2; ++it) {
-      const int tl = 2 * it + half;
-      const int64_t t = t0 + tl;
-      double acc = 0.0;
-      if (t < T) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(base + t * ks.token));
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    // 8 independent 16-byte loads per lane are in flight before any math
+    constexpr int kBatch = 8;
+#pragma unroll 1
+    for (int it0 = 0; it0 < kScoreTok / 2; it0 += kBatch) {
+      uint4 q[kBatch];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int64_t t = t0 + 2 * (it0 + b) + half;
+        q[b] = t < T ? __ldg(reinterpret_cast<const uint4*>(base + t * ks.token))
+                     : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const uint32_t w[4] = {q[b].x, q[b].y, q[b].z, q[b].w};
+        double acc = 0.0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           acc = fma(static_cast<double>(bf16lo(w[k])), m[2 * k], acc);
           acc = fma(static_cast<double>(bf16hi(w[k])), m[2 * k + 1], acc);
         }
-      }
 #pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (chunk == 0) part[h * kScoreTok + tl] = acc;
+        for (int o = 8; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (chunk == 0) part[h * kScoreTok + 2 * (it0 + b) + half] = acc;
+      }
     }
   }
   __syncthreads();
@@ -107,12 +114,17 @@ __device__ __forceinline__ void block_exclusive_scan32(int* vals /*[32] smem*/) 
   __syncthreads();
 }
 
+constexpr int kDigitBits = 11;
+constexpr int kBins = 1 << kDigitBits;  // 2 bins per thread
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __restrict__ scores,
                                                              int64_t T, int W, int64_t n_kept,
                                                              int32_t* __restrict__ kept,
                                                              int64_t kept_stride) {
   extern __shared__ uint32_t flagbits[];  // ceil(T/32) words
-  __shared__ unsigned int hist[256];
+  __shared__ unsigned int hist[kBins];
+  __shared__ uint64_t s_min[kSelWarps], s_max[kSelWarps];
+  __shared__ unsigned int s_wsum[kSelWarps];
   __shared__ uint64_t s_prefix;
   __shared__ int64_t s_k;
   __shared__ int warp_cnt[kSelWarps];
@@ -130,35 +142,87 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   const int64_t n_mid = n_kept - 1 - W;
 
   // --- radix select: the n_mid-th largest key among the middle tokens
-  uint64_t prefix = 0, pmask = 0;
+  uint64_t prefix = 0;
   int64_t k = n_mid;
   if (n_mid > 0) {
-    for (int pass = 0; pass < 8; ++pass) {
-      const int shift = 56 - 8 * pass;
-      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    // every candidate key lies in [kmin, kmax], so they share its common prefix
+    uint64_t kmin = ~0ull, kmax = 0ull;
+    for (int64_t t = lo + tid; t < hi; t += blockDim.x) {
+      const uint64_t key = score_key(__ldg(s + t));
+      kmin = key < kmin ? key : kmin;
+      kmax = key > kmax ? key : kmax;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const uint64_t a = __shfl_xor_sync(0xffffffffu, kmin, o);
+      const uint64_t b = __shfl_xor_sync(0xffffffffu, kmax, o);
+      kmin = a < kmin ? a : kmin;
+      kmax = b > kmax ? b : kmax;
+    }
+    if (lane == 0) {
+      s_min[warp] = kmin;
+      s_max[warp] = kmax;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint64_t mn = ~0ull, mx = 0ull;
+      for (int w = 0; w < kSelWarps; ++w) {
+        mn = s_min[w] < mn ? s_min[w] : mn;
+        mx = s_max[w] > mx ? s_max[w] : mx;
+      }
+      s_min[0] = mn;
+      s_max[0] = mx;
+    }
+    __syncthreads();
+    const uint64_t diff = s_min[0] ^ s_max[0];
+    int rem = diff ? 64 - __clzll(static_cast<long long>(diff)) : 0;  // bits still undecided
+    prefix = s_min[0] & (rem == 64 ? 0ull : ~((1ull << rem) - 1ull));
+    __syncthreads();
+    while (rem > 0) {
+      const int width = rem < kDigitBits ? rem : kDigitBits;
+      const int shift = rem - width;
+      const uint64_t pmask = rem == 64 ? 0ull : ~((1ull << rem) - 1ull);
+      for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
       __syncthreads();
       for (int64_t t = lo + tid; t < hi; t += blockDim.x) {
         const uint64_t key = score_key(__ldg(s + t));
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        if ((key & pmask) == prefix)
+          atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
       }
       __syncthreads();
-      if (tid == 0) {
-        int64_t cum = 0;
-        int sel = 0;
-        for (int d = 255; d >= 0; --d) {
-          if (cum + hist[d] >= k) {
-            sel = d;
-            break;
-          }
-          cum += hist[d];
+      // descending bins: thread t owns bins 2047-2t and 2046-2t
+      const int b0 = kBins - 1 - 2 * tid, b1 = b0 - 1;
+      const unsigned int c0 = hist[b0], c1 = hist[b1];
+      const unsigned int own = c0 + c1;
+      unsigned int inc = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (lane == 31) s_wsum[warp] = inc;
+      __syncthreads();
+      if (warp == 0) {
+        unsigned int w = s_wsum[lane], wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned int v = __shfl_up_sync(0xffffffffu, wi, o);
+          if (lane >= o) wi += v;
         }
-        s_k = k - cum;
-        s_prefix = prefix | (static_cast<uint64_t>(sel) << shift);
+        s_wsum[lane] = wi - w;  // exclusive prefix of warp totals
+      }
+      __syncthreads();
+      const int64_t before = static_cast<int64_t>(s_wsum[warp]) + (inc - own);  // keys in higher bins
+      if (before < k && k <= before + own) {
+        const bool first = k <= before + c0;
+        const int d = first ? b0 : b1;
+        s_k = k - before - (first ? 0 : c0);
+        s_prefix = prefix | (static_cast<uint64_t>(d) << shift);
       }
       __syncthreads();
       prefix = s_prefix;
       k = s_k;
-      pmask |= 0xFFull << shift;
+      rem = shift;
       __syncthreads();
     }
   }

@@ -28,7 +28,7 @@
  *   contiguous bf16 coordinates.  Its three strides are in ELEMENTS and must
  *   be multiples of 8, and the base pointer 16-byte aligned (16-byte vector
  *   loads).  A "unit" is one layer of one sequence.
- * - Inputs must be finite with |x| <= 2^32; other values are out of
+ * - Inputs must be finite with |x| <= 2^30; other values are out of
  *   contract (no fault: the kernels stay within their buffers, the codes of
  *   such a vector are unspecified).
  * - Kernels with bounded waits (mbarrier completion of bulk copies) give up
@@ -100,8 +100,9 @@ int64_t nq_packed_bytes_per_vector(int bits);
  *   B[b][i] = (cos(b*w_i),    sin(b*w_i)),     b < 256
  * as float2 pairs, A first then B.  The kernels combine them in fp32:
  *   c = fmaf(cA, cB, -(sA*sB)),  s = fmaf(sA, cB, cA*sB).
- * The caller copies the filled host buffer to device memory once per theta
- * and passes that device pointer with the same max_pos. */
+ * The caller copies the filled host buffer to device memory (16-byte
+ * aligned) once per theta and passes that device pointer with the same
+ * max_pos. */
 size_t nq_rope_tables_bytes(int64_t max_pos);
 nq_status nq_rope_tables_fill_host(double theta, int64_t max_pos, void *host_buf, size_t bytes);
 
