@@ -115,6 +115,7 @@ __device__ __forceinline__ void block_exclusive_scan32(int* vals /*[32] smem*/) 
 }
 
 constexpr int kDigitBits = 11;
+constexpr int kUnroll = 8;  // independent score loads in flight per thread
 constexpr int kBins = 1 << kDigitBits;  // 2 bins per thread
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __restrict__ scores,
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   __shared__ unsigned int s_wsum[kSelWarps];
   __shared__ uint64_t s_prefix;
   __shared__ int64_t s_k;
+  __shared__ int64_t s_eq;
   __shared__ int warp_cnt[kSelWarps];
 
   const int u = blockIdx.x;
@@ -144,13 +146,25 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   // --- radix select: the n_mid-th largest key among the middle tokens
   uint64_t prefix = 0;
   int64_t k = n_mid;
+  int64_t n_eq = hi - lo;  // keys equal to the threshold (all, until a radix pass splits them)
   if (n_mid > 0) {
     // every candidate key lies in [kmin, kmax], so they share its common prefix
     uint64_t kmin = ~0ull, kmax = 0ull;
-    for (int64_t t = lo + tid; t < hi; t += blockDim.x) {
-      const uint64_t key = score_key(__ldg(s + t));
-      kmin = key < kmin ? key : kmin;
-      kmax = key > kmax ? key : kmax;
+    for (int64_t t0 = lo + tid; t0 < hi; t0 += kUnroll * blockDim.x) {
+      double v[kUnroll];
+#pragma unroll
+      for (int j = 0; j < kUnroll; ++j) {
+        const int64_t t = t0 + j * blockDim.x;
+        v[j] = t < hi ? __ldg(s + t) : 0.0;
+      }
+#pragma unroll
+      for (int j = 0; j < kUnroll; ++j) {
+        if (t0 + j * blockDim.x < hi) {
+          const uint64_t key = score_key(v[j]);
+          kmin = key < kmin ? key : kmin;
+          kmax = key > kmax ? key : kmax;
+        }
+      }
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
@@ -184,10 +198,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
       const uint64_t pmask = rem == 64 ? 0ull : ~((1ull << rem) - 1ull);
       for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
       __syncthreads();
-      for (int64_t t = lo + tid; t < hi; t += blockDim.x) {
-        const uint64_t key = score_key(__ldg(s + t));
-        if ((key & pmask) == prefix)
-          atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
+      // warp-uniform loop bound (lanes past the end are masked by `in`)
+      for (int64_t w0 = lo + (tid & ~31); w0 < hi; w0 += kUnroll * blockDim.x) {
+        const int64_t t0 = w0 + lane;
+        double v[kUnroll];
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+          const int64_t t = t0 + j * blockDim.x;
+          v[j] = t < hi ? __ldg(s + t) : 0.0;
+        }
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+          const uint64_t key = score_key(v[j]);
+          const bool in = t0 + j * blockDim.x < hi && (key & pmask) == prefix;
+          if (in) atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
+        }
       }
       __syncthreads();
       // descending bins: thread t owns bins 2047-2t and 2046-2t
@@ -218,10 +243,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
         const int d = first ? b0 : b1;
         s_k = k - before - (first ? 0 : c0);
         s_prefix = prefix | (static_cast<uint64_t>(d) << shift);
+        s_eq = first ? c0 : c1;  // keys sharing the prefix so far (all of it after the last pass)
       }
       __syncthreads();
       prefix = s_prefix;
       k = s_k;
+      n_eq = s_eq;
       rem = shift;
       __syncthreads();
     }
@@ -233,13 +260,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   const int64_t seg = ((T + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
   const int64_t s0 = warp * seg, s1 = min64(T, s0 + seg);
 
-  // pass A: keys equal to the threshold, per warp
+  // pass A (only when ties at the threshold must be split by position):
+  // keys equal to the threshold, per warp
+  const bool rank_ties = n_mid > 0 && need_eq < n_eq;
   int eq = 0;
-  if (n_mid > 0) {
-    for (int64_t b = s0; b < s1; b += 32) {
-      const int64_t t = b + lane;
-      const bool is_eq = (t < s1) && (t >= lo) && (t < hi) && score_key(__ldg(s + t)) == kstar;
-      eq += __popc(__ballot_sync(0xffffffffu, is_eq));
+  if (rank_ties) {
+    for (int64_t b0 = s0; b0 < s1; b0 += 32 * kUnroll) {
+      double v[kUnroll];
+#pragma unroll
+      for (int j = 0; j < kUnroll; ++j) {
+        const int64_t t = b0 + 32 * j + lane;
+        v[j] = (t < s1 && t >= lo && t < hi) ? __ldg(s + t) : 0.0;
+      }
+#pragma unroll
+      for (int j = 0; j < kUnroll; ++j) {
+        const int64_t t = b0 + 32 * j + lane;
+        const bool is_eq = t < s1 && t >= lo && t < hi && score_key(v[j]) == kstar;
+        eq += __popc(__ballot_sync(0xffffffffu, is_eq));
+      }
     }
   }
   if (lane == 0) warp_cnt[warp] = eq;
@@ -250,20 +288,31 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
 
   // pass B: keep flags (bitmask in smem) and per-warp kept counts
   int cnt = 0;
-  for (int64_t b = s0; b < s1; b += 32) {
-    const int64_t t = b + lane;
-    const bool in_range = t < s1;
-    const bool mid = in_range && t >= lo && t < hi;
-    const uint64_t key = mid ? score_key(__ldg(s + t)) : 0ull;
-    const bool is_eq = mid && n_mid > 0 && key == kstar;
-    const uint32_t eqb = __ballot_sync(0xffffffffu, is_eq);
-    const int64_t r = eq_rank + __popc(eqb & ((1u << lane) - 1u));
-    const bool keep =
-        in_range && (!mid || (n_mid > 0 && (key > kstar || (is_eq && r < need_eq))));
-    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-    eq_rank += __popc(eqb);
-    if (lane == 0) flagbits[b >> 5] = kb;
-    cnt += __popc(kb);
+  for (int64_t b0 = s0; b0 < s1; b0 += 32 * kUnroll) {
+    double v[kUnroll];
+#pragma unroll
+    for (int j = 0; j < kUnroll; ++j) {
+      const int64_t t = b0 + 32 * j + lane;
+      v[j] = (t < s1 && t >= lo && t < hi && n_mid > 0) ? __ldg(s + t) : 0.0;
+    }
+#pragma unroll
+    for (int j = 0; j < kUnroll; ++j) {
+      const int64_t b = b0 + 32 * j;
+      if (b >= s1) break;
+      const int64_t t = b + lane;
+      const bool in_range = t < s1;
+      const bool mid = in_range && t >= lo && t < hi;
+      const uint64_t key = mid ? score_key(v[j]) : 0ull;
+      const bool is_eq = mid && n_mid > 0 && key == kstar;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, is_eq);
+      const int64_t r = eq_rank + __popc(eqb & ((1u << lane) - 1u));
+      const bool keep = in_range && (!mid || (n_mid > 0 && (key > kstar ||
+                                                           (is_eq && (!rank_ties || r < need_eq)))));
+      const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+      eq_rank += __popc(eqb);
+      if (lane == 0) flagbits[b >> 5] = kb;
+      cnt += __popc(kb);
+    }
   }
   if (lane == 0) warp_cnt[warp] = cnt;
   __syncthreads();

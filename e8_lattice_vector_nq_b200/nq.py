@@ -305,3 +305,88 @@ class Codec:
         if self.kept is not None:
             b += self.kept.numel() * 4
         return b
+
+
+# ------------------------------------------------------- whole-cache pipelines
+class LayeredCache:
+    """A model's cache [layers][heads][T][128] compressed layer-batched, with
+    boundary layers kept in bf16 (NexusQuant "Implementation details":
+    protect_boundary keeps the first/last layers at full precision).
+
+    The quantised layers must form one contiguous range (they do for
+    protect_boundary).  Protected layers pass through as a bf16 device copy;
+    every quantised layer runs score -> select -> encode through the C ABI."""
+
+    def __init__(self, layers: int, heads: int, T: int, theta: float, bits_k: int = 3,
+                 bits_v: int = 2, window: int = 64, evict_pct: int = 0,
+                 protected: tuple = (), device="cuda"):
+        q = [l for l in range(layers) if l not in set(protected)]
+        if q and q != list(range(q[0], q[-1] + 1)):
+            raise ValueError("quantised layers must be contiguous")
+        self.layers, self.q0, self.q1 = layers, (q[0] if q else 0), (q[-1] + 1 if q else 0)
+        self.protected = tuple(sorted(set(protected)))
+        self.codec = Codec(self.q1 - self.q0, heads, T, theta, bits_k, bits_v, window, evict_pct,
+                           device) if q else None
+        self.kept_bf16_K = {}
+        self.kept_bf16_V = {}
+
+    def encode(self, K: torch.Tensor, V: torch.Tensor, stream=None):
+        for l in self.protected:
+            self.kept_bf16_K[l] = K[l].clone()
+            self.kept_bf16_V[l] = V[l].clone()
+        if self.codec is not None:
+            self.codec.encode(K[self.q0:self.q1], V[self.q0:self.q1], stream)
+
+    def decode_quantised(self, K_out: torch.Tensor, V_out: torch.Tensor, stream=None):
+        """Reconstruct the quantised layers into [q1-q0][heads][n][128] outputs."""
+        self.codec.decode(K_out, V_out, stream)
+
+    @property
+    def stored_bits(self) -> int:
+        b = 0 if self.codec is None else self.codec.packed_bytes * 8
+        for l in self.protected:
+            b += 16 * (self.kept_bf16_K[l].numel() + self.kept_bf16_V[l].numel()) if l in self.kept_bf16_K else 0
+        return b
+
+
+class AppendStore:
+    """Packed caches of many sequences x layers with room to append tokens
+    (the decode-append regime): units = sequences * layers, slot capacity cap.
+    append() encodes one new token per unit at its position (slot = position);
+    decode_layer() reconstructs all tokens of one layer for every sequence."""
+
+    def __init__(self, sequences: int, layers: int, heads: int, cap: int, theta: float,
+                 bits_k: int = 2, bits_v: int = 2, device="cuda"):
+        self.S, self.L, self.H, self.cap = sequences, layers, heads, cap
+        self.bits_k, self.bits_v = bits_k, bits_v
+        self.rope = rope_tables(theta, cap, device)
+        self.k = PackedStore.empty(sequences * layers, heads, cap, bits_k, device)
+        self.v = PackedStore.empty(sequences * layers, heads, cap, bits_v, device)
+
+    def _units(self, store: PackedStore, seq: int | None = None, layer: int | None = None):
+        c = store.codes.view(self.S, self.L, self.H, self.cap, -1)
+        m = store.meta.view(self.S, self.L, self.H, self.cap)
+        if seq is not None:
+            c, m = c[seq:seq + 1], m[seq:seq + 1]
+        if layer is not None:
+            c, m = c[:, layer], m[:, layer]
+        else:
+            c, m = c.reshape(-1, self.H, self.cap, c.shape[-1]), m.reshape(-1, self.H, self.cap)
+        return PackedStore(c, m, store.bits)
+
+    def fill(self, seq: int, K: torch.Tensor, V: torch.Tensor, stream=None):
+        """Encode an initial cache [layers][heads][T0][128] of one sequence at positions 0..T0-1."""
+        n = K.shape[2]
+        nq_encode(K, V, self._units(self.k, seq), self._units(self.v, seq), n, self.rope, self.cap,
+                  stream=stream)
+
+    def append(self, K_new: torch.Tensor, V_new: torch.Tensor, pos: int, stream=None):
+        """K_new/V_new [sequences*layers][heads][1][128]: one token per unit at position pos."""
+        nq_encode(K_new, V_new, self.k, self.v, 1, self.rope, self.cap, pos_base=pos, slot0=pos,
+                  stream=stream)
+
+    def decode_layer(self, layer: int, n: int, K_out: torch.Tensor, V_out: torch.Tensor,
+                     stream=None):
+        """Slots 0..n-1 of `layer` for every sequence into [sequences][heads][n][128]."""
+        nq_decode(self._units(self.k, layer=layer), self._units(self.v, layer=layer), n, K_out,
+                  V_out, self.rope, self.cap, stream=stream)
