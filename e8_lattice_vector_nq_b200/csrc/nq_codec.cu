@@ -18,13 +18,19 @@
 // runs two groups per packed instruction (__fadd2_rn / __ffma2_rn /
 // __fmul2_rn: per-lane IEEE round-to-nearest, the same bits as scalar code).
 // A persistent CTA of HG warps (HG heads) walks tiles of 16 slots x HG heads.
-// Encode stages every input row with a 256-byte bulk async copy (TMA engine,
-// mbarrier completion) into a padded shared-memory row, double buffered, so
-// the loads of tile k+2 overlap the arithmetic of tile k; the RoPE (cos, sin)
-// pairs of a tile are combined once per CTA and shared by its heads.  Decode
-// loads the next tile's codes one tile ahead and writes each reconstructed
-// row through shared memory with a 256-byte bulk async store.  Every
+// Encode stages the input rows with warp-cooperative 16-byte async copies
+// (each warp instruction moves two whole 256-byte rows, gathered through the
+// kept list) into padded shared-memory rows, double buffered, so the loads of
+// tile k+2 overlap the arithmetic of tile k; the RoPE (cos, sin) pairs of a
+// tile are combined once per CTA and shared by its heads.  Decode loads the
+// next tile's codes one tile ahead and writes each warp's 16 reconstructed
+// rows into a 128-byte-swizzled shared tile that one lane stores with two
+// TMA tensor stores (cp.async.bulk.tensor, 4-D map of the output).  Every
 // (bits, RoPE) variant is its own kernel: keys and values are two launches.
+#include <cuda.h>
+
+#include <mutex>
+
 #include "nq_internal.h"
 
 namespace nq {
@@ -332,44 +338,43 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   const int slot_l = lane & 15, half = lane >> 4;
   const int rows_bytes = (nthreads / 2) * kRowPad;
   const int stage_bytes = rows_bytes + (ROPE ? kCsBytes : 0);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * stage_bytes);
   const int row_idx = warp * kSlots + slot_l;  // this vector's staged row
 
   const int64_t first = blockIdx.x, step = gridDim.x;
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
-  if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
 
+  // Stage the warp's 16 rows (one head, 16 slots) with 16-byte async copies:
+  // in copy j, lane l moves chunk l%16 of row 2j + l/16, so each warp
+  // instruction reads two whole 256-byte rows.
   auto issue = [&](int64_t k, int s) {
     const Tile tl = tile_of(a, first + k * step);
     unsigned char* st = smem + s * stage_bytes;
     const int h = tl.group * a.hg + warp;
-    const int64_t slot = tl.stile * kSlots + slot_l;
-    const int64_t valid = min64(kSlots, a.n - tl.stile * kSlots);
-    if (tid == 0) mbar_arrive_expect_tx(&bars[s], static_cast<uint32_t>(valid * a.hg * 256));
-    if (half == 0 && slot < a.n) {
-      int64_t src = slot;
-      if (a.idx) src = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot);
-      src = src < 0 ? 0 : (src >= a.T_in ? a.T_in - 1 : src);
-      const uint16_t* g = a.kv + tl.unit * a.su + h * a.sh + src * a.st;
-      bulk_g2s(st + row_idx * kRowPad, g, 256, &bars[s]);
+    const int64_t my_slot = tl.stile * kSlots + slot_l;
+    int64_t src = my_slot;
+    if (a.idx && my_slot < a.n)
+      src = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + my_slot);
+    src = src < 0 ? 0 : (src >= a.T_in ? a.T_in - 1 : src);
+    const uint16_t* base = a.kv + tl.unit * a.su + h * a.sh + slot_l * 8;
+    const uint32_t dst0 = smem_u32(st + warp * kSlots * kRowPad) + slot_l * 16;
+#pragma unroll
+    for (int j = 0; j < kSlots / 2; ++j) {
+      const int r = 2 * j + half;
+      const int64_t tok = __shfl_sync(0xffffffffu, src, r);
+      if (tl.stile * kSlots + r < a.n) cp_async16(dst0 + r * kRowPad, base + tok * a.st);
     }
     if (ROPE) fill_cs(a, tl, reinterpret_cast<float4*>(st + rows_bytes), tid, nthreads);
   };
 
   if (my_tiles > 0) issue(0, 0);
+  cp_async_commit();
   if (my_tiles > 1) issue(1, 1);
-  __syncthreads();
+  cp_async_commit();
 
   for (int64_t k = 0; k < my_tiles; ++k) {
     const int s = static_cast<int>(k & 1);
-    const uint32_t parity = static_cast<uint32_t>((k >> 1) & 1);
-    const bool ok = mbar_wait_bounded(&bars[s], parity);
-    if (!__syncthreads_and(ok)) return;  // a copy never landed: error word set, stop
+    cp_async_wait<1>();  // this thread's copies of tile k have landed
+    __syncthreads();     // ... and everyone's (plus the tile's RoPE pairs)
 
     const Tile tl = tile_of(a, first + k * step);
     const int h = tl.group * a.hg + warp;
@@ -386,9 +391,11 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
     }
     __syncthreads();  // everyone is done with stage s
     if (k + 2 < my_tiles) issue(k + 2, s);
+    cp_async_commit();  // one group per iteration keeps the wait count uniform
     const int64_t vec = tl.unit * a.pu + h * a.ph + a.slot0 + slot;
     quantise_half<BITS>(v, half, valid, a.codes + vec * (4 * BITS), a.meta + vec);
   }
+  cp_async_wait<0>();
 }
 
 // --------------------------------------------------------------- decode
@@ -414,7 +421,7 @@ __device__ __forceinline__ float code_as_float(const uint32_t (&w)[BITS], int c)
 
 template <int BITS, bool ROPE>
 __device__ __forceinline__ void decode_half(const uint32_t (&w)[4 * BITS], uint32_t meta,
-                                            uint32_t csa, uint32_t row, int half) {
+                                            uint32_t csa, uint32_t row, int rsw, int half) {
   // This half's blocks: coordinates [32h, 32h+32) and [64+32h, 96+32h), each
   // BITS words starting at word BITS*h and BITS*(2+h).
   uint32_t wa[BITS], wb[BITS];
@@ -469,8 +476,10 @@ __device__ __forceinline__ void decode_half(const uint32_t (&w)[4 * BITS], uint3
       A[t] = *reinterpret_cast<const uint32_t*>(&pa);
       B[t] = *reinterpret_cast<const uint32_t*>(&pb);
     }
-    sts128(row + 16 * (4 * half + q), make_uint4(A[0], A[1], A[2], A[3]));
-    sts128(row + 16 * (8 + 4 * half + q), make_uint4(B[0], B[1], B[2], B[3]));
+    // chunk 4h+q of columns 0-63 and of columns 64-127, swizzled by row % 8
+    const uint32_t cc = static_cast<uint32_t>(((4 * half + q) ^ rsw) << 4);
+    sts128(row + cc, make_uint4(A[0], A[1], A[2], A[3]));
+    sts128(row + kSlots * 128 + cc, make_uint4(B[0], B[1], B[2], B[3]));
   }
 }
 
@@ -496,16 +505,23 @@ __device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int wa
   }
 }
 
+// Output tile of one warp: 16 rows x 256 bytes as two 16 x 128-byte boxes
+// (columns 0-63 and 64-127) in the 128-byte swizzled layout of the tensor
+// store: 16-byte chunk c of row r sits at chunk (c ^ (r % 8)) of its box row.
+constexpr int kOutTileBytes = 2 * kSlots * 128;
+
 template <int BITS, bool ROPE>
-__global__ void __launch_bounds__(256, 2) decode_kernel(const CodecArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
+__global__ void __launch_bounds__(256, 2)
+    decode_kernel(const CodecArgs a, const __grid_constant__ CUtensorMap out_map) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the swizzled tiles need a 1024-byte aligned base (1 KB of slack is allocated)
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int nthreads = blockDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int slot_l = lane & 15, half = lane >> 4;
-  unsigned char* out_rows = smem;
-  unsigned char* cs_base = smem + (nthreads / 2) * kRowPad;  // two cs buffers, kCsBytes each
-  const int row_idx = warp * kSlots + slot_l;
-  const uint32_t row = smem_u32(out_rows + row_idx * kRowPad);
+  const int nwarps = nthreads / 32;
+  const uint32_t tile_base = smem_u32(smem) + warp * kOutTileBytes;
+  unsigned char* cs_base = smem + nwarps * kOutTileBytes;  // two cs buffers, kCsBytes each
 
   const int64_t first = blockIdx.x, step = gridDim.x;
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
@@ -528,29 +544,29 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(const CodecArgs a) {
   for (int64_t k = 0; k < my_tiles; ++k) {
     const Tile tl = tile_of(a, first + k * step);
     const int h = tl.group * a.hg + warp;
-    const int64_t slot = tl.stile * kSlots + slot_l;
     uint32_t wc[4 * BITS];
 #pragma unroll
     for (int i = 0; i < 4 * BITS; ++i) wc[i] = w[i];
     const uint32_t mc = meta;
     if (k + 1 < my_tiles) load_codes<BITS>(a, first + (k + 1) * step, warp, slot_l, w, meta);
-    const bool valid = slot < a.n;
-    // the row's previous bulk store (issued by half 0) has finished reading smem
-    if (half == 0) bulk_wait_read_all();
+    // the warp's previous tensor store has finished reading the tile
+    if (lane == 0) bulk_wait_read_all();
     __syncwarp();
     const uint32_t csa = smem_u32(cs_base + (k & 1) * kCsBytes) + (16 * half * kSlots + slot_l) * 16;
-    decode_half<BITS, ROPE>(wc, mc, csa, row, half);
+    decode_half<BITS, ROPE>(wc, mc, csa, tile_base + slot_l * 128, slot_l & 7, half);
     fence_proxy_async_smem();
     __syncwarp();
-    if (valid && half == 0) {
-      uint16_t* dst = const_cast<uint16_t*>(a.kv) + tl.unit * a.su + h * a.sh + slot * a.st;
-      bulk_s2g(dst, out_rows + row_idx * kRowPad, 256);
+    if (lane == 0) {
+      // rows past n are clipped by the tensor map (its token extent is n)
+      const int y = static_cast<int>(tl.stile * kSlots);
+      tma_store_4d(&out_map, tile_base, 0, y, h, tl.unit);
+      tma_store_4d(&out_map, tile_base + kSlots * 128, 64, y, h, tl.unit);
       bulk_commit();
     }
     if (k + 1 < my_tiles) prep_cs(k + 1, static_cast<int>((k + 1) & 1));
     __syncthreads();
   }
-  bulk_wait_all();
+  if (lane == 0) bulk_wait_all();
 }
 
 // ---------------------------------------------------------------- launch
@@ -558,6 +574,48 @@ static int pick_head_group(int heads) {
   for (int g = 8; g >= 1; --g)
     if (heads % g == 0) return g;
   return 1;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D map of a bf16 [units][heads][n][128] output: boxes of 64 coordinates x
+// 16 tokens, 128-byte swizzle.  Strides in bytes; a unit dimension of extent
+// 1 may carry any stride, so it is given a valid one.
+static cudaError_t make_out_map(CUtensorMap* m, const CodecArgs& a, int units) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const uint64_t st = static_cast<uint64_t>(a.st) * 2;
+  uint64_t sh = static_cast<uint64_t>(a.sh) * 2, su = static_cast<uint64_t>(a.su) * 2;
+  if (a.heads == 1 || sh == 0) sh = st * static_cast<uint64_t>(a.n);
+  if (units == 1 || su == 0) su = sh * static_cast<uint64_t>(a.heads);
+  cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(a.n), static_cast<cuuint64_t>(a.heads),
+                        static_cast<cuuint64_t>(units)};
+  cuuint64_t strides[3] = {st, sh, su};
+  cuuint32_t box[4] = {64, kSlots, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(a.kv), dims,
+                  strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int BITS, bool ROPE>
@@ -574,11 +632,14 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   const int rows_bytes = (threads / 2) * kRowPad;
   size_t smem;
   const void* fn;
+  CUtensorMap map;
   if (decode) {
-    smem = static_cast<size_t>(rows_bytes) + (ROPE ? 2 * kCsBytes : 0);
+    cudaError_t e = make_out_map(&map, a, units);
+    if (e != cudaSuccess) return e;
+    smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes + (ROPE ? 2 * kCsBytes : 0);
     fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE>);
   } else {
-    smem = 2 * (static_cast<size_t>(rows_bytes) + (ROPE ? kCsBytes : 0)) + 16;
+    smem = 2 * (static_cast<size_t>(rows_bytes) + (ROPE ? kCsBytes : 0));
     fn = reinterpret_cast<const void*>(encode_kernel<BITS, ROPE>);
   }
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -594,7 +655,7 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   if (per_sm < 1) per_sm = 1;
   const int64_t grid = min64(a.num_tiles, static_cast<int64_t>(sms) * per_sm);
   if (decode)
-    decode_kernel<BITS, ROPE><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
+    decode_kernel<BITS, ROPE><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a, map);
   else
     encode_kernel<BITS, ROPE><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
   return cudaGetLastError();
