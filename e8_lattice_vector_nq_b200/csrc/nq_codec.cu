@@ -94,37 +94,52 @@ __device__ __forceinline__ Tile tile_of(const CodecArgs& a, int64_t t64) {
   return r;
 }
 
-// cs table of one tile: float4 cs[j][slot] = (c_2j, s_2j, c_2j+1, s_2j+1) at
-// that slot's RoPE position; a thread of half h reads j in [16h, 16h+16).
-// Thread t fills slot t % 16 for j = t/16, t/16 + nthreads/16, ... : one
-// position lookup, then two table rows read at consecutive frequencies.
-__device__ __forceinline__ void fill_cs(const CodecArgs& a, const Tile& tl, float4* cs, int tid,
-                                        int nthreads) {
-  const int slot_l = tid % kSlots;
+// Source token of this lane's slot (lanes l and l+16 share slot l % 16) in
+// tile tl: the kept-list entry, or the slot itself; -1 past the last slot.
+__device__ __forceinline__ int32_t slot_src(const CodecArgs& a, const Tile& tl, int slot_l) {
   const int64_t slot = tl.stile * kSlots + slot_l;
-  const float2* rowA = a.tab;
-  const float2* rowB = a.tab + a.n_a * kHalf;
-  if (slot < a.n) {
-    int64_t p = slot;
-    if (a.idx) p = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot);
-    p += a.pos_base;
-    int64_t hi = p >> 8;
+  if (slot >= a.n) return -1;
+  return a.idx ? __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot)
+               : static_cast<int32_t>(slot);
+}
+
+// RoPE table rows of a tile, staged raw: for each of the 16 slots the A row
+// (angle 256a) and the B row (angle b) of its position p = 256a + b, 512
+// bytes each, at a padded stride of kRawSlot bytes per slot.
+constexpr int kRawSlot = 1024 + 16;
+constexpr int kRawBytes = kSlots * kRawSlot;
+
+__device__ __forceinline__ void issue_raw(const CodecArgs& a, int32_t src_lane, uint32_t raw,
+                                          int tid, int nthreads) {
+  // 1024 16-byte chunks; every warp runs the same number of iterations
+  for (int c = tid; c < kSlots * 64; c += nthreads) {
+    const int slot = c >> 6;
+    const int32_t src = __shfl_sync(0xffffffffu, src_lane, slot);
+    if (src < 0) continue;
+    const int64_t pos = a.pos_base + src;
+    int64_t hi = pos >> 8;
     hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
-    rowA = a.tab + hi * kHalf;
-    rowB = a.tab + (a.n_a + (p & 255)) * kHalf;
+    const int which = (c >> 5) & 1, part = c & 31;
+    const float2* row = which ? a.tab + (a.n_a + (pos & 255)) * kHalf : a.tab + hi * kHalf;
+    cp_async16(raw + slot * kRawSlot + which * 512 + part * 16,
+               reinterpret_cast<const char*>(row) + part * 16);
   }
-  for (int j = tid / kSlots; j < 32; j += nthreads / kSlots) {
-    float4 v = make_float4(1.f, 0.f, 1.f, 0.f);
-    if (slot < a.n) {
-      const float4 A = __ldg(reinterpret_cast<const float4*>(rowA + 2 * j));
-      const float4 B = __ldg(reinterpret_cast<const float4*>(rowB + 2 * j));
-      // c = fmaf(cA, cB, -(sA sB)),  s = fmaf(sA, cB, cA sB)
-      v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
-      v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
-      v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
-      v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
-    }
-    cs[j * kSlots + slot_l] = v;
+}
+
+// cs table of one tile: float4 cs[j][slot] = (c_2j, s_2j, c_2j+1, s_2j+1),
+// c = fmaf(cA, cB, -(sA sB)), s = fmaf(sA, cB, cA sB); a thread of half h
+// later reads j in [16h, 16h+16).
+__device__ __forceinline__ void combine_raw(uint32_t raw, float4* cs, int tid, int nthreads) {
+  for (int e = tid; e < 32 * kSlots; e += nthreads) {
+    const int slot = e & 15, j = e >> 4;
+    const float4 A = lds128f(raw + slot * kRawSlot + j * 16);
+    const float4 B = lds128f(raw + slot * kRawSlot + 512 + j * 16);
+    float4 v;
+    v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
+    v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
+    v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
+    v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
+    cs[j * kSlots + slot] = v;
   }
 }
 
@@ -171,30 +186,36 @@ __device__ __forceinline__ void fwht_half(float2 (&v)[32], int half) {
 // coordinate toward u); the half coset wins only when strictly closer.
 // Returns the clamped b-bit codes of each lane packed as code i at bits
 // [BITS*i, BITS*i + BITS), and the coset bit of each lane.
-template <int BITS>
-__device__ __forceinline__ void e8_pair(const float2 (&y)[8], uint32_t& gx, uint32_t& gy,
-                                        uint32_t& hx, uint32_t& hy) {
+// Decision half of the decoder for two groups (lanes x, y): returns, per
+// lane, whether the half coset wins, whether its coordinate sum was odd (a
+// fix is needed) and the largest rounding error of the chosen coset.
+struct E8Choice {
+  float2 hh;     // 1 for the half coset, 0 for the integer coset
+  float mx, my;  // largest |e| of the chosen coset
+  bool oddx, oddy;
+};
+
+__device__ __forceinline__ E8Choice e8_decide(const float2 (&y)[8]) {
   const float2 M2 = make_float2(kMagicRound, kMagicRound);
   const float2 H2 = make_float2(0.5f, 0.5f);
-  float2 e0[8], e1[8];
   float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
   float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);  // sums of f (exact)
   float m0x = 0.f, m0y = 0.f, m1x = 0.f, m1y = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float2 f0 = sub2(add2(y[i], M2), M2);
-    e0[i] = sub2(y[i], f0);
+    const float2 e0 = sub2(y[i], f0);
     const float2 u = sub2(y[i], H2);
     const float2 f1 = sub2(add2(u, M2), M2);
-    e1[i] = sub2(u, f1);
+    const float2 e1 = sub2(u, f1);
     s0 = add2(s0, f0);
     s1 = add2(s1, f1);
-    d0 = i == 0 ? mul2(e0[i], e0[i]) : fma2(e0[i], e0[i], d0);
-    d1 = i == 0 ? mul2(e1[i], e1[i]) : fma2(e1[i], e1[i], d1);
-    m0x = fmaxf(m0x, fabsf(e0[i].x));
-    m0y = fmaxf(m0y, fabsf(e0[i].y));
-    m1x = fmaxf(m1x, fabsf(e1[i].x));
-    m1y = fmaxf(m1y, fabsf(e1[i].y));
+    d0 = i == 0 ? mul2(e0, e0) : fma2(e0, e0, d0);
+    d1 = i == 0 ? mul2(e1, e1) : fma2(e1, e1, d1);
+    m0x = fmaxf(m0x, fabsf(e0.x));
+    m0y = fmaxf(m0y, fabsf(e0.y));
+    m1x = fmaxf(m1x, fabsf(e1.x));
+    m1y = fmaxf(m1y, fabsf(e1.y));
   }
   // parity of an integer-valued sum: the LSB of its 1.5*2^23-biased bits
   const float2 b0 = add2(s0, M2), b1 = add2(s1, M2);
@@ -206,42 +227,69 @@ __device__ __forceinline__ void e8_pair(const float2 (&y)[8], uint32_t& gx, uint
   const float D0x = o0x ? fix0.x : d0.x, D0y = o0y ? fix0.y : d0.y;
   const float D1x = o1x ? fix1.x : d1.x, D1y = o1y ? fix1.y : d1.y;
   const bool halfx = D1x < D0x, halfy = D1y < D0y;
-  hx = halfx;
-  hy = halfy;
+  E8Choice c;
+  c.hh = make_float2(halfx ? 1.f : 0.f, halfy ? 1.f : 0.f);
+  c.mx = halfx ? m1x : m0x;
+  c.my = halfy ? m1y : m0y;
+  c.oddx = halfx ? o1x : o0x;
+  c.oddy = halfy ? o1y : o0y;
+  return c;
+}
 
-  // chosen coset per lane: residual E, shifted input U, rounded F = U - E
-  const float2 hh = make_float2(halfx ? 1.f : 0.f, halfy ? 1.f : 0.f);
-  const float mx = halfx ? m1x : m0x, my = halfy ? m1y : m0y;
-  bool fx = !(halfx ? o1x : o0x), fy = !(halfy ? o1y : o0y);  // "fix done" flags
+// Code half of the decoder for two pairs of groups at once (four
+// independent fix chains): the chosen coset's rounding is recomputed
+// (U = y - shift, F = rint(U), E = U - F), the first coordinate with
+// |E| = m moves one step toward U when the sum was odd, then F is clamped
+// to the b-bit range and packed (code i at bits [BITS*i, BITS*i + BITS)).
+template <int BITS>
+__device__ __forceinline__ void e8_codes2(const float2 (&ya)[8], const float2 (&yb)[8],
+                                          const E8Choice& ca, const E8Choice& cb,
+                                          uint32_t (&g)[4]) {
+  const float2 M2 = make_float2(kMagicRound, kMagicRound);
   constexpr float kOffH = static_cast<float>(1 << (BITS - 1)) + kTwo23;
   constexpr float kOffI = static_cast<float>((1 << (BITS - 1)) - 1) + kTwo23;
   constexpr float kLoH = -static_cast<float>(1 << (BITS - 1));
-  constexpr float kHiH = static_cast<float>((1 << (BITS - 1)) - 1);
   constexpr float kLoI = -static_cast<float>((1 << (BITS - 1)) - 1);
-  constexpr float kHiI = static_cast<float>((1 << (BITS - 1)) - 1);
-  const float2 off = make_float2(halfx ? kOffH : kOffI, halfy ? kOffH : kOffI);
-  const float lox = halfx ? kLoH : kLoI, loy = halfy ? kLoH : kLoI;
-  const float hix = halfx ? kHiH : kHiI, hiy = halfy ? kHiH : kHiI;
-  uint32_t ax = 0, ay = 0;
+  constexpr float kHi = static_cast<float>((1 << (BITS - 1)) - 1);
+  const E8Choice* cc[2] = {&ca, &cb};
+  float2 off[2], lo[2];
+  bool fx[2], fy[2];
+  uint32_t ax[2] = {0u, 0u}, ay[2] = {0u, 0u};
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const E8Choice& c = *cc[p];
+    off[p] = make_float2(c.hh.x != 0.f ? kOffH : kOffI, c.hh.y != 0.f ? kOffH : kOffI);
+    lo[p] = make_float2(c.hh.x != 0.f ? kLoH : kLoI, c.hh.y != 0.f ? kLoH : kLoI);
+    fx[p] = !c.oddx;  // "fix done" flags
+    fy[p] = !c.oddy;
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float2 E = make_float2(halfx ? e1[i].x : e0[i].x, halfy ? e1[i].y : e0[i].y);
-    const float2 U = fma2(hh, make_float2(-0.5f, -0.5f), y[i]);
-    float2 F = sub2(U, E);
-    const bool hitx = !fx && fabsf(E.x) == mx;
-    const bool hity = !fy && fabsf(E.y) == my;
-    fx = fx || hitx;
-    fy = fy || hity;
-    // E is never -0 (y carries no -0), so its sign bit decides the direction
-    if (hitx) F.x = __fadd_rn(F.x, copysignf(1.0f, E.x));
-    if (hity) F.y = __fadd_rn(F.y, copysignf(1.0f, E.y));
-    F = make_float2(fminf(fmaxf(F.x, lox), hix), fminf(fmaxf(F.y, loy), hiy));
-    const float2 J = add2(F, off);  // 2^23 + code: the code sits in the low mantissa bits
-    ax += __float_as_uint(J.x) << (BITS * i);
-    ay += __float_as_uint(J.y) << (BITS * i);
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      const E8Choice& c = *cc[p];
+      const float2 yy = p ? yb[i] : ya[i];
+      const float2 U = fma2(c.hh, make_float2(-0.5f, -0.5f), yy);
+      float2 F = sub2(add2(U, M2), M2);
+      const float2 E = sub2(U, F);
+      const bool hitx = !fx[p] && fabsf(E.x) == c.mx;
+      const bool hity = !fy[p] && fabsf(E.y) == c.my;
+      fx[p] = fx[p] || hitx;
+      fy[p] = fy[p] || hity;
+      // E is never -0 (y carries no -0), so its sign bit decides the direction
+      if (hitx) F.x = __fadd_rn(F.x, copysignf(1.0f, E.x));
+      if (hity) F.y = __fadd_rn(F.y, copysignf(1.0f, E.y));
+      F = make_float2(fminf(fmaxf(F.x, lo[p].x), kHi), fminf(fmaxf(F.y, lo[p].y), kHi));
+      const float2 J = add2(F, off[p]);  // 2^23 + code: the code sits in the low mantissa bits
+      ax[p] += __float_as_uint(J.x) << (BITS * i);
+      ay[p] += __float_as_uint(J.y) << (BITS * i);
+    }
   }
-  gx = ax & ((1u << (8 * BITS)) - 1u);
-  gy = ay & ((1u << (8 * BITS)) - 1u);
+  constexpr uint32_t kMask = (1u << (8 * BITS)) - 1u;
+  g[0] = ax[0] & kMask;
+  g[1] = ay[0] & kMask;
+  g[2] = ax[1] & kMask;
+  g[3] = ay[1] & kMask;
 }
 
 // --------------------------------------------------------------- encode
@@ -293,13 +341,25 @@ __device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool va
   uint32_t gx[4], gy[4];
   uint32_t cm = 0;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    float2 y[8];
+  for (int q = 0; q < 4; q += 2) {
+    float2 ya[8], yb[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = add2(mul2(v[8 * q + i], r2), make_float2(0.f, 0.f));
-    uint32_t hx, hy;
-    e8_pair<BITS>(y, gx[q], gy[q], hx, hy);
-    cm |= (hx << (4 * half + q)) | (hy << (8 + 4 * half + q));
+    for (int i = 0; i < 8; ++i) {
+      ya[i] = add2(mul2(v[8 * q + i], r2), make_float2(0.f, 0.f));
+      yb[i] = add2(mul2(v[8 * (q + 1) + i], r2), make_float2(0.f, 0.f));
+    }
+    const E8Choice ca = e8_decide(ya);
+    const E8Choice cb = e8_decide(yb);
+    uint32_t g[4];
+    e8_codes2<BITS>(ya, yb, ca, cb, g);
+    gx[q] = g[0];
+    gy[q] = g[1];
+    gx[q + 1] = g[2];
+    gy[q + 1] = g[3];
+    cm |= ((ca.hh.x != 0.f ? 1u : 0u) << (4 * half + q)) |
+          ((ca.hh.y != 0.f ? 1u : 0u) << (8 + 4 * half + q)) |
+          ((cb.hh.x != 0.f ? 1u : 0u) << (4 * half + q + 1)) |
+          ((cb.hh.y != 0.f ? 1u : 0u) << (8 + 4 * half + q + 1));
   }
   cm |= __shfl_xor_sync(0xffffffffu, cm, 16);
   if (!valid) return;
@@ -338,45 +398,70 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   const int slot_l = lane & 15, half = lane >> 4;
   const int rows_bytes = (nthreads / 2) * kRowPad;
   const int stage_bytes = rows_bytes + (ROPE ? kCsBytes : 0);
-  const int row_idx = warp * kSlots + slot_l;  // this vector's staged row
+  const uint32_t raw = smem_u32(smem + 2 * stage_bytes);  // RoPE rows of the next tile
+  const int row_idx = warp * kSlots + slot_l;             // this vector's staged row
 
   const int64_t first = blockIdx.x, step = gridDim.x;
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
+  auto tile = [&](int64_t k) { return tile_of(a, first + k * step); };
 
-  // Stage the warp's 16 rows (one head, 16 slots) with 16-byte async copies:
-  // in copy j, lane l moves chunk l%16 of row 2j + l/16, so each warp
-  // instruction reads two whole 256-byte rows.
-  auto issue = [&](int64_t k, int s) {
-    const Tile tl = tile_of(a, first + k * step);
-    unsigned char* st = smem + s * stage_bytes;
+  // The warp's 16 rows (one head, 16 slots) with 16-byte async copies: in copy
+  // j, lane l moves chunk l%16 of row 2j + l/16, two whole rows per instruction.
+  auto issue_rows = [&](const Tile& tl, int32_t src_lane, int s) {
     const int h = tl.group * a.hg + warp;
-    const int64_t my_slot = tl.stile * kSlots + slot_l;
-    int64_t src = my_slot;
-    if (a.idx && my_slot < a.n)
-      src = __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + my_slot);
-    src = src < 0 ? 0 : (src >= a.T_in ? a.T_in - 1 : src);
     const uint16_t* base = a.kv + tl.unit * a.su + h * a.sh + slot_l * 8;
-    const uint32_t dst0 = smem_u32(st + warp * kSlots * kRowPad) + slot_l * 16;
+    const uint32_t dst0 = smem_u32(smem + s * stage_bytes + warp * kSlots * kRowPad) + slot_l * 16;
 #pragma unroll
     for (int j = 0; j < kSlots / 2; ++j) {
       const int r = 2 * j + half;
-      const int64_t tok = __shfl_sync(0xffffffffu, src, r);
-      if (tl.stile * kSlots + r < a.n) cp_async16(dst0 + r * kRowPad, base + tok * a.st);
+      const int32_t tok = __shfl_sync(0xffffffffu, src_lane, r);
+      if (tok >= 0) {
+        const int64_t t = tok < a.T_in ? tok : a.T_in - 1;
+        cp_async16(dst0 + r * kRowPad, base + t * a.st);
+      }
     }
-    if (ROPE) fill_cs(a, tl, reinterpret_cast<float4*>(st + rows_bytes), tid, nthreads);
+  };
+  // cross-warp data (the shared RoPE table) needs the CTA barrier; value
+  // tiles only touch the warp's own rows
+  auto sync = [&]() {
+    if (ROPE) __syncthreads();
+    else __syncwarp();
   };
 
-  if (my_tiles > 0) issue(0, 0);
+  // prologue: tile 0 (rows + its RoPE table), then tile 1 in flight
+  int32_t src_pref = -1;
+  if (my_tiles > 0) {
+    const Tile t0 = tile(0);
+    const int32_t s0 = slot_src(a, t0, slot_l);
+    if (ROPE) issue_raw(a, s0, raw, tid, nthreads);
+    issue_rows(t0, s0, 0);
+  }
   cp_async_commit();
-  if (my_tiles > 1) issue(1, 1);
-  cp_async_commit();
+  cp_async_wait<0>();
+  sync();
+  if (ROPE && my_tiles > 0) combine_raw(raw, reinterpret_cast<float4*>(smem + rows_bytes), tid, nthreads);
+  sync();
+  if (my_tiles > 1) {
+    const Tile t1 = tile(1);
+    const int32_t s1 = slot_src(a, t1, slot_l);
+    if (ROPE) issue_raw(a, s1, raw, tid, nthreads);
+    cp_async_commit();
+    issue_rows(t1, s1, 1);
+    cp_async_commit();
+  } else {
+    cp_async_commit();
+    cp_async_commit();
+  }
+  if (my_tiles > 2) src_pref = slot_src(a, tile(2), slot_l);
 
+  // Per iteration two groups are committed, [RoPE rows of k+2] then [rows of
+  // k+2]; waiting for all but the newest leaves only rows(k+1) in flight.
   for (int64_t k = 0; k < my_tiles; ++k) {
     const int s = static_cast<int>(k & 1);
-    cp_async_wait<1>();  // this thread's copies of tile k have landed
-    __syncthreads();     // ... and everyone's (plus the tile's RoPE pairs)
+    cp_async_wait<1>();
+    sync();
 
-    const Tile tl = tile_of(a, first + k * step);
+    const Tile tl = tile(k);
     const int h = tl.group * a.hg + warp;
     const int64_t slot = tl.stile * kSlots + slot_l;
     const bool valid = slot < a.n;
@@ -389,9 +474,20 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = make_float2(0.f, 0.f);
     }
-    __syncthreads();  // everyone is done with stage s
-    if (k + 2 < my_tiles) issue(k + 2, s);
-    cp_async_commit();  // one group per iteration keeps the wait count uniform
+    if (ROPE && k + 1 < my_tiles)  // RoPE table of tile k+1 into the other stage
+      combine_raw(raw, reinterpret_cast<float4*>(smem + (s ^ 1) * stage_bytes + rows_bytes), tid,
+                  nthreads);
+    sync();  // stage s and the raw rows are free
+    if (k + 2 < my_tiles) {
+      if (ROPE) issue_raw(a, src_pref, raw, tid, nthreads);
+      cp_async_commit();
+      issue_rows(tile(k + 2), src_pref, s);
+      cp_async_commit();
+      if (k + 3 < my_tiles) src_pref = slot_src(a, tile(k + 3), slot_l);  // used next iteration
+    } else {
+      cp_async_commit();
+      cp_async_commit();
+    }
     const int64_t vec = tl.unit * a.pu + h * a.ph + a.slot0 + slot;
     quantise_half<BITS>(v, half, valid, a.codes + vec * (4 * BITS), a.meta + vec);
   }
@@ -530,19 +626,27 @@ __global__ void __launch_bounds__(256, 2)
   uint32_t meta = 0;
 #pragma unroll
   for (int i = 0; i < 4 * BITS; ++i) w[i] = 0;
-  auto prep_cs = [&](int64_t k, int b) {
-    if (ROPE)
-      fill_cs(a, tile_of(a, first + k * step), reinterpret_cast<float4*>(cs_base + b * kCsBytes),
-              tid, nthreads);
-  };
+  const uint32_t raw = smem_u32(cs_base + 2 * kCsBytes);  // RoPE rows of the next tile
+  auto tile = [&](int64_t k) { return tile_of(a, first + k * step); };
+  auto cs_of = [&](int b) { return reinterpret_cast<float4*>(cs_base + b * kCsBytes); };
 
-  if (my_tiles > 0) {
-    prep_cs(0, 0);
-    load_codes<BITS>(a, first, warp, slot_l, w, meta);
+  // prologue: RoPE table of tile 0, codes of tile 0, table rows of tile 1 in flight
+  int32_t src_pref = -1;
+  if (ROPE) {
+    if (my_tiles > 0) issue_raw(a, slot_src(a, tile(0), slot_l), raw, tid, nthreads);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    if (my_tiles > 0) combine_raw(raw, cs_of(0), tid, nthreads);
+    __syncthreads();
+    if (my_tiles > 1) issue_raw(a, slot_src(a, tile(1), slot_l), raw, tid, nthreads);
+    cp_async_commit();
+    if (my_tiles > 2) src_pref = slot_src(a, tile(2), slot_l);
   }
-  __syncthreads();
+  if (my_tiles > 0) load_codes<BITS>(a, first, warp, slot_l, w, meta);
+
   for (int64_t k = 0; k < my_tiles; ++k) {
-    const Tile tl = tile_of(a, first + k * step);
+    const Tile tl = tile(k);
     const int h = tl.group * a.hg + warp;
     uint32_t wc[4 * BITS];
 #pragma unroll
@@ -563,8 +667,16 @@ __global__ void __launch_bounds__(256, 2)
       tma_store_4d(&out_map, tile_base + kSlots * 128, 64, y, h, tl.unit);
       bulk_commit();
     }
-    if (k + 1 < my_tiles) prep_cs(k + 1, static_cast<int>((k + 1) & 1));
-    __syncthreads();
+    if (ROPE) {
+      // table of tile k+1 from the rows fetched during tile k-1; then fetch k+2
+      cp_async_wait<0>();
+      __syncthreads();  // everyone's rows landed, everyone is done with cs[(k+1)&1]
+      if (k + 1 < my_tiles) combine_raw(raw, cs_of(static_cast<int>((k + 1) & 1)), tid, nthreads);
+      __syncthreads();  // table ready, raw rows free
+      if (k + 2 < my_tiles) issue_raw(a, src_pref, raw, tid, nthreads);
+      cp_async_commit();
+      if (k + 3 < my_tiles) src_pref = slot_src(a, tile(k + 3), slot_l);
+    }
   }
   if (lane == 0) bulk_wait_all();
 }
@@ -636,10 +748,11 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   if (decode) {
     cudaError_t e = make_out_map(&map, a, units);
     if (e != cudaSuccess) return e;
-    smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes + (ROPE ? 2 * kCsBytes : 0);
+    smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes +
+           (ROPE ? 2 * kCsBytes + kRawBytes : 0);
     fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE>);
   } else {
-    smem = 2 * (static_cast<size_t>(rows_bytes) + (ROPE ? kCsBytes : 0));
+    smem = 2 * (static_cast<size_t>(rows_bytes) + (ROPE ? kCsBytes : 0)) + (ROPE ? kRawBytes : 0);
     fn = reinterpret_cast<const void*>(encode_kernel<BITS, ROPE>);
   }
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
