@@ -1,6 +1,6 @@
 // nq_device.cuh -- device-side helpers shared by the libnq kernels (sm_100a):
-// bulk-copy (TMA, non-tensor) and mbarrier wrappers in inline PTX, bounded
-// waits, bf16 unpacking, packed fp32x2 arithmetic and the shared error word.
+// cp.async, bulk and TMA tensor copies in inline PTX, bf16 unpacking, packed
+// fp32x2 arithmetic and the device error word.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -23,8 +23,8 @@ constexpr uint32_t kG2Bits = 0x3D715BEFu;
 constexpr float kMagicRound = 12582912.0f;  // 1.5 * 2^23: x + M - M = rint(x) for |x| < 2^22
 constexpr float kTwo23 = 8388608.0f;        // 2^23: bits(2^23 + j) = 0x4B000000 | j
 
-// Device error word of this translation unit: bit 0 = a bounded wait on a
-// bulk copy gave up.  Read and cleared through the ABI (nq_device_error).
+// Device error word of this translation unit, reserved for in-kernel
+// failure reports; read and cleared through the ABI (nq_device_error).
 static __device__ unsigned int g_nq_error;
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -33,67 +33,7 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// ---------------------------------------------------------------- mbarrier
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase with the given parity to complete; give up after about
-// one second, set the device error word and return false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > 1000000000ull) {
-      atomicOr(&g_nq_error, 1u);
-      return false;
-    }
-  }
-}
-
 // ------------------------------------------------------- bulk async copies
-// global -> shared, completion counted on an mbarrier (bytes % 16 == 0,
-// both addresses 16-byte aligned).
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // shared -> global, tracked by this thread's bulk groups.
 __device__ __forceinline__ void bulk_s2g(void* gmem_dst, const void* smem_src, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),

@@ -31,9 +31,10 @@
  * - Inputs must be finite with |x| <= 2^30; other values are out of
  *   contract (no fault: the kernels stay within their buffers, the codes of
  *   such a vector are unspecified).
- * - Kernels with bounded waits (mbarrier completion of bulk copies) give up
- *   after about one second and set a device error word that
- *   nq_device_error() reads; they never spin forever.
+ * - No kernel spin-waits: staging uses cp.async groups and bulk-copy groups,
+ *   whose waits complete in hardware.  nq_device_error() reads the device
+ *   error word reserved for in-kernel failure reports (no current kernel
+ *   sets it, so it reads 0 after any sequence of valid calls).
  */
 #ifndef NQ_H
 #define NQ_H
@@ -209,9 +210,9 @@ nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int
                     nq_kv_strides kos, void *V_out, nq_kv_strides vos, nq_stream_t stream);
 
 /* -------------------------------------------------------------- status
- * Reads and clears the device error word that kernels set when a bounded
- * wait gave up (bit 0: bulk-copy completion timed out).  Synchronises the
- * current device.  Returns NQ_ERR_CUDA if the read itself failed. */
+ * Reads and clears the device error word reserved for in-kernel failure
+ * reports (bit 0: an asynchronous copy did not complete).  Synchronises the
+ * current device, so a pending launch error surfaces here as NQ_ERR_CUDA. */
 nq_status nq_device_error(uint32_t *flags_out);
 
 #ifdef __cplusplus
