@@ -153,6 +153,15 @@ def dist_setup(args):
     return world, rank, local
 
 
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank's device-timed duration, max-reduced."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def build_workload(args):
     wl = synth.WORKLOADS[args.workload]
     kw = {}
@@ -321,11 +330,8 @@ def run_ours(args, world, rank, local):
         per_stage["select"] = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     per_stage["encode"] = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
     per_stage["decode"] = sum(e[3].elapsed_time(e[4]) for e in evs) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    assert nq.device_error() == 0, "a kernel reported a bounded-wait timeout"
+    ms = max_over_ranks(ms, world, device)
+    assert nq.device_error() == 0, "a kernel reported an in-kernel failure"
 
     in_bytes = K.numel() * 2 + V.numel() * 2
     ms_step = ms / args.steps
@@ -404,11 +410,7 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
         step()
     e.record(stream)
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([ms], device=K.device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, world, K.device)
     return {"value": world * in_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": Kd.numel() * 2 + Vd.numel() * 2,
             "ms_per_step": ms, "steps": args.e2e_steps}
