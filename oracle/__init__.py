@@ -55,7 +55,8 @@ def _load():
     with _lock:
         if _lib is not None:
             return _lib
-        lib = ctypes.CDLL(build())
+        # NQ_ORACLE_SO points the tests that plant mistakes at a mutated build
+        lib = ctypes.CDLL(os.environ.get("NQ_ORACLE_SO") or build())
         P = ctypes.c_void_p
         i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         sig = {
