@@ -270,6 +270,19 @@ nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int
                      "nq_decode launch");
 }
 
+nq_status nq_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
+                         uint8_t* coset, nq_stream_t stream) {
+  if (bits != 2 && bits != 3) return fail(NQ_ERR_INVALID, "bits must be 2 or 3 (got %d)", bits);
+  if (groups < 0) return fail(NQ_ERR_INVALID, "groups must be >= 0");
+  if (groups == 0) return NQ_OK;
+  if (!y || !codes || !coset) return fail(NQ_ERR_INVALID, "y, codes and coset must be non-NULL");
+  if (!aligned(y, 4) || !aligned(codes, 4))
+    return fail(NQ_ERR_INVALID, "y and codes must be 4-byte aligned");
+  return cuda_status(nq::launch_e8_quantise(y, groups, bits, codes, coset,
+                                            reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_e8_quantise launch");
+}
+
 nq_status nq_device_error(uint32_t* flags_out) {
   if (!flags_out) return fail(NQ_ERR_INVALID, "flags_out is NULL");
   return cuda_status(nq::codec_read_clear_error(flags_out), "nq_device_error");

@@ -184,11 +184,12 @@ __device__ __forceinline__ void fwht_half(float2 (&v)[32], int half) {
 // (ties to even via the 1.5*2^23 trick), e = u - f, d = e0^2 then an fma
 // chain, an odd sum of f adds 1 - 2 max|e| (moving the first largest-error
 // coordinate toward u); the half coset wins only when strictly closer.
-// Returns the clamped b-bit codes of each lane packed as code i at bits
-// [BITS*i, BITS*i + BITS), and the coset bit of each lane.
-// Decision half of the decoder for two groups (lanes x, y): returns, per
-// lane, whether the half coset wins, whether its coordinate sum was odd (a
-// fix is needed) and the largest rounding error of the chosen coset.
+// e8_decide is that decision written out for both cosets; e8_choose reaches
+// the same decision from the integer coset alone when the two distances are
+// not close, and e8_codes then recomputes the chosen coset and packs it.
+// e8_decide returns, per lane, whether the half coset wins, whether its
+// coordinate sum was odd (a fix is needed) and the largest rounding error of
+// the chosen coset.
 struct E8Choice {
   float2 hh;     // 1 for the half coset, 0 for the integer coset
   float mx, my;  // largest |e| of the chosen coset
@@ -236,60 +237,150 @@ __device__ __forceinline__ E8Choice e8_decide(const float2 (&y)[8]) {
   return c;
 }
 
-// Code half of the decoder for two pairs of groups at once (four
-// independent fix chains): the chosen coset's rounding is recomputed
-// (U = y - shift, F = rint(U), E = U - F), the first coordinate with
-// |E| = m moves one step toward U when the sum was odd, then F is clamped
-// to the b-bit range and packed (code i at bits [BITS*i, BITS*i + BITS)).
-template <int BITS>
-__device__ __forceinline__ void e8_codes2(const float2 (&ya)[8], const float2 (&yb)[8],
-                                          const E8Choice& ca, const E8Choice& cb,
-                                          uint32_t (&g)[4]) {
+// max of eight non-negative values as chains of three-input maxima.
+__device__ __forceinline__ float max8(const float (&a)[8]) {
+  return fmaxf(fmaxf(fmaxf(fmaxf(a[0], a[1]), a[2]), fmaxf(fmaxf(a[3], a[4]), a[5])),
+               fmaxf(a[6], a[7]));
+}
+
+// fp32 fma with the result saturated to [0, 1] (one instruction).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Coset choice without the half coset's rounding.  Let e = y - rint(y) (exact)
+// and a_i = |e_i|.  Up to the rounding of y - 1/2 (below 2^-22 for |y| < 8)
+// the half coset's errors are 1/2 - a_i, so in exact arithmetic
+//   d1 - d0 = 2 - sum(a) + odd1 * 2 min(a) - odd0 * (1 - 2 max(a)),
+// with odd0 the parity of sum rint(y) (the LSB of each 1.5*2^23-biased value)
+// and, once every a_i >= 2^-20 (so that the rounding of y - 1/2 cannot move
+// its nearest integer), odd1 = odd0 xor (number of negative e_i).  The
+// decoder's two fp32 distances (eight fma roundings each on sums <= 2, plus
+// the fix term and the y - 1/2 roundings) and this fp32 estimate each stay
+// within 4e-6 of their exact values, so when the estimate is at least 6e-5
+// away from zero its sign is the sign of the fp32 comparison d1 < d0.  Any
+// other lane makes its warp run the full two-coset decision (e8_decide).
+// Per lane: whether the half coset wins and whether its rounded sum is odd.
+constexpr float kFastMargin = 6e-5f;
+constexpr float kFastMinErr = 9.5367431640625e-7f;  // 2^-20
+
+__device__ __forceinline__ void e8_fast_lane(const float (&a)[8], const uint32_t (&tb)[8],
+                                             const uint32_t (&eb)[8], bool& half, bool& odd,
+                                             bool& slow) {
+  const float A = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  const float mx = max8(a);
+  const float mn = fminf(fminf(fminf(fminf(a[0], a[1]), a[2]), fminf(fminf(a[3], a[4]), a[5])),
+                         fminf(a[6], a[7]));
+  const uint32_t P = (tb[0] ^ tb[1] ^ tb[2]) ^ (tb[3] ^ tb[4] ^ tb[5]) ^ (tb[6] ^ tb[7]);
+  const uint32_t S = (eb[0] ^ eb[1] ^ eb[2]) ^ (eb[3] ^ eb[4] ^ eb[5]) ^ (eb[6] ^ eb[7]);
+  const bool odd0 = P & 1u;
+  const bool odd1 = odd0 ^ static_cast<bool>(S >> 31);
+  float d = __fsub_rn(2.0f, A);
+  if (odd1) d = __fmaf_rn(2.0f, mn, d);
+  if (odd0) d = __fsub_rn(d, __fmaf_rn(-2.0f, mx, 1.0f));
+  slow = !(fabsf(d) >= kFastMargin) || !(mn >= kFastMinErr);
+  half = d < 0.0f;
+  odd = half ? odd1 : odd0;
+}
+
+// Coset and parity of the chosen coset for the two groups of y (lanes x, y).
+// The estimate above needs |y| < 7 (the y - 1/2 rounding bound); a lane whose
+// groups may exceed it passes force and always takes the full decision.
+__device__ __forceinline__ void e8_choose(const float2 (&y)[8], bool force, bool& halfx,
+                                          bool& halfy, bool& oddx, bool& oddy) {
   const float2 M2 = make_float2(kMagicRound, kMagicRound);
-  constexpr float kOffH = static_cast<float>(1 << (BITS - 1)) + kTwo23;
-  constexpr float kOffI = static_cast<float>((1 << (BITS - 1)) - 1) + kTwo23;
-  constexpr float kLoH = -static_cast<float>(1 << (BITS - 1));
-  constexpr float kLoI = -static_cast<float>((1 << (BITS - 1)) - 1);
-  constexpr float kHi = static_cast<float>((1 << (BITS - 1)) - 1);
-  const E8Choice* cc[2] = {&ca, &cb};
-  float2 off[2], lo[2];
-  bool fx[2], fy[2];
-  uint32_t ax[2] = {0u, 0u}, ay[2] = {0u, 0u};
-#pragma unroll
-  for (int p = 0; p < 2; ++p) {
-    const E8Choice& c = *cc[p];
-    off[p] = make_float2(c.hh.x != 0.f ? kOffH : kOffI, c.hh.y != 0.f ? kOffH : kOffI);
-    lo[p] = make_float2(c.hh.x != 0.f ? kLoH : kLoI, c.hh.y != 0.f ? kLoH : kLoI);
-    fx[p] = !c.oddx;  // "fix done" flags
-    fy[p] = !c.oddy;
-  }
+  float ax[8], ay[8];
+  uint32_t tx[8], ty[8], ex[8], ey[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-#pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      const E8Choice& c = *cc[p];
-      const float2 yy = p ? yb[i] : ya[i];
-      const float2 U = fma2(c.hh, make_float2(-0.5f, -0.5f), yy);
-      float2 F = sub2(add2(U, M2), M2);
-      const float2 E = sub2(U, F);
-      const bool hitx = !fx[p] && fabsf(E.x) == c.mx;
-      const bool hity = !fy[p] && fabsf(E.y) == c.my;
-      fx[p] = fx[p] || hitx;
-      fy[p] = fy[p] || hity;
-      // E is never -0 (y carries no -0), so its sign bit decides the direction
-      if (hitx) F.x = __fadd_rn(F.x, copysignf(1.0f, E.x));
-      if (hity) F.y = __fadd_rn(F.y, copysignf(1.0f, E.y));
-      F = make_float2(fminf(fmaxf(F.x, lo[p].x), kHi), fminf(fmaxf(F.y, lo[p].y), kHi));
-      const float2 J = add2(F, off[p]);  // 2^23 + code: the code sits in the low mantissa bits
-      ax[p] += __float_as_uint(J.x) << (BITS * i);
-      ay[p] += __float_as_uint(J.y) << (BITS * i);
+    const float2 t = add2(y[i], M2);
+    const float2 e = sub2(y[i], sub2(t, M2));
+    ax[i] = fabsf(e.x);
+    ay[i] = fabsf(e.y);
+    tx[i] = __float_as_uint(t.x);
+    ty[i] = __float_as_uint(t.y);
+    ex[i] = __float_as_uint(e.x);
+    ey[i] = __float_as_uint(e.y);
+  }
+  bool slowx, slowy;
+  e8_fast_lane(ax, tx, ex, halfx, oddx, slowx);
+  e8_fast_lane(ay, ty, ey, halfy, oddy, slowy);
+  slowx = slowx || force;
+  slowy = slowy || force;
+  if (__any_sync(0xffffffffu, slowx || slowy)) {
+    const E8Choice c = e8_decide(y);
+    if (slowx) {
+      halfx = c.hh.x != 0.f;
+      oddx = c.oddx;
+    }
+    if (slowy) {
+      halfy = c.hh.y != 0.f;
+      oddy = c.oddy;
     }
   }
+}
+
+// Codes of the chosen cosets for the two groups of y (lanes x, y): the
+// coset's rounding is recomputed (U = y - shift with a +0 shift for the
+// integer coset, so U is never -0; F = rint(U), E = U - F), m = max |E|; when
+// the sum was odd the first coordinate with |E| = m moves one step toward U
+// (E >= 0: up).  The clamp to [lo, lo + R] (R = 2^b - 1 for the half coset,
+// 2^b - 2 for the integer one) and the code j = F - lo come from
+// a = sat((F - lo) / R), evaluated as one saturating fma with fp32 1/R and
+// -lo/R (error below 1e-6 in a*R for |F| < 8, so a*R + 2^23 rounds to
+// 2^23 + j exactly; values beyond the range saturate to 0 or 1), then
+// J = fma(a, R, 2^23), whose low mantissa bits hold j.  Code i is packed at
+// bits [BITS*i, BITS*i + BITS).
+template <int BITS>
+__device__ __forceinline__ void e8_codes(const float2 (&y)[8], bool halfx, bool halfy, bool oddx,
+                                         bool oddy, uint32_t& gx, uint32_t& gy) {
+  const float2 M2 = make_float2(kMagicRound, kMagicRound);
+  constexpr float kRH = static_cast<float>((1 << BITS) - 1);
+  constexpr float kRI = static_cast<float>((1 << BITS) - 2);
+  constexpr float kInvH = 1.0f / kRH, kInvI = 1.0f / kRI;
+  constexpr float kCH = static_cast<float>(1 << (BITS - 1)) / kRH;
+  constexpr float kCI = static_cast<float>((1 << (BITS - 1)) - 1) / kRI;
+  const float2 sh = make_float2(halfx ? -1.0f : 0.0f, halfy ? -1.0f : 0.0f);
+  const float2 H2 = make_float2(0.5f, 0.5f);
+  float2 F[8], E[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 U = fma2(sh, H2, y[i]);
+    F[i] = sub2(add2(U, M2), M2);
+    E[i] = sub2(U, F[i]);
+  }
+  float ex[8], ey[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    ex[i] = fabsf(E[i].x);
+    ey[i] = fabsf(E[i].y);
+  }
+  const float mx = max8(ex), my = max8(ey);
+  const float2 R2 = make_float2(halfx ? kRH : kRI, halfy ? kRH : kRI);
+  const float ix = halfx ? kInvH : kInvI, iy = halfy ? kInvH : kInvI;
+  const float cx = halfx ? kCH : kCI, cy = halfy ? kCH : kCI;
+  const float2 B2 = make_float2(kTwo23, kTwo23);
+  bool fx = !oddx, fy = !oddy;  // "fix done" flags
+  uint32_t ax = 0u, ay = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float2 f = F[i];
+    const bool hitx = !fx && ex[i] == mx;
+    const bool hity = !fy && ey[i] == my;
+    fx = fx || hitx;
+    fy = fy || hity;
+    if (hitx) f.x = __fadd_rn(f.x, copysignf(1.0f, E[i].x));
+    if (hity) f.y = __fadd_rn(f.y, copysignf(1.0f, E[i].y));
+    const float2 a2 = make_float2(fma_sat(f.x, ix, cx), fma_sat(f.y, iy, cy));
+    const float2 J = fma2(a2, R2, B2);  // 2^23 + code: the code sits in the low mantissa bits
+    ax += __float_as_uint(J.x) << (BITS * i);
+    ay += __float_as_uint(J.y) << (BITS * i);
+  }
   constexpr uint32_t kMask = (1u << (8 * BITS)) - 1u;
-  g[0] = ax[0] & kMask;
-  g[1] = ay[0] & kMask;
-  g[2] = ax[1] & kMask;
-  g[3] = ay[1] & kMask;
+  gx = ax & kMask;
+  gy = ay & kMask;
 }
 
 // --------------------------------------------------------------- encode
@@ -327,13 +418,18 @@ template <int BITS>
 __device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool valid,
                                               uint32_t* codes, uint32_t* meta) {
   fwht_half(v, half);
-  float M = 0.0f;
+  float m4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four chains for latency
 #pragma unroll
-  for (int j = 0; j < 32; ++j) M = fmaxf(M, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
+  for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(fmaxf(m4[j & 3], fabsf(v[j].x)), fabsf(v[j].y));
+  float M = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
   M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
   const float G = __uint_as_float(BITS == 3 ? kG3Bits : kG2Bits);
   const float C = __uint_as_float(kCBits);
-  const __half sh = __float2half_rn(fminf(__fmul_rn(M, G), 65504.0f));
+  const float P = __fmul_rn(M, G);
+  const __half sh = __float2half_rn(fminf(P, 65504.0f));
+  // Unsaturated, sigma >= P / 1.5 (fp16 subnormals included), so |y| <=
+  // 1.5 * A_b <= 5.25; a saturated scale can leave |y| larger.
+  const bool big = !(P <= 65504.0f);
   const float sig = __half2float(sh);
   const float r = (sig == 0.0f) ? 0.0f : __fdiv_rn(C, sig);
   const float2 r2 = make_float2(r, r);
@@ -341,25 +437,15 @@ __device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool va
   uint32_t gx[4], gy[4];
   uint32_t cm = 0;
 #pragma unroll
-  for (int q = 0; q < 4; q += 2) {
-    float2 ya[8], yb[8];
+  for (int q = 0; q < 4; ++q) {
+    float2 y[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      ya[i] = add2(mul2(v[8 * q + i], r2), make_float2(0.f, 0.f));
-      yb[i] = add2(mul2(v[8 * (q + 1) + i], r2), make_float2(0.f, 0.f));
-    }
-    const E8Choice ca = e8_decide(ya);
-    const E8Choice cb = e8_decide(yb);
-    uint32_t g[4];
-    e8_codes2<BITS>(ya, yb, ca, cb, g);
-    gx[q] = g[0];
-    gy[q] = g[1];
-    gx[q + 1] = g[2];
-    gy[q + 1] = g[3];
-    cm |= ((ca.hh.x != 0.f ? 1u : 0u) << (4 * half + q)) |
-          ((ca.hh.y != 0.f ? 1u : 0u) << (8 + 4 * half + q)) |
-          ((cb.hh.x != 0.f ? 1u : 0u) << (4 * half + q + 1)) |
-          ((cb.hh.y != 0.f ? 1u : 0u) << (8 + 4 * half + q + 1));
+    for (int i = 0; i < 8; ++i) y[i] = mul2(v[8 * q + i], r2);
+    bool hx, hy, ox, oy;
+    e8_choose(y, big, hx, hy, ox, oy);
+    e8_codes<BITS>(y, hx, hy, ox, oy, gx[q], gy[q]);
+    cm |= (static_cast<uint32_t>(hx) << (4 * half + q)) |
+          (static_cast<uint32_t>(hy) << (8 + 4 * half + q));
   }
   cm |= __shfl_xor_sync(0xffffffffu, cm, 16);
   if (!valid) return;
@@ -869,6 +955,65 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
     return launch_kind(true, v, L.v_in.bits, false, L.units, stream);
   }
   return cudaSuccess;
+}
+
+// ------------------------------------------------------ E8 quantiser alone
+// One thread per pair of groups (2p in lane x, 2p + 1 in lane y) of a
+// [groups][8] fp32 array, with the encode kernel's decision and code
+// functions.  The CTA loop bound is uniform across each warp (threads past
+// the end run on zeros), as the warp vote in e8_choose needs.
+template <int BITS>
+__global__ void __launch_bounds__(256) e8_quantise_kernel(const float* __restrict__ y,
+                                                          int64_t groups, uint32_t* codes,
+                                                          uint8_t* coset) {
+  const int64_t pairs = (groups + 1) / 2;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x; base < pairs;
+       base += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t p = base + threadIdx.x;
+    const int64_t g0 = 2 * p, g1 = 2 * p + 1;
+    float a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      a[i] = g0 < groups ? __ldg(y + 8 * g0 + i) : 0.0f;
+      b[i] = g1 < groups ? __ldg(y + 8 * g1 + i) : 0.0f;
+    }
+    float2 yy[8];
+    float big = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      yy[i] = make_float2(a[i], b[i]);
+      big = fmaxf(big, fmaxf(fabsf(a[i]), fabsf(b[i])));
+    }
+    bool hx, hy, ox, oy;
+    e8_choose(yy, !(big < 7.0f), hx, hy, ox, oy);
+    uint32_t cx, cy;
+    e8_codes<BITS>(yy, hx, hy, ox, oy, cx, cy);
+    if (g0 < groups) {
+      codes[g0] = cx;
+      coset[g0] = hx ? 1 : 0;
+    }
+    if (g1 < groups) {
+      codes[g1] = cy;
+      coset[g1] = hy ? 1 : 0;
+    }
+  }
+}
+
+cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
+                               uint8_t* coset, cudaStream_t stream) {
+  if (groups <= 0) return cudaSuccess;
+  int dev = 0, sms = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  const int64_t pairs = (groups + 1) / 2;
+  const int64_t grid = min64((pairs + 255) / 256, static_cast<int64_t>(sms) * 8);
+  if (bits == 3)
+    e8_quantise_kernel<3><<<static_cast<unsigned>(grid), 256, 0, stream>>>(y, groups, codes, coset);
+  else
+    e8_quantise_kernel<2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(y, groups, codes, coset);
+  return cudaGetLastError();
 }
 
 }  // namespace nq

@@ -46,6 +46,8 @@ cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 
 cudaError_t codec_read_clear_error(uint32_t* flags);
+cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
+                               uint8_t* coset, cudaStream_t stream);
 
 cudaError_t launch_score(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
                          double* scores, float* mean_ws, cudaStream_t stream);

@@ -42,7 +42,7 @@ EXPORTS = (
     "nq_last_error", "nq_version", "nq_packed_bytes_per_vector", "nq_rope_tables_bytes",
     "nq_rope_tables_fill_host", "nq_score_workspace_bytes", "nq_score", "nq_score_static",
     "nq_kept_count",
-    "nq_select", "nq_encode", "nq_decode", "nq_device_error",
+    "nq_select", "nq_encode", "nq_decode", "nq_e8_quantise", "nq_device_error",
 )
 
 
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
                             PK, PK, i64, P]),
         "nq_decode": (i32, [PK, PK, i32, i32, i64, i64, P, i64, i64, P, i64, P, KVStrides, P,
                             KVStrides, P]),
+        "nq_e8_quantise": (i32, [P, i64, i32, P, P, P]),
         "nq_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32)]),
     }
     for name, (res, args) in sig.items():
@@ -256,6 +257,20 @@ def nq_decode(k_in: PackedStore | None, v_in: PackedStore | None, n: int,
                            positions.stride(0) if positions is not None else 0, int(pos_base),
                            _ptr(rope_tab), int(rope_max_pos), _ptr(K_out), kos, _ptr(V_out),
                            vos, _stream(stream)))
+
+
+def nq_e8_quantise(y: torch.Tensor, bits: int, stream=None):
+    """E8 step alone on [groups][8] fp32 rows (device): returns (codes int32
+    [groups], code k of a group at bits [bits*k, bits*k + bits); coset uint8
+    [groups], 1 = half-integer coset)."""
+    _require_cuda(y)
+    if y.dtype != torch.float32 or y.dim() != 2 or y.shape[1] != 8 or not y.is_contiguous():
+        raise ValueError("y must be a contiguous float32 [groups, 8] tensor")
+    g = y.shape[0]
+    codes = torch.empty(g, dtype=torch.int32, device=y.device)
+    coset = torch.empty(g, dtype=torch.uint8, device=y.device)
+    _check(lib().nq_e8_quantise(_ptr(y), g, int(bits), _ptr(codes), _ptr(coset), _stream(stream)))
+    return codes, coset
 
 
 def device_error() -> int:

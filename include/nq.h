@@ -209,6 +209,23 @@ nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int
                     int64_t pos_base, const float *rope_tab, int64_t rope_max_pos, void *K_out,
                     nq_kv_strides kos, void *V_out, nq_kv_strides vos, nq_stream_t stream);
 
+/* ------------------------------------------------------ E8 quantiser
+ * The lattice step of nq_encode on its own ([NQ-zh] "E8 lattice
+ * quantisation"; [NQ-pt] step 4), for coordinates that are already rotated
+ * and scaled: each row g of y ([groups][8] fp32, contiguous) is snapped to
+ * the nearest E8 point with exactly nq_encode's fp32 decoder (D8 and
+ * D8 + 1/2, round to nearest even, the odd-sum fix on the first
+ * largest-error coordinate, fp32 fma distance chains, a tie keeps the
+ * integer coset), then clamped and coded as in nq_encode:
+ *   codes[g]: the 8 b-bit codes of the group, code i at bits [b*i, b*i + b)
+ *   coset[g]: 1 when the point lies in D8 + 1/2, else 0.
+ * y, codes (uint32 [groups]) and coset (uint8 [groups]) are device arrays
+ * owned by the caller; y and codes 4-byte aligned.  bits is 2 or 3;
+ * groups = 0 launches nothing.  y must be finite with |y| < 2^22; other
+ * values are out of contract (no fault, unspecified codes). */
+nq_status nq_e8_quantise(const float *y, int64_t groups, int bits, uint32_t *codes,
+                         uint8_t *coset, nq_stream_t stream);
+
 /* -------------------------------------------------------------- status
  * Reads and clears the device error word reserved for in-kernel failure
  * reports (bit 0: an asynchronous copy did not complete).  Synchronises the

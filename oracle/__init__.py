@@ -66,6 +66,7 @@ def _load():
             "oq_encode_unit": (i64, [P, P, i32, i64, i64, P, i64, dbl, i32, i32, P, P, P, P]),
             "oq_decode_unit": (None, [P, P, P, P, i32, i64, P, i64, dbl, i32, i32, P, P]),
             "oq_e8_batch": (None, [P, i64, P, P, P]),
+            "oq_e8_code_batch": (None, [P, i64, ctypes.c_int, P, P]),
             "oq_fwht_batch": (None, [P, i64]),
             "oq_f32_to_f16_batch": (None, [P, i64, P]),
             "oq_f32_to_bf16_batch": (None, [P, i64, P]),
@@ -155,6 +156,17 @@ def e8_nearest(y) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
     d = np.empty(n, np.float32)
     _load().oq_e8_batch(_p(y), n, _p(t), _p(cs), _p(d))
     return t, cs, d
+
+
+def e8_codes(y, bits: int) -> tuple[np.ndarray, np.ndarray]:
+    """E8 step with codes of [n][8] fp32 groups: (codes uint32 [n], code k of a
+    group at bits [bits*k, bits*k + bits); coset int32 [n])."""
+    y = np.ascontiguousarray(y, dtype=np.float32).reshape(-1, 8)
+    n = y.shape[0]
+    codes = np.empty(n, np.uint32)
+    cs = np.empty(n, np.int32)
+    _load().oq_e8_code_batch(_p(y), n, int(bits), _p(codes), _p(cs))
+    return codes, cs
 
 
 # ------------------------------------------------------ vector codec

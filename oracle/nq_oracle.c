@@ -481,6 +481,23 @@ void oq_e8_batch(const float *y, int64_t n, int32_t *t_out, int32_t *coset_out, 
         coset_out[i] = oq_e8_nearest(y + 8 * i, t_out + 8 * i, dist_out + i);
 }
 
+/* Batched E8 step with codes: nearest point (oq_e8_nearest), then the clamp
+ * and code rule (oq_code); codes_out[i] holds the 8 b-bit codes of group i,
+ * code k at bits [b*k, b*k + b). */
+void oq_e8_code_batch(const float *y, int64_t n, int bits, uint32_t *codes_out,
+                      int32_t *coset_out)
+{
+    for (int64_t i = 0; i < n; i++) {
+        int32_t t[8];
+        int clamped = 0;
+        int half = oq_e8_nearest(y + 8 * i, t, NULL);
+        uint32_t w = 0;
+        for (int k = 0; k < 8; k++) w |= oq_code(t[k], half, bits, &clamped) << (bits * k);
+        codes_out[i] = w;
+        coset_out[i] = half;
+    }
+}
+
 void oq_fwht_batch(float *v, int64_t n)
 {
     for (int64_t i = 0; i < n; i++) oq_fwht128(v + OQ_D * i);

@@ -190,3 +190,22 @@ def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
         for k in range(bits):
             codes[:, c] |= stream[:, bits * c + k].astype(np.int64) << k
     return codes
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_e8_codes_are_clamped_nearest_points(oq, bits):
+    """The batched E8 step with codes: each code decodes (t = 2j - lim) to the
+    nearest point's 2q clipped to the b-bit range of its coset."""
+    rng = np.random.default_rng(15)
+    y = np.concatenate([
+        rng.uniform(-4.5, 4.5, (20000, 8)),
+        rng.integers(-8, 9, (2000, 8)) / 2.0,
+        rng.normal(0, 1, (2000, 8)) * 1e-6,
+    ]).astype(np.float32)
+    codes, coset = oq.e8_codes(y, bits)
+    t, cs, _ = oq.e8_nearest(y)
+    assert np.array_equal(coset, cs)
+    j = (codes[:, None].astype(np.int64) >> (bits * np.arange(8))[None, :]) & ((1 << bits) - 1)
+    lim = np.where(coset == 1, (1 << bits) - 1, (1 << bits) - 2)[:, None]
+    assert np.array_equal(2 * j - lim, np.clip(t, -lim, lim))
+    assert np.all(codes < (1 << (8 * bits)))
