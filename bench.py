@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mistral7b_32k")
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-chunk", type=int, default=2, help="layers per pipelined chunk (e2e)")
     ap.add_argument("--cpu-layers", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -461,7 +462,8 @@ def run_ours(args, world, rank, local):
 
 def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     """Same metric through the public API with HOST buffers: pinned H2D of the
-    inputs, the four calls, D2H of the reconstructed cache, every step."""
+    inputs, the four calls, D2H of the reconstructed cache, every step, as
+    nq.HostRoundTrip pipelines them (chunks of layers on three streams)."""
     from e8_lattice_vector_nq_b200 import nq
 
     Kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
@@ -470,14 +472,10 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     Vh.copy_(V)
     Koh = torch.empty(Kd.shape, dtype=Kd.dtype, pin_memory=True)
     Voh = torch.empty(Vd.shape, dtype=Vd.dtype, pin_memory=True)
+    rt = nq.HostRoundTrip(codec, K, V, Kd, Vd, chunk_units=args.e2e_chunk)
 
     def step():
-        K.copy_(Kh, non_blocking=True)
-        V.copy_(Vh, non_blocking=True)
-        codec.encode(K, V)
-        codec.decode(Kd, Vd)
-        Koh.copy_(Kd, non_blocking=True)
-        Voh.copy_(Vd, non_blocking=True)
+        rt.run(Kh, Vh, Koh, Voh)
 
     step()
     torch.cuda.synchronize()
@@ -490,7 +488,7 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     ms = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, world, K.device)
     return {"value": world * in_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": Kd.numel() * 2 + Vd.numel() * 2,
-            "ms_per_step": ms, "steps": args.e2e_steps}
+            "ms_per_step": ms, "steps": args.e2e_steps, "chunk_layers": args.e2e_chunk}
 
 
 def main():

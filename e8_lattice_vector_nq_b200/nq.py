@@ -303,16 +303,26 @@ class Codec:
         else:
             self.kept = None
 
-    def encode(self, K: torch.Tensor, V: torch.Tensor, stream=None):
+    def encode(self, K: torch.Tensor, V: torch.Tensor, stream=None, units: slice | None = None):
+        """Compress K, V [units][heads][T][128]; with `units`, only that range
+        of units (K and V are then the full-cache tensors)."""
+        u = units or slice(0, self.units)
+        kept = self.kept[u] if self.kept is not None else None
         if self.evict:
-            nq_score(K, self.W, self.scores, self.ws, stream)
-            nq_select(self.scores, self.W, self.pct, self.kept, stream)
-        nq_encode(K, V, self.k_store, self.v_store, self.n, self.rope, self.max_pos,
-                  kept=self.kept, stream=stream)
+            ws = self.ws.view(self.units, -1)[u] if self.ws.numel() % self.units == 0 else self.ws
+            nq_score(K[u] if units else K, self.W, self.scores[u], ws, stream)
+            nq_select(self.scores[u], self.W, self.pct, kept, stream)
+        nq_encode(K[u] if units else K, V[u] if units else V, self.k_store.select_units(u),
+                  self.v_store.select_units(u), self.n, self.rope, self.max_pos, kept=kept,
+                  stream=stream)
 
-    def decode(self, K_out: torch.Tensor, V_out: torch.Tensor, stream=None):
-        nq_decode(self.k_store, self.v_store, self.n, K_out, V_out, self.rope, self.max_pos,
-                  positions=self.kept, stream=stream)
+    def decode(self, K_out: torch.Tensor, V_out: torch.Tensor, stream=None,
+               units: slice | None = None):
+        u = units or slice(0, self.units)
+        nq_decode(self.k_store.select_units(u), self.v_store.select_units(u), self.n,
+                  K_out[u] if units else K_out, V_out[u] if units else V_out, self.rope,
+                  self.max_pos, positions=self.kept[u] if self.kept is not None else None,
+                  stream=stream)
 
     @property
     def packed_bytes(self) -> int:
@@ -320,6 +330,54 @@ class Codec:
         if self.kept is not None:
             b += self.kept.numel() * 4
         return b
+
+
+class HostRoundTrip:
+    """Compress a cache that lives in pinned host memory and write its
+    reconstruction back to pinned host memory, in chunks of units on three
+    streams: the host-to-device copy of chunk c+1, the kernels of chunk c and
+    the device-to-host copy of chunk c-1 run at the same time (the two copy
+    directions share nothing on a full-duplex link).  The device tensors are
+    the codec's working copies; every run() is asynchronous on the caller's
+    current stream, which afterwards waits for the last copy."""
+
+    def __init__(self, codec: Codec, K: torch.Tensor, V: torch.Tensor, K_out: torch.Tensor,
+                 V_out: torch.Tensor, chunk_units: int = 4):
+        self.codec, self.K, self.V, self.K_out, self.V_out = codec, K, V, K_out, V_out
+        self.chunks = [slice(u, min(u + chunk_units, codec.units))
+                       for u in range(0, codec.units, chunk_units)]
+        self.h2d, self.comp, self.d2h = (torch.cuda.Stream(K.device) for _ in range(3))
+        ev = lambda: [torch.cuda.Event() for _ in self.chunks]  # noqa: E731
+        self.in_ready, self.comp_done, self.out_done = ev(), ev(), ev()
+        self.ran = False
+
+    def run(self, Kh: torch.Tensor, Vh: torch.Tensor, K_out_h: torch.Tensor,
+            V_out_h: torch.Tensor):
+        caller = torch.cuda.current_stream(self.K.device)
+        start = torch.cuda.Event()
+        start.record(caller)
+        for s in (self.h2d, self.comp, self.d2h):
+            s.wait_event(start)
+        for c, u in enumerate(self.chunks):
+            with torch.cuda.stream(self.h2d):
+                if self.ran:  # the previous run's kernels are done reading this chunk
+                    self.h2d.wait_event(self.comp_done[c])
+                self.K[u].copy_(Kh[u], non_blocking=True)
+                self.V[u].copy_(Vh[u], non_blocking=True)
+                self.in_ready[c].record(self.h2d)
+            self.comp.wait_event(self.in_ready[c])
+            if self.ran:  # the previous run's copy-out of this chunk is done
+                self.comp.wait_event(self.out_done[c])
+            self.codec.encode(self.K, self.V, self.comp, units=u)
+            self.codec.decode(self.K_out, self.V_out, self.comp, units=u)
+            self.comp_done[c].record(self.comp)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(self.comp_done[c])
+                K_out_h[u].copy_(self.K_out[u], non_blocking=True)
+                V_out_h[u].copy_(self.V_out[u], non_blocking=True)
+                self.out_done[c].record(self.d2h)
+        caller.wait_event(self.out_done[-1])
+        self.ran = True
 
 
 # ------------------------------------------------------- whole-cache pipelines
