@@ -342,7 +342,10 @@ __device__ __forceinline__ void e8_codes(const float2 (&y)[8], bool halfx, bool 
   constexpr float kInvH = 1.0f / kRH, kInvI = 1.0f / kRI;
   constexpr float kCH = static_cast<float>(1 << (BITS - 1)) / kRH;
   constexpr float kCI = static_cast<float>((1 << (BITS - 1)) - 1) / kRI;
-  const float2 sh = make_float2(halfx ? -1.0f : 0.0f, halfy ? -1.0f : 0.0f);
+  // per-lane coset constants from the coset flag hf in {0, 1} with packed fmas
+  // (1/R and -lo/R need not be exact: only a*R + 2^23 must round to 2^23 + j)
+  const float2 hf = make_float2(halfx ? 1.0f : 0.0f, halfy ? 1.0f : 0.0f);
+  const float2 sh = fma2(hf, make_float2(-1.0f, -1.0f), make_float2(0.0f, 0.0f));
   const float2 H2 = make_float2(0.5f, 0.5f);
   float2 F[8], E[8];
 #pragma unroll
@@ -358,9 +361,10 @@ __device__ __forceinline__ void e8_codes(const float2 (&y)[8], bool halfx, bool 
     ey[i] = fabsf(E[i].y);
   }
   const float mx = max8(ex), my = max8(ey);
-  const float2 R2 = make_float2(halfx ? kRH : kRI, halfy ? kRH : kRI);
-  const float ix = halfx ? kInvH : kInvI, iy = halfy ? kInvH : kInvI;
-  const float cx = halfx ? kCH : kCI, cy = halfy ? kCH : kCI;
+  const float2 R2 = add2(hf, make_float2(kRI, kRI));
+  const float2 i2 = fma2(hf, make_float2(kInvH - kInvI, kInvH - kInvI), make_float2(kInvI, kInvI));
+  const float2 c2 = fma2(hf, make_float2(kCH - kCI, kCH - kCI), make_float2(kCI, kCI));
+  const float ix = i2.x, iy = i2.y, cx = c2.x, cy = c2.y;
   const float2 B2 = make_float2(kTwo23, kTwo23);
   bool fx = !oddx, fy = !oddy;  // "fix done" flags
   uint32_t ax = 0u, ay = 0u;
@@ -552,14 +556,11 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
     const int64_t slot = tl.stile * kSlots + slot_l;
     const bool valid = slot < a.n;
     unsigned char* st = smem + s * stage_bytes;
+    // lanes past the last slot run on whatever their staging row holds; none
+    // of their results is stored
     float2 v[32];
-    if (valid) {
-      load_half<ROPE>(v, smem_u32(st + row_idx * kRowPad),
-                      smem_u32(st + rows_bytes) + (16 * half * kSlots + slot_l) * 16, half);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = make_float2(0.f, 0.f);
-    }
+    load_half<ROPE>(v, smem_u32(st + row_idx * kRowPad),
+                    smem_u32(st + rows_bytes) + (16 * half * kSlots + slot_l) * 16, half);
     if (ROPE && k + 1 < my_tiles)  // RoPE table of tile k+1 into the other stage
       combine_raw(raw, reinterpret_cast<float4*>(smem + (s ^ 1) * stage_bytes + rows_bytes), tid,
                   nthreads);
