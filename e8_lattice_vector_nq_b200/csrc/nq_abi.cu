@@ -114,7 +114,7 @@ nq_status nq_score(const void* K, nq_kv_strides ks, int units, int heads, int64_
   if (units < 0 || heads < 1 || heads > 1024)
     return fail(NQ_ERR_INVALID, "need units >= 0 and 1 <= heads <= 1024");
   if (T < 1 || W < 1 || W > T) return fail(NQ_ERR_INVALID, "need 1 <= W <= T");
-  if (heads > 256) return fail(NQ_ERR_UNSUPPORTED, "nq_score supports at most 256 heads");
+  if (heads > 128) return fail(NQ_ERR_UNSUPPORTED, "nq_score supports at most 128 heads");
   if (units == 0) return NQ_OK;
   if (nq_status st = check_kv(K, ks, "K")) return st;
   if (!scores || !aligned(scores, 8)) return fail(NQ_ERR_INVALID, "scores NULL or misaligned");
@@ -122,7 +122,7 @@ nq_status nq_score(const void* K, nq_kv_strides ks, int units, int heads, int64_
   if (ws_bytes < nq_score_workspace_bytes(units, heads))
     return fail(NQ_ERR_WORKSPACE, "score workspace too small: %zu < %zu", ws_bytes,
                 nq_score_workspace_bytes(units, heads));
-  if (static_cast<int64_t>(units) * ((T + 63) / 64) > 0x7FFFFFFF)
+  if (static_cast<int64_t>(units) * ((T + 127) / 128) > 0x7FFFFFFF)
     return fail(NQ_ERR_UNSUPPORTED, "units * T too large for one launch");
   return cuda_status(nq::launch_score(K, ks, units, heads, T, W, scores, static_cast<float*>(ws),
                                       reinterpret_cast<cudaStream_t>(stream)),
@@ -131,9 +131,10 @@ nq_status nq_score(const void* K, nq_kv_strides ks, int units, int heads, int64_
 
 nq_status nq_score_static(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
                           double* scores, nq_stream_t stream) {
-  if (units < 0 || heads < 1 || heads > 256)
-    return fail(NQ_ERR_INVALID, "need units >= 0 and 1 <= heads <= 256");
+  if (units < 0 || heads < 1 || heads > 1024)
+    return fail(NQ_ERR_INVALID, "need units >= 0 and 1 <= heads <= 1024");
   if (T < 1 || W < 1 || W > T) return fail(NQ_ERR_INVALID, "need 1 <= W <= T");
+  if (heads > 128) return fail(NQ_ERR_UNSUPPORTED, "nq_score_static supports at most 128 heads");
   if (static_cast<int64_t>(units) * heads > NQ_SCORE_STATIC_MAX_VECTORS)
     return fail(NQ_ERR_UNSUPPORTED,
                 "nq_score_static: units * heads = %lld exceeds its fixed scratch of %d "
@@ -142,7 +143,7 @@ nq_status nq_score_static(const void* K, nq_kv_strides ks, int units, int heads,
   if (units == 0) return NQ_OK;
   if (nq_status st = check_kv(K, ks, "K")) return st;
   if (!scores || !aligned(scores, 8)) return fail(NQ_ERR_INVALID, "scores NULL or misaligned");
-  if (static_cast<int64_t>(units) * ((T + 63) / 64) > 0x7FFFFFFF)
+  if (static_cast<int64_t>(units) * ((T + 127) / 128) > 0x7FFFFFFF)
     return fail(NQ_ERR_UNSUPPORTED, "units * T too large for one launch");
   return cuda_status(nq::launch_score_static(K, ks, units, heads, T, W, scores,
                                              reinterpret_cast<cudaStream_t>(stream)),

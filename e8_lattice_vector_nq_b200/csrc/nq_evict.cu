@@ -9,10 +9,13 @@
 //   window_mean_kernel: m[u][h][d] = fp32(fp64 sum of the last W keys / W)
 //   score_kernel:       scores[u][t] = sum_h sum_d K[u][h][t][d] * m[u][h][d]
 //                       in fp64 (one coalesced pass over K)
-//   select_kernel:      per unit, an 8-pass MSD radix select of the
+//   select_kernel:      per unit, an MSD radix select (11-bit digits, after
+//                       the prefix that every middle key shares) of the
 //                       (score desc, position asc) threshold on
-//                       order-preserving 64-bit keys, then an ordered
-//                       compaction with warp ballots.
+//                       order-preserving 64-bit keys; once at most 8192 keys
+//                       share the prefix they move to shared memory and the
+//                       remaining digits are read from there; then an
+//                       ordered compaction with warp ballots.
 #include <mutex>
 
 #include "nq_internal.h"
@@ -30,10 +33,12 @@ __global__ void window_mean_kernel(const uint16_t* __restrict__ K, nq_kv_strides
 }
 
 // ---------------------------------------------------------------- score
-constexpr int kScoreTok = 64;      // tokens per CTA
+constexpr int kScoreTok = 128;     // tokens per CTA
 constexpr int kScoreThreads = 256;
 
-__global__ void __launch_bounds__(kScoreThreads) score_kernel(const uint16_t* __restrict__ K,
+// 4 CTAs (32 warps) per SM: more 16-byte loads in flight per SM (a few
+// registers spill to L1).
+__global__ void __launch_bounds__(kScoreThreads, 4) score_kernel(const uint16_t* __restrict__ K,
                                                               nq_kv_strides ks, int heads,
                                                               int64_t T,
                                                               const float* __restrict__ mean,
@@ -117,13 +122,16 @@ __device__ __forceinline__ void block_exclusive_scan32(int* vals /*[32] smem*/) 
 constexpr int kDigitBits = 11;
 constexpr int kUnroll = 8;  // independent score loads in flight per thread
 constexpr int kBins = 1 << kDigitBits;  // 2 bins per thread
+constexpr int kCandCap = 8192;          // candidate keys kept in shared memory
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __restrict__ scores,
                                                              int64_t T, int W, int64_t n_kept,
                                                              int32_t* __restrict__ kept,
                                                              int64_t kept_stride) {
-  extern __shared__ uint32_t flagbits[];  // ceil(T/32) words
+  extern __shared__ uint32_t flagbits[];  // ceil(T/32) words, then the candidate keys
+  uint64_t* cand = reinterpret_cast<uint64_t*>(flagbits + ((T + 63) / 64) * 2);
   __shared__ unsigned int hist[kBins];
+  __shared__ unsigned int s_ncand;
   __shared__ uint64_t s_min[kSelWarps], s_max[kSelWarps];
   __shared__ unsigned int s_wsum[kSelWarps];
   __shared__ uint64_t s_prefix;
@@ -192,26 +200,34 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
     int rem = diff ? 64 - __clzll(static_cast<long long>(diff)) : 0;  // bits still undecided
     prefix = s_min[0] & (rem == 64 ? 0ull : ~((1ull << rem) - 1ull));
     __syncthreads();
+    int64_t ncand = -1;  // >= 0 once the candidates sit in cand[]
     while (rem > 0) {
       const int width = rem < kDigitBits ? rem : kDigitBits;
       const int shift = rem - width;
       const uint64_t pmask = rem == 64 ? 0ull : ~((1ull << rem) - 1ull);
       for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
       __syncthreads();
-      // warp-uniform loop bound (lanes past the end are masked by `in`)
-      for (int64_t w0 = lo + (tid & ~31); w0 < hi; w0 += kUnroll * blockDim.x) {
-        const int64_t t0 = w0 + lane;
-        double v[kUnroll];
-#pragma unroll
-        for (int j = 0; j < kUnroll; ++j) {
-          const int64_t t = t0 + j * blockDim.x;
-          v[j] = t < hi ? __ldg(s + t) : 0.0;
+      if (ncand >= 0) {
+        for (int64_t i = tid; i < ncand; i += blockDim.x) {
+          const uint64_t key = cand[i];
+          if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
         }
+      } else {
+        // warp-uniform loop bound (lanes past the end are masked by `in`)
+        for (int64_t w0 = lo + (tid & ~31); w0 < hi; w0 += kUnroll * blockDim.x) {
+          const int64_t t0 = w0 + lane;
+          double v[kUnroll];
 #pragma unroll
-        for (int j = 0; j < kUnroll; ++j) {
-          const uint64_t key = score_key(v[j]);
-          const bool in = t0 + j * blockDim.x < hi && (key & pmask) == prefix;
-          if (in) atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
+          for (int j = 0; j < kUnroll; ++j) {
+            const int64_t t = t0 + j * blockDim.x;
+            v[j] = t < hi ? __ldg(s + t) : 0.0;
+          }
+#pragma unroll
+          for (int j = 0; j < kUnroll; ++j) {
+            const uint64_t key = score_key(v[j]);
+            const bool in = t0 + j * blockDim.x < hi && (key & pmask) == prefix;
+            if (in) atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
+          }
         }
       }
       __syncthreads();
@@ -251,6 +267,29 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
       n_eq = s_eq;
       rem = shift;
       __syncthreads();
+      if (ncand < 0 && rem > 0 && n_eq <= kCandCap) {
+        // few keys share the prefix now: copy them to shared memory once, so
+        // the remaining passes read cand[] instead of every score
+        if (tid == 0) s_ncand = 0;
+        __syncthreads();
+        const uint64_t pm = ~((1ull << rem) - 1ull);
+        for (int64_t w0 = lo + (tid & ~31); w0 < hi; w0 += kUnroll * blockDim.x) {
+          const int64_t t0 = w0 + lane;
+          double v[kUnroll];
+#pragma unroll
+          for (int j = 0; j < kUnroll; ++j) {
+            const int64_t t = t0 + j * blockDim.x;
+            v[j] = t < hi ? __ldg(s + t) : 0.0;
+          }
+#pragma unroll
+          for (int j = 0; j < kUnroll; ++j) {
+            const uint64_t key = score_key(v[j]);
+            if (t0 + j * blockDim.x < hi && (key & pm) == prefix) cand[atomicAdd(&s_ncand, 1u)] = key;
+          }
+        }
+        __syncthreads();
+        ncand = n_eq;  // exactly the keys counted in the chosen bin
+      }
     }
   }
   const uint64_t kstar = prefix;  // threshold key
@@ -393,7 +432,9 @@ cudaError_t launch_select(const double* scores, int units, int64_t T, int W, int
                           int64_t n_kept, int32_t* kept, int64_t kept_stride,
                           cudaStream_t stream) {
   (void)evict_pct;
-  const size_t smem = static_cast<size_t>((T + 31) / 32 + kSelWarps) * sizeof(uint32_t);
+  // flag words rounded up to an even count (8-byte alignment of the keys), then the keys
+  const size_t smem = static_cast<size_t>((T + 63) / 64) * 2 * sizeof(uint32_t) +
+                      static_cast<size_t>(kCandCap) * sizeof(uint64_t);
   cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;

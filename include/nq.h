@@ -116,7 +116,8 @@ nq_status nq_rope_tables_fill_host(double theta, int64_t max_pos, void *host_buf
  * (fp64 accumulation; products are exact, summation order is the kernel's).
  * K: bf16 [units][heads][T][128] with strides ks.  scores: fp64
  * [units][T], row-contiguous.  ws: device workspace of at least
- * nq_score_workspace_bytes(units, heads) bytes (holds m).  1 <= W <= T. */
+ * nq_score_workspace_bytes(units, heads) bytes (holds m), 16-byte aligned.
+ * 1 <= W <= T; heads <= 128 (more: NQ_ERR_UNSUPPORTED). */
 size_t nq_score_workspace_bytes(int units, int heads);
 nq_status nq_score(const void *K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
                    double *scores, void *ws, size_t ws_bytes, nq_stream_t stream);

@@ -109,6 +109,10 @@ def test_validation_rejects_bad_arguments(nq):
     # score: window larger than T, small workspace
     assert L.nq_score(fake, ok, 1, 8, 64, 65, fake, fake, 1 << 20, None) == nq.NQ_ERR_INVALID
     assert L.nq_score(fake, ok, 1, 8, 64, 64, fake, fake, 16, None) == nq.NQ_ERR_WORKSPACE
+    assert L.nq_score(fake, ok, 1, 129, 64, 64, fake, fake, 1 << 30, None) == nq.NQ_ERR_UNSUPPORTED
+    assert L.nq_score_static(fake, ok, 1, 129, 64, 64, fake, None) == nq.NQ_ERR_UNSUPPORTED
+    assert L.nq_e8_quantise(fake, 4, 5, fake, fake, None) == nq.NQ_ERR_INVALID
+    assert L.nq_e8_quantise(fake, -1, 3, fake, fake, None) == nq.NQ_ERR_INVALID
     # select: percentage range, stride, size limit
     assert L.nq_select(fake, 1, 100, 10, 101, fake, 100, None) == nq.NQ_ERR_INVALID
     assert L.nq_select(fake, 1, 100, 10, 50, fake, 10, None) == nq.NQ_ERR_INVALID
