@@ -105,13 +105,32 @@ __device__ __forceinline__ int32_t slot_src(const CodecArgs& a, const Tile& tl, 
 
 // RoPE table rows of a tile, staged raw: for each of the 16 slots the A row
 // (angle 256a) and the B row (angle b) of its position p = 256a + b, 512
-// bytes each, at a padded stride of kRawSlot bytes per slot.
+// bytes each, at a padded stride of kRawSlot bytes per slot.  Warp w copies
+// the rows of slots w, w + nwarps, ...: one 16-byte chunk per lane per row.
 constexpr int kRawSlot = 1024 + 16;
 constexpr int kRawBytes = kSlots * kRawSlot;
 
 __device__ __forceinline__ void issue_raw(const CodecArgs& a, int32_t src_lane, uint32_t raw,
-                                          int tid, int nthreads) {
-  // 1024 16-byte chunks; every warp runs the same number of iterations
+                                          int warp, int nwarps, int lane) {
+  for (int slot = warp; slot < kSlots; slot += nwarps) {  // warp-uniform
+    const int32_t src = __shfl_sync(0xffffffffu, src_lane, slot);
+    if (src < 0) continue;
+    const int64_t pos = a.pos_base + src;
+    int64_t hi = pos >> 8;
+    hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
+    const char* rowA = reinterpret_cast<const char*>(a.tab + hi * kHalf);
+    const char* rowB = reinterpret_cast<const char*>(a.tab + (a.n_a + (pos & 255)) * kHalf);
+    const uint32_t dst = raw + slot * kRawSlot + lane * 16;
+    cp_async16(dst, rowA + lane * 16);
+    cp_async16(dst + 512, rowB + lane * 16);
+  }
+}
+
+// Decode's variant: 1024 16-byte chunks spread over all threads (thread c
+// copies chunk c % 32 of row (c / 32) % 2 of slot c / 64, stepping by the
+// CTA size); every warp runs the same number of iterations.
+__device__ __forceinline__ void issue_raw_spread(const CodecArgs& a, int32_t src_lane, uint32_t raw,
+                                                 int tid, int nthreads) {
   for (int c = tid; c < kSlots * 64; c += nthreads) {
     const int slot = c >> 6;
     const int32_t src = __shfl_sync(0xffffffffu, src_lane, slot);
@@ -523,7 +542,7 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   if (my_tiles > 0) {
     const Tile t0 = tile(0);
     const int32_t s0 = slot_src(a, t0, slot_l);
-    if (ROPE) issue_raw(a, s0, raw, tid, nthreads);
+    if (ROPE) issue_raw(a, s0, raw, warp, nthreads / 32, lane);
     issue_rows(t0, s0, 0);
   }
   cp_async_commit();
@@ -534,7 +553,7 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   if (my_tiles > 1) {
     const Tile t1 = tile(1);
     const int32_t s1 = slot_src(a, t1, slot_l);
-    if (ROPE) issue_raw(a, s1, raw, tid, nthreads);
+    if (ROPE) issue_raw(a, s1, raw, warp, nthreads / 32, lane);
     cp_async_commit();
     issue_rows(t1, s1, 1);
     cp_async_commit();
@@ -566,7 +585,7 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
                   nthreads);
     sync();  // stage s and the raw rows are free
     if (k + 2 < my_tiles) {
-      if (ROPE) issue_raw(a, src_pref, raw, tid, nthreads);
+      if (ROPE) issue_raw(a, src_pref, raw, warp, nthreads / 32, lane);
       cp_async_commit();
       issue_rows(tile(k + 2), src_pref, s);
       cp_async_commit();
@@ -713,26 +732,36 @@ __global__ void __launch_bounds__(256, 2)
   uint32_t meta = 0;
 #pragma unroll
   for (int i = 0; i < 4 * BITS; ++i) w[i] = 0;
-  const uint32_t raw = smem_u32(cs_base + 2 * kCsBytes);  // RoPE rows of the next tile
+  // RoPE rows of tiles k+1 and k+2 in two raw buffers: one CTA barrier per tile
+  const uint32_t raw0 = smem_u32(cs_base + 2 * kCsBytes);
+  auto raw_of = [&](int64_t k) { return raw0 + static_cast<uint32_t>(k & 1) * kRawBytes; };
   auto tile = [&](int64_t k) { return tile_of(a, first + k * step); };
-  auto cs_of = [&](int b) { return reinterpret_cast<float4*>(cs_base + b * kCsBytes); };
+  auto cs_of = [&](int64_t k) { return reinterpret_cast<float4*>(cs_base + (k & 1) * kCsBytes); };
 
-  // prologue: RoPE table of tile 0, codes of tile 0, table rows of tile 1 in flight
+  // prologue: rows of tiles 0 and 1 in flight, table of tile 0 combined
   int32_t src_pref = -1;
   if (ROPE) {
-    if (my_tiles > 0) issue_raw(a, slot_src(a, tile(0), slot_l), raw, tid, nthreads);
+    if (my_tiles > 0) issue_raw_spread(a, slot_src(a, tile(0), slot_l), raw_of(0), tid, nthreads);
     cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    if (my_tiles > 0) combine_raw(raw, cs_of(0), tid, nthreads);
-    __syncthreads();
-    if (my_tiles > 1) issue_raw(a, slot_src(a, tile(1), slot_l), raw, tid, nthreads);
+    if (my_tiles > 1) issue_raw_spread(a, slot_src(a, tile(1), slot_l), raw_of(1), tid, nthreads);
     cp_async_commit();
     if (my_tiles > 2) src_pref = slot_src(a, tile(2), slot_l);
+    cp_async_wait<1>();
+    __syncthreads();
+    if (my_tiles > 0) combine_raw(raw_of(0), cs_of(0), tid, nthreads);
   }
   if (my_tiles > 0) load_codes<BITS>(a, first, warp, slot_l, w, meta);
 
   for (int64_t k = 0; k < my_tiles; ++k) {
+    if (ROPE) {
+      // rows of tile k+1 landed (everyone's), table k combined, tile k-1 decoded
+      cp_async_wait<0>();
+      __syncthreads();
+      if (k + 2 < my_tiles) issue_raw_spread(a, src_pref, raw_of(k), tid, nthreads);
+      cp_async_commit();
+      if (k + 3 < my_tiles) src_pref = slot_src(a, tile(k + 3), slot_l);
+      if (k + 1 < my_tiles) combine_raw(raw_of(k + 1), cs_of(k + 1), tid, nthreads);
+    }
     const Tile tl = tile(k);
     const int h = tl.group * a.hg + warp;
     uint32_t wc[4 * BITS];
@@ -743,7 +772,7 @@ __global__ void __launch_bounds__(256, 2)
     // the warp's previous tensor store has finished reading the tile
     if (lane == 0) bulk_wait_read_all();
     __syncwarp();
-    const uint32_t csa = smem_u32(cs_base + (k & 1) * kCsBytes) + (16 * half * kSlots + slot_l) * 16;
+    const uint32_t csa = smem_u32(cs_of(k)) + (16 * half * kSlots + slot_l) * 16;
     decode_half<BITS, ROPE>(wc, mc, csa, tile_base + slot_l * 128, slot_l & 7, half);
     fence_proxy_async_smem();
     __syncwarp();
@@ -753,16 +782,6 @@ __global__ void __launch_bounds__(256, 2)
       tma_store_4d(&out_map, tile_base, 0, y, h, tl.unit);
       tma_store_4d(&out_map, tile_base + kSlots * 128, 64, y, h, tl.unit);
       bulk_commit();
-    }
-    if (ROPE) {
-      // table of tile k+1 from the rows fetched during tile k-1; then fetch k+2
-      cp_async_wait<0>();
-      __syncthreads();  // everyone's rows landed, everyone is done with cs[(k+1)&1]
-      if (k + 1 < my_tiles) combine_raw(raw, cs_of(static_cast<int>((k + 1) & 1)), tid, nthreads);
-      __syncthreads();  // table ready, raw rows free
-      if (k + 2 < my_tiles) issue_raw(a, src_pref, raw, tid, nthreads);
-      cp_async_commit();
-      if (k + 3 < my_tiles) src_pref = slot_src(a, tile(k + 3), slot_l);
     }
   }
   if (lane == 0) bulk_wait_all();
@@ -836,7 +855,7 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
     cudaError_t e = make_out_map(&map, a, units);
     if (e != cudaSuccess) return e;
     smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes +
-           (ROPE ? 2 * kCsBytes + kRawBytes : 0);
+           (ROPE ? 2 * kCsBytes + 2 * kRawBytes : 0);
     fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE>);
   } else {
     smem = 2 * (static_cast<size_t>(rows_bytes) + (ROPE ? kCsBytes : 0)) + (ROPE ? kRawBytes : 0);
