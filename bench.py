@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--cpu-layers", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-attend", action="store_true", help="skip the decode-attention timing")
     ap.add_argument("--layers", type=int, default=0, help="override layer count (small runs)")
     ap.add_argument("--tokens", type=int, default=0, help="override token count (small runs)")
     return ap.parse_args()
@@ -449,6 +450,8 @@ def run_ours(args, world, rank, local):
     if clocks:
         line["clocks"] = clocks
 
+    if not args.no_attend:
+        line["decode_attention"] = attend_timing(args, codec, Kd, Vd, stream, world)
     if not args.no_e2e:
         line["e2e"] = e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes)
     if not args.no_cpu_baseline and rank == 0:
@@ -458,6 +461,55 @@ def run_ours(args, world, rank, local):
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_layers, device, hl=hl)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def attend_timing(args, codec, Kd, Vd, stream, world, G: int = 4):
+    """One decode step of attention (one query per query head, G query heads
+    per KV head) over the whole packed cache: nq_attend (reconstruction inside
+    the attention) against nq_decode to bf16 followed by torch's
+    scaled_dot_product_attention on the bf16 cache.  CUDA events, max over ranks."""
+    import torch.nn.functional as F
+
+    from e8_lattice_vector_nq_b200 import nq
+
+    units, heads, n = codec.units, codec.heads, codec.n
+    scale = 128 ** -0.5
+    g = torch.Generator(device=Kd.device)
+    g.manual_seed(7)
+    q = torch.randn(units, heads * G, 128, device=Kd.device, generator=g)
+    qb = q.to(torch.bfloat16).view(units, heads * G, 1, 128)
+    ws = torch.empty(max(nq.lib().nq_attend_workspace_bytes(units, heads, G, n), 16) // 4,
+                     dtype=torch.float32, device=Kd.device)
+
+    def fused():
+        nq.nq_attend(q, codec.k_store, codec.v_store, n, G, codec.rope, codec.max_pos, scale=scale,
+                     positions=codec.kept, ws=ws)
+
+    def sdpa():
+        F.scaled_dot_product_attention(qb, Kd, Vd, scale=scale, enable_gqa=True)
+
+    def unfused():
+        codec.decode(Kd, Vd)
+        sdpa()
+
+    def t(fn, reps=max(args.steps, 10)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            fn()
+        e.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(s.elapsed_time(e) / reps, world, Kd.device)
+
+    f_ms, u_ms, s_ms = t(fused), t(unfused), t(sdpa)
+    packed = codec.k_store.nbytes + codec.v_store.nbytes
+    return {"query_heads_per_kv_head": G, "tokens": n, "units": units, "kv_heads": heads,
+            "fused_ms": f_ms, "decode_then_sdpa_ms": u_ms, "sdpa_on_bf16_ms": s_ms,
+            "speedup_vs_decode_then_sdpa": u_ms / f_ms,
+            "fused_packed_read_gbs": packed / (f_ms * 1e-3) / 1e9}
 
 
 def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):

@@ -271,6 +271,64 @@ nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int
                      "nq_decode launch");
 }
 
+size_t nq_attend_workspace_bytes(int units, int heads, int G, int64_t n) {
+  if (units < 0 || heads < 1 || G < 1 || n < 1) return 0;
+  return nq::attend_workspace_floats(units, heads, G, n) * sizeof(float);
+}
+
+nq_status nq_attend(const float* q, int units, int heads, int G, const nq_packed* k_in,
+                    const nq_packed* v_in, int64_t n, int64_t slot0, const int32_t* positions,
+                    int64_t pos_stride, int64_t pos_base, const float* rope_tab,
+                    int64_t rope_max_pos, float scale, float* out, float* lse, void* ws,
+                    size_t ws_bytes, nq_stream_t stream) {
+  if (units < 0 || heads < 1 || heads > 1024 || G < 1 || G > 8)
+    return fail(NQ_ERR_INVALID, "need units >= 0, 1 <= heads <= 1024, 1 <= G <= 8");
+  if (n < 1 || slot0 < 0 || pos_base < 0)
+    return fail(NQ_ERR_INVALID, "need n >= 1, slot0 >= 0, pos_base >= 0");
+  if (!std::isfinite(scale)) return fail(NQ_ERR_INVALID, "scale must be finite");
+  if (units == 0) return NQ_OK;
+  if (!q || !aligned(q, 16)) return fail(NQ_ERR_INVALID, "q NULL or not 16-byte aligned");
+  if (!out || !aligned(out, 4)) return fail(NQ_ERR_INVALID, "out NULL or misaligned");
+  if (lse && !aligned(lse, 4)) return fail(NQ_ERR_INVALID, "lse misaligned");
+  if (nq_status st = check_packed(k_in, "k_in")) return st;
+  if (nq_status st = check_packed(v_in, "v_in")) return st;
+  if (nq_status st = check_rope(rope_tab, rope_max_pos)) return st;
+  if (positions) {
+    if (!aligned(positions, 4)) return fail(NQ_ERR_INVALID, "positions misaligned");
+    if (pos_stride < n) return fail(NQ_ERR_INVALID, "pos_stride < n");
+  } else if (pos_base + n > rope_max_pos) {
+    return fail(NQ_ERR_INVALID, "positions up to %lld exceed rope_max_pos %lld",
+                static_cast<long long>(pos_base + n - 1), static_cast<long long>(rope_max_pos));
+  }
+  if (!ws || !aligned(ws, 16)) return fail(NQ_ERR_INVALID, "workspace NULL or not 16-byte aligned");
+  const size_t need = nq_attend_workspace_bytes(units, heads, G, n);
+  if (ws_bytes < need)
+    return fail(NQ_ERR_WORKSPACE, "attend workspace too small: %zu < %zu", ws_bytes, need);
+  if (static_cast<int64_t>(units) * heads * ((n + 255) / 256) > 0x7FFFFFFF ||
+      static_cast<int64_t>(units) * heads * G > 0x7FFFFFFF)
+    return fail(NQ_ERR_UNSUPPORTED, "units * heads * chunks too large for one launch");
+  nq::AttendLaunch L{};
+  L.q = q;
+  L.units = units;
+  L.heads = heads;
+  L.G = G;
+  L.k_in = *k_in;
+  L.v_in = *v_in;
+  L.n = n;
+  L.slot0 = slot0;
+  L.positions = positions;
+  L.pos_stride = pos_stride;
+  L.pos_base = pos_base;
+  L.rope_tab = rope_tab;
+  L.rope_max_pos = rope_max_pos;
+  L.scale = scale;
+  L.out = out;
+  L.lse = lse;
+  L.ws = ws;
+  return cuda_status(nq::launch_attend(L, reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_attend launch");
+}
+
 nq_status nq_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
                          uint8_t* coset, nq_stream_t stream) {
   if (bits != 2 && bits != 3) return fail(NQ_ERR_INVALID, "bits must be 2 or 3 (got %d)", bits);

@@ -42,10 +42,27 @@ struct DecodeLaunch {
   nq_kv_strides vos;
 };
 
+struct AttendLaunch {
+  const float* q;
+  int units, heads, G;
+  nq_packed k_in, v_in;
+  int64_t n, slot0;
+  const int32_t* positions;
+  int64_t pos_stride, pos_base;
+  const float* rope_tab;
+  int64_t rope_max_pos;
+  float scale;
+  float* out;
+  float* lse;
+  void* ws;
+};
+
 cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 
 cudaError_t codec_read_clear_error(uint32_t* flags);
+size_t attend_workspace_floats(int units, int heads, int G, int64_t n);
+cudaError_t launch_attend(const AttendLaunch& L, cudaStream_t stream);
 cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
                                uint8_t* coset, cudaStream_t stream);
 

@@ -42,7 +42,8 @@ EXPORTS = (
     "nq_last_error", "nq_version", "nq_packed_bytes_per_vector", "nq_rope_tables_bytes",
     "nq_rope_tables_fill_host", "nq_score_workspace_bytes", "nq_score", "nq_score_static",
     "nq_kept_count",
-    "nq_select", "nq_encode", "nq_decode", "nq_e8_quantise", "nq_device_error",
+    "nq_select", "nq_encode", "nq_decode", "nq_e8_quantise", "nq_attend_workspace_bytes",
+    "nq_attend", "nq_device_error",
 )
 
 
@@ -72,6 +73,9 @@ def lib() -> ctypes.CDLL:
         "nq_decode": (i32, [PK, PK, i32, i32, i64, i64, P, i64, i64, P, i64, P, KVStrides, P,
                             KVStrides, P]),
         "nq_e8_quantise": (i32, [P, i64, i32, P, P, P]),
+        "nq_attend_workspace_bytes": (sz, [i32, i32, i32, i64]),
+        "nq_attend": (i32, [P, i32, i32, i32, PK, PK, i64, i64, P, i64, i64, P, i64,
+                            ctypes.c_float, P, P, P, sz, P]),
         "nq_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32)]),
     }
     for name, (res, args) in sig.items():
@@ -257,6 +261,37 @@ def nq_decode(k_in: PackedStore | None, v_in: PackedStore | None, n: int,
                            positions.stride(0) if positions is not None else 0, int(pos_base),
                            _ptr(rope_tab), int(rope_max_pos), _ptr(K_out), kos, _ptr(V_out),
                            vos, _stream(stream)))
+
+
+def nq_attend(q: torch.Tensor, k_in: PackedStore, v_in: PackedStore, n: int, G: int,
+              rope_tab: torch.Tensor, rope_max_pos: int, scale: float | None = None,
+              positions: torch.Tensor | None = None, pos_base: int = 0, slot0: int = 0,
+              ws: torch.Tensor | None = None, stream=None):
+    """Decode-phase attention of q [units][heads*G][128] (fp32) over n packed
+    slots per (unit, KV head): returns (out fp32 [units][heads*G][128],
+    lse fp32 [units][heads*G]) (see nq.h, nq_attend)."""
+    _require_cuda(q, positions, rope_tab)
+    if q.dtype != torch.float32 or not q.is_contiguous() or q.dim() != 3 or q.shape[2] != 128:
+        raise ValueError("q must be a contiguous float32 [units, heads*G, 128] tensor")
+    units, Hq = q.shape[0], q.shape[1]
+    heads = k_in.meta.shape[1]
+    if Hq != heads * G:
+        raise ValueError("q has %d heads, expected heads * G = %d" % (Hq, heads * G))
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.stride(-1) == 1
+    out = torch.empty(units, Hq, 128, dtype=torch.float32, device=q.device)
+    lse = torch.empty(units, Hq, dtype=torch.float32, device=q.device)
+    need = lib().nq_attend_workspace_bytes(units, heads, G, int(n))
+    if ws is None or ws.numel() * ws.element_size() < need:
+        ws = torch.empty(max(need, 16) // 4, dtype=torch.float32, device=q.device)
+    kd, vd = k_in.desc(), v_in.desc()
+    _check(lib().nq_attend(_ptr(q), units, heads, int(G), ctypes.byref(kd), ctypes.byref(vd),
+                           int(n), int(slot0), _ptr(positions),
+                           positions.stride(0) if positions is not None else 0, int(pos_base),
+                           _ptr(rope_tab), int(rope_max_pos),
+                           float(scale if scale is not None else 128 ** -0.5), _ptr(out),
+                           _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return out, lse
 
 
 def nq_e8_quantise(y: torch.Tensor, bits: int, stream=None):

@@ -210,6 +210,33 @@ nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int
                     int64_t pos_base, const float *rope_tab, int64_t rope_max_pos, void *K_out,
                     nq_kv_strides kos, void *V_out, nq_kv_strides vos, nq_stream_t stream);
 
+/* ----------------------------------------------------- decode attention
+ * Decode-phase attention over the packed cache, reconstructing keys and
+ * values inside the attention (the on-demand reconstruction within
+ * FlashAttention described for VQKV, section "Decoding"; the NexusQuant pages
+ * give no attention formula, so this reading is the library's):
+ *   for unit u, query head j (KV head h = j / G), over the n slots
+ *   slot0 .. slot0+n-1 of (u, h):
+ *     s_t = scale * dot(q[u][j], k_t)      k_t: the fp32 key that nq_decode
+ *                                          rounds to bf16 (RoPE re-applied at
+ *                                          pos = pos_base + (positions ?
+ *                                          positions[u*pos_stride + t] : t))
+ *     out[u][j] = sum_t softmax(s)_t v_t   v_t: the fp32 value before bf16
+ *     lse[u][j] = log(sum_t exp(s_t))      (natural log; lse may be NULL)
+ * fp32 arithmetic in the kernels' own order (scores, fp32 exp, chunked
+ * sums), so results agree with an exact evaluation to about 1e-5 relative,
+ * not bit for bit.  q: fp32 [units][heads*G][128], 16-byte aligned.
+ * out: fp32 [units][heads*G][128].  k_in/v_in: packed stores as for
+ * nq_decode (any bits 2/3).  1 <= G <= 8, n >= 1.  ws: device workspace of
+ * nq_attend_workspace_bytes(units, heads, G, n) bytes, 16-byte aligned
+ * (per-chunk partial results).  rope_tab as for nq_decode. */
+size_t nq_attend_workspace_bytes(int units, int heads, int G, int64_t n);
+nq_status nq_attend(const float *q, int units, int heads, int G, const nq_packed *k_in,
+                    const nq_packed *v_in, int64_t n, int64_t slot0, const int32_t *positions,
+                    int64_t pos_stride, int64_t pos_base, const float *rope_tab,
+                    int64_t rope_max_pos, float scale, float *out, float *lse, void *ws,
+                    size_t ws_bytes, nq_stream_t stream);
+
 /* ------------------------------------------------------ E8 quantiser
  * The lattice step of nq_encode on its own ([NQ-zh] "E8 lattice
  * quantisation"; [NQ-pt] step 4), for coordinates that are already rotated

@@ -67,6 +67,10 @@ def _load():
             "oq_decode_unit": (None, [P, P, P, P, i32, i64, P, i64, dbl, i32, i32, P, P]),
             "oq_e8_batch": (None, [P, i64, P, P, P]),
             "oq_e8_code_batch": (None, [P, i64, ctypes.c_int, P, P]),
+            "oq_reconstruct_batch": (None, [P, P, i64, ctypes.c_int, P, P, ctypes.c_int, P]),
+            "oq_attend_unit": (None, [P, P, P, P, ctypes.c_int, ctypes.c_int, i64, P, i64,
+                                      ctypes.c_double, ctypes.c_int, ctypes.c_int, P,
+                                      ctypes.c_double, P, P]),
             "oq_fwht_batch": (None, [P, i64]),
             "oq_f32_to_f16_batch": (None, [P, i64, P]),
             "oq_f32_to_bf16_batch": (None, [P, i64, P]),
@@ -204,6 +208,22 @@ def decode_vectors(words, meta, bits: int, rope: bool = False, c=None, s=None):
     return out
 
 
+def reconstruct_vectors(words, meta, bits: int, rope: bool = False, c=None, s=None):
+    """fp32 reconstructions [n][128] of [n] packed vectors (the decode output
+    before its bf16 rounding)."""
+    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, 4 * bits)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32).ravel()
+    n = words.shape[0]
+    if c is None:
+        c = np.zeros((n, D // 2), np.float32)
+        s = np.zeros((n, D // 2), np.float32)
+    c = np.ascontiguousarray(c, dtype=np.float32).reshape(n, D // 2)
+    s = np.ascontiguousarray(s, dtype=np.float32).reshape(n, D // 2)
+    out = np.empty((n, D), np.float32)
+    _load().oq_reconstruct_batch(_p(words), _p(meta), n, int(rope), _p(c), _p(s), bits, _p(out))
+    return out
+
+
 # ------------------------------------------------------ unit level
 def score_unit(K_unit, W: int, return_mean: bool = False):
     """Key-key proxy scores of one layer; K_unit [H][T][128] bf16."""
@@ -263,3 +283,21 @@ def decode_unit(k_codes, k_meta, v_codes, v_meta, positions=None, pos_base: int 
     _load().oq_decode_unit(_p(kc), _p(km), _p(vc), _p(vm), H, n, _p(pp), int(pos_base),
                            float(theta), bits_k, bits_v, _p(Ko), _p(Vo))
     return Ko, Vo
+
+
+def attend_unit(k_codes, k_meta, v_codes, v_meta, q, G: int, scale: float, positions=None,
+                pos_base: int = 0, theta: float = 1e4, bits_k: int = 3, bits_v: int = 2):
+    """Decode-phase attention of q [H*G][128] (fp32) over one packed unit
+    ([H][n] vectors): returns (out fp64 [H*G][128], lse fp64 [H*G])."""
+    kc = np.ascontiguousarray(k_codes, dtype=np.uint32)
+    km = np.ascontiguousarray(k_meta, dtype=np.uint32)
+    vc = np.ascontiguousarray(v_codes, dtype=np.uint32)
+    vm = np.ascontiguousarray(v_meta, dtype=np.uint32)
+    H, n = km.shape
+    q = np.ascontiguousarray(q, dtype=np.float32).reshape(H * G, D)
+    pp = None if positions is None else np.ascontiguousarray(positions, dtype=np.int32)
+    out = np.empty((H * G, D), np.float64)
+    lse = np.empty(H * G, np.float64)
+    _load().oq_attend_unit(_p(kc), _p(km), _p(vc), _p(vm), H, G, n, _p(pp), int(pos_base),
+                           float(theta), bits_k, bits_v, _p(q), float(scale), _p(out), _p(lse))
+    return out, lse

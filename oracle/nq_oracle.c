@@ -318,10 +318,12 @@ int oq_encode_vector(const uint16_t *x, int rope, const float *c, const float *s
  *  w   = FWHT(t)                 (integers, |w| <= 896: exact in fp32)
  *  kappa = fp32(fp32(sigma / 2) * C);  x_c = fp32(w_c * kappa)
  *  keys: re-apply RoPE at this position; then bf16 round-to-nearest-even. */
-void oq_decode_vector(const uint32_t *words, uint32_t meta, int rope, const float *c,
-                      const float *s, int bits, uint16_t *out)
+/* The fp32 reconstruction of one packed vector, before the bf16 rounding of
+ * the decode output: codes -> 2q -> Walsh-Hadamard -> x = fp32(w * kappa),
+ * keys re-rotated (RoPE at the (c, s) row given). */
+void oq_reconstruct_vector(const uint32_t *words, uint32_t meta, int rope, const float *c,
+                           const float *s, int bits, float *w)
 {
-    float w[OQ_D];
     for (int cidx = 0; cidx < OQ_D; cidx++) {
         uint32_t j = 0;
         int bitpos = bits * cidx;
@@ -336,6 +338,13 @@ void oq_decode_vector(const uint32_t *words, uint32_t meta, int rope, const floa
     float kappa = (sig * 0.5f) * oq_u2f(OQ_C_BITS);
     for (int i = 0; i < OQ_D; i++) w[i] = w[i] * kappa;
     if (rope) oq_rope_redo(w, c, s);
+}
+
+void oq_decode_vector(const uint32_t *words, uint32_t meta, int rope, const float *c,
+                      const float *s, int bits, uint16_t *out)
+{
+    float w[OQ_D];
+    oq_reconstruct_vector(words, meta, rope, c, s, bits, w);
     for (int i = 0; i < OQ_D; i++) out[i] = oq_f32_to_bf16(w[i]);
 }
 
@@ -469,6 +478,67 @@ void oq_decode_unit(const uint32_t *k_codes, const uint32_t *k_meta, const uint3
                                  V_out + vec * OQ_D);
         }
     }
+}
+
+/* ------------------------------------------------------ decode attention */
+
+/* Attention of G query heads per KV head over one packed unit (decode phase:
+ * one query vector per head).  This is the reading taken for attention on
+ * the compressed cache (the pages only say that reconstruction happens inside
+ * the attention computation, VQKV "Decoding": rebuild the needed KV pieces on
+ * demand within FlashAttention): scaled dot-product softmax attention over the
+ * fp32 reconstructions of the n kept tokens, keys re-rotated at their
+ * positions.  Query head j attends with KV head j / G.  Everything after the
+ * fp32 reconstruction is fp64:
+ *   s_t = scale * sum_i q_i k_t,i,  m = max_t s_t,  l = sum_t exp(s_t - m),
+ *   o   = sum_t exp(s_t - m) v_t / l,  lse = m + log(l).
+ * q [H*G][128] fp32, out [H*G][128] fp64, lse [H*G] fp64.  Codes/meta are
+ * [H][n] vectors as in oq_decode_unit.  n >= 1. */
+void oq_attend_unit(const uint32_t *k_codes, const uint32_t *k_meta, const uint32_t *v_codes,
+                    const uint32_t *v_meta, int H, int G, int64_t n, const int32_t *positions,
+                    int64_t pos_base, double theta, int bits_k, int bits_v, const float *q,
+                    double scale, double *out, double *lse)
+{
+    float c[OQ_HALF], sn[OQ_HALF], k[OQ_D], v[OQ_D];
+    double *sc = (double *)malloc((size_t)n * (size_t)G * sizeof(double));
+    for (int h = 0; h < H; h++) {
+        for (int64_t t = 0; t < n; t++) {
+            int64_t pos = pos_base + (positions ? (int64_t)positions[t] : t);
+            size_t vec = (size_t)h * n + (size_t)t;
+            oq_rope_cs(theta, pos, c, sn);
+            oq_reconstruct_vector(k_codes + vec * 4 * bits_k, k_meta[vec], 1, c, sn, bits_k, k);
+            for (int g = 0; g < G; g++) {
+                const float *qj = q + (size_t)(h * G + g) * OQ_D;
+                double dot = 0.0;
+                for (int i = 0; i < OQ_D; i++) dot += (double)qj[i] * (double)k[i];
+                sc[(size_t)t * G + g] = scale * dot;
+            }
+        }
+        for (int g = 0; g < G; g++) {
+            double m = -INFINITY, l = 0.0, acc[OQ_D];
+            for (int64_t t = 0; t < n; t++) m = fmax(m, sc[(size_t)t * G + g]);
+            for (int i = 0; i < OQ_D; i++) acc[i] = 0.0;
+            for (int64_t t = 0; t < n; t++) {
+                size_t vec = (size_t)h * n + (size_t)t;
+                double p = exp(sc[(size_t)t * G + g] - m);
+                l += p;
+                oq_reconstruct_vector(v_codes + vec * 4 * bits_v, v_meta[vec], 0, c, sn, bits_v, v);
+                for (int i = 0; i < OQ_D; i++) acc[i] += p * (double)v[i];
+            }
+            for (int i = 0; i < OQ_D; i++) out[(size_t)(h * G + g) * OQ_D + i] = acc[i] / l;
+            lse[h * G + g] = m + log(l);
+        }
+    }
+    free(sc);
+}
+
+/* fp32 reconstructions of a batch of vectors (keys: rope = 1 with c, s rows). */
+void oq_reconstruct_batch(const uint32_t *words, const uint32_t *meta, int64_t n, int rope,
+                          const float *c, const float *s, int bits, float *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        oq_reconstruct_vector(words + 4 * bits * i, meta[i], rope, c + OQ_HALF * i,
+                              s + OQ_HALF * i, bits, out + OQ_D * i);
 }
 
 /* ------------------------------------------------ helpers for the pins */

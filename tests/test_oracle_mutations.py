@@ -50,6 +50,11 @@ MUTATIONS = [
      "tests/test_oracle_select.py::test_select_ties_prefer_lower_position"),
     ("kept-count", "return T - (mid * pct) / 100;", "return T - (T * pct) / 100;",
      "tests/test_oracle_select.py::test_kept_count_rule"),
+    ("attend-gqa-index", "const float *qj = q + (size_t)(h * G + g) * OQ_D;",
+     "const float *qj = q + (size_t)(g * H + h) * OQ_D;",
+     "tests/test_oracle_attend.py::test_attention_equals_library_softmax"),
+    ("attend-lse", "lse[h * G + g] = m + log(l);", "lse[h * G + g] = log(l);",
+     "tests/test_oracle_attend.py::test_attention_equals_library_softmax"),
 ]
 
 
