@@ -286,8 +286,10 @@ __global__ void __launch_bounds__(32) attend_combine_kernel(const AttendArgs a, 
   const float* base = a.part + ((u * a.heads + h) * a.nsplit) * a.GT * kPartFloats + g * kPartFloats;
   const int64_t sstride = static_cast<int64_t>(a.GT) * kPartFloats;
   float M = -INFINITY;
+#pragma unroll 8
   for (int64_t s = 0; s < a.nsplit; ++s) M = fmaxf(M, base[s * sstride]);
   float L = 0.f, A[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
   for (int64_t s = 0; s < a.nsplit; ++s) {
     const float* p = base + s * sstride;
     const float f = __expf(p[0] - M);
