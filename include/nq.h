@@ -136,7 +136,8 @@ nq_status nq_score(const void *K, nq_kv_strides ks, int units, int heads, int64_
  * NQ_SCORE_STATIC_MAX_VECTORS (unit, head) pairs (1 MiB); every GPU that
  * loads the library holds that array until the process exits.  It calls no
  * cudaMalloc, cudaFree or other allocating routine.
- *   - units * heads above the maximum: NQ_ERR_UNSUPPORTED, nothing launched.
+ *   - units * heads above the maximum, or heads above 128: NQ_ERR_UNSUPPORTED,
+ *     nothing launched.
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before
  *     any stream capture.
