@@ -76,6 +76,8 @@ struct CodecArgs {
   int64_t n_a;
   int64_t slot_tiles, num_tiles;
   FastDiv div_groups, div_stiles;
+  int64_t pairs;  // encode: units * n (unit, slot) pairs, below 2^31
+  FastDiv div_n;  // encode: division by n
 };
 
 struct Tile {
@@ -102,6 +104,42 @@ __device__ __forceinline__ int32_t slot_src(const CodecArgs& a, const Tile& tl, 
   if (slot >= a.n) return -1;
   return a.idx ? __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot)
                : static_cast<int32_t>(slot);
+}
+
+// Encode tiles walk the (unit, slot) pairs of all units as one list, 16 pairs
+// per tile (pair p = unit * n + slot), so a tile may span units: an append of
+// one token per unit fills whole tiles.  Tile index -> (head group, p0).
+struct EncTile {
+  int group;
+  int64_t p0;
+};
+__device__ __forceinline__ EncTile enc_tile(const CodecArgs& a, int64_t t64) {
+  const uint32_t t = static_cast<uint32_t>(t64);
+  const uint32_t q = fdiv(t, a.div_groups);
+  EncTile r;
+  r.group = static_cast<int>(t - q * a.div_groups.d);
+  r.p0 = static_cast<int64_t>(q) * kSlots;
+  return r;
+}
+// This lane's pair of a tile (lanes l and l+16 share pair p0 + l % 16).
+struct EncPair {
+  bool valid;
+  int64_t unit, slot;
+};
+__device__ __forceinline__ EncPair enc_pair(const CodecArgs& a, int64_t p0, int slot_l) {
+  EncPair e;
+  const int64_t p = p0 + slot_l;
+  e.valid = p < a.pairs;
+  const uint32_t pp = static_cast<uint32_t>(e.valid ? p : 0);
+  const uint32_t u = fdiv(pp, a.div_n);
+  e.unit = u;
+  e.slot = static_cast<int64_t>(pp) - static_cast<int64_t>(u) * a.n;
+  return e;
+}
+// Source token of a pair (its RoPE position is pos_base + src), -1 if invalid.
+__device__ __forceinline__ int32_t enc_src(const CodecArgs& a, const EncPair& e) {
+  if (!e.valid) return -1;
+  return a.idx ? __ldg(a.idx + e.unit * a.idx_stride + e.slot) : static_cast<int32_t>(e.slot);
 }
 
 // RoPE table rows of a tile, staged raw: for each of the 16 slots the A row
@@ -478,22 +516,23 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
 
   const int64_t first = blockIdx.x, step = gridDim.x;
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
-  auto tile = [&](int64_t k) { return tile_of(a, first + k * step); };
+  auto tile = [&](int64_t k) { return enc_tile(a, first + k * step); };
 
-  // The warp's 16 rows (one head, 16 slots) with 16-byte async copies: in copy
-  // j, lane l moves chunk l%16 of row 2j + l/16, two whole rows per instruction.
-  auto issue_rows = [&](const Tile& tl, int32_t src_lane, int s) {
+  // The warp's 16 rows (one head, 16 pairs) with 16-byte async copies: in copy
+  // j, lane l moves chunk l%16 of row 2j + l/16, two whole rows per
+  // instruction.  Each lane supplies its pair's row offset in elements
+  // (unit * su + token * st, -1 past the last pair) through a shuffle.
+  auto issue_rows = [&](const EncTile& tl, const EncPair& ep, int32_t src, int s) {
     const int h = tl.group * a.hg + warp;
-    const uint16_t* base = a.kv + tl.unit * a.su + h * a.sh + slot_l * 8;
+    const int64_t tok = src < a.T_in ? src : a.T_in - 1;
+    const long long roff = src >= 0 ? static_cast<long long>(ep.unit * a.su + tok * a.st) : -1ll;
+    const uint16_t* base = a.kv + h * a.sh + slot_l * 8;
     const uint32_t dst0 = smem_u32(smem + s * stage_bytes + warp * kSlots * kRowPad) + slot_l * 16;
 #pragma unroll
     for (int j = 0; j < kSlots / 2; ++j) {
       const int r = 2 * j + half;
-      const int32_t tok = __shfl_sync(0xffffffffu, src_lane, r);
-      if (tok >= 0) {
-        const int64_t t = tok < a.T_in ? tok : a.T_in - 1;
-        cp_async16(dst0 + r * kRowPad, base + t * a.st);
-      }
+      const long long ro = __shfl_sync(0xffffffffu, roff, r);
+      if (ro >= 0) cp_async16(dst0 + r * kRowPad, base + ro);
     }
   };
   // cross-warp data (the shared RoPE table) needs the CTA barrier; value
@@ -504,12 +543,14 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   };
 
   // prologue: tile 0 (rows + its RoPE table), then tile 1 in flight
+  EncPair pp_pref{};
   int32_t src_pref = -1;
   if (my_tiles > 0) {
-    const Tile t0 = tile(0);
-    const int32_t s0 = slot_src(a, t0, slot_l);
+    const EncTile t0 = tile(0);
+    const EncPair p0 = enc_pair(a, t0.p0, slot_l);
+    const int32_t s0 = enc_src(a, p0);
     if (ROPE) issue_raw(a, s0, raw, warp, nthreads / 32, lane);
-    issue_rows(t0, s0, 0);
+    issue_rows(t0, p0, s0, 0);
   }
   cp_async_commit();
   cp_async_wait<0>();
@@ -517,17 +558,21 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   if (ROPE && my_tiles > 0) combine_raw(raw, reinterpret_cast<float4*>(smem + rows_bytes), tid, nthreads);
   sync();
   if (my_tiles > 1) {
-    const Tile t1 = tile(1);
-    const int32_t s1 = slot_src(a, t1, slot_l);
+    const EncTile t1 = tile(1);
+    const EncPair p1 = enc_pair(a, t1.p0, slot_l);
+    const int32_t s1 = enc_src(a, p1);
     if (ROPE) issue_raw(a, s1, raw, warp, nthreads / 32, lane);
     cp_async_commit();
-    issue_rows(t1, s1, 1);
+    issue_rows(t1, p1, s1, 1);
     cp_async_commit();
   } else {
     cp_async_commit();
     cp_async_commit();
   }
-  if (my_tiles > 2) src_pref = slot_src(a, tile(2), slot_l);
+  if (my_tiles > 2) {
+    pp_pref = enc_pair(a, tile(2).p0, slot_l);
+    src_pref = enc_src(a, pp_pref);
+  }
 
   // Per iteration two groups are committed, [RoPE rows of k+2] then [rows of
   // k+2]; waiting for all but the newest leaves only rows(k+1) in flight.
@@ -536,12 +581,11 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
     cp_async_wait<1>();
     sync();
 
-    const Tile tl = tile(k);
+    const EncTile tl = tile(k);
     const int h = tl.group * a.hg + warp;
-    const int64_t slot = tl.stile * kSlots + slot_l;
-    const bool valid = slot < a.n;
+    const EncPair ep = enc_pair(a, tl.p0, slot_l);
     unsigned char* st = smem + s * stage_bytes;
-    // lanes past the last slot run on whatever their staging row holds; none
+    // lanes past the last pair run on whatever their staging row holds; none
     // of their results is stored
     float2 v[32];
     load_half<ROPE>(v, smem_u32(st + row_idx * kRowPad),
@@ -553,15 +597,18 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
     if (k + 2 < my_tiles) {
       if (ROPE) issue_raw(a, src_pref, raw, warp, nthreads / 32, lane);
       cp_async_commit();
-      issue_rows(tile(k + 2), src_pref, s);
+      issue_rows(tile(k + 2), pp_pref, src_pref, s);
       cp_async_commit();
-      if (k + 3 < my_tiles) src_pref = slot_src(a, tile(k + 3), slot_l);  // used next iteration
+      if (k + 3 < my_tiles) {  // used next iteration
+        pp_pref = enc_pair(a, tile(k + 3).p0, slot_l);
+        src_pref = enc_src(a, pp_pref);
+      }
     } else {
       cp_async_commit();
       cp_async_commit();
     }
-    const int64_t vec = tl.unit * a.pu + h * a.ph + a.slot0 + slot;
-    quantise_half<BITS>(v, half, valid, a.codes + vec * (4 * BITS), a.meta + vec);
+    const int64_t vec = ep.unit * a.pu + h * a.ph + a.slot0 + ep.slot;
+    quantise_half<BITS>(v, half, ep.valid, a.codes + vec * (4 * BITS), a.meta + vec);
   }
   cp_async_wait<0>();
 }
@@ -759,7 +806,15 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   a.hg = pick_head_group(a.heads);
   a.ngroups = a.heads / a.hg;
   a.slot_tiles = (a.n + kSlots - 1) / kSlots;
-  a.num_tiles = static_cast<int64_t>(units) * a.slot_tiles * a.ngroups;
+  if (decode) {
+    a.num_tiles = static_cast<int64_t>(units) * a.slot_tiles * a.ngroups;
+  } else {
+    // encode: tiles of 16 (unit, slot) pairs over all units
+    a.pairs = static_cast<int64_t>(units) * a.n;
+    if (a.pairs >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+    a.num_tiles = (a.pairs + kSlots - 1) / kSlots * a.ngroups;
+    if (a.n > 0) a.div_n = make_fastdiv(static_cast<uint32_t>(a.n));
+  }
   if (a.num_tiles == 0) return cudaSuccess;
   if (a.num_tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
   a.div_groups = make_fastdiv(static_cast<uint32_t>(a.ngroups));
