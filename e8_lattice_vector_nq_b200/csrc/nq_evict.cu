@@ -9,18 +9,23 @@
 //   window_mean_kernel: m[u][h][d] = fp32(fp64 sum of the last W keys / W)
 //   score_kernel:       scores[u][t] = sum_h sum_d K[u][h][t][d] * m[u][h][d]
 //                       in fp64 (one coalesced pass over K)
-//   select_kernel:      per unit, an MSD radix select (11-bit digits, after
-//                       the prefix that every middle key shares) of the
+//   select_kernel:      per unit (one cluster of 4 CTAs sharing histograms
+//                       through distributed shared memory), an MSD radix
+//                       select (11-bit digits, after the prefix that every
+//                       middle key shares) of the
 //                       (score desc, position asc) threshold on
 //                       order-preserving 64-bit keys; once at most 8192 keys
 //                       share the prefix they move to shared memory and the
 //                       remaining digits are read from there; then an
 //                       ordered compaction with warp ballots.
+#include <cooperative_groups.h>
+
 #include <mutex>
 
 #include "nq_internal.h"
 
 namespace nq {
+namespace cg = cooperative_groups;
 
 // ----------------------------------------------------------- window mean
 __global__ void window_mean_kernel(const uint16_t* __restrict__ K, nq_kv_strides ks, int heads,
@@ -123,33 +128,52 @@ constexpr int kDigitBits = 11;
 constexpr int kUnroll = 8;  // independent score loads in flight per thread
 constexpr int kBins = 1 << kDigitBits;  // 2 bins per thread
 constexpr int kCandCap = 8192;          // candidate keys kept in shared memory
+constexpr int kSelCluster = 4;          // CTAs (one cluster) per unit
 
+// One unit per cluster of kSelCluster CTAs (thread-block cluster, distributed
+// shared memory).  CTA r owns the r-th contiguous slice of the middle range for
+// the radix passes and the r-th contiguous segment of positions for the
+// ordered compaction.  Every radix pass builds a local histogram, then each
+// CTA sums the cluster's histograms for its two bins through DSMEM and runs
+// the same descending scan, so all CTAs derive the same prefix and rank; the
+// compaction offsets are exclusive sums over the lower-ranked CTAs' counts.
+// Every CTA of a cluster executes the same sequence of cluster barriers.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __restrict__ scores,
                                                              int64_t T, int W, int64_t n_kept,
                                                              int32_t* __restrict__ kept,
                                                              int64_t kept_stride) {
-  extern __shared__ uint32_t flagbits[];  // ceil(T/32) words, then the candidate keys
-  uint64_t* cand = reinterpret_cast<uint64_t*>(flagbits + ((T + 63) / 64) * 2);
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  extern __shared__ uint32_t flagbits[];  // this CTA's segment flag words, then candidate keys
   __shared__ unsigned int hist[kBins];
-  __shared__ unsigned int s_ncand;
   __shared__ uint64_t s_min[kSelWarps], s_max[kSelWarps];
+  __shared__ uint64_t c_minmax[2];        // this CTA's min and max key (read by the cluster)
   __shared__ unsigned int s_wsum[kSelWarps];
   __shared__ uint64_t s_prefix;
   __shared__ int64_t s_k;
   __shared__ int64_t s_eq;
   __shared__ int warp_cnt[kSelWarps];
+  __shared__ long long c_count[2];        // this CTA's tie and kept counts (read by the cluster)
+  __shared__ unsigned int s_ncand;
 
-  const int u = blockIdx.x;
+  const int u = blockIdx.x / kSelCluster;
   const double* s = scores + static_cast<int64_t>(u) * T;
   int32_t* out = kept + static_cast<int64_t>(u) * kept_stride;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // this CTA's segment of positions, a multiple of 32 wide
+  const int64_t seg_cta = ((T + kSelCluster - 1) / kSelCluster + 31) / 32 * 32;
+  const int64_t S0 = min64(T, rank * seg_cta), S1 = min64(T, S0 + seg_cta);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(flagbits + ((seg_cta + 63) / 64) * 2);
 
-  if (n_kept >= T) {
-    for (int64_t t = tid; t < T; t += blockDim.x) out[t] = static_cast<int32_t>(t);
+  if (n_kept >= T) {  // the same branch in every CTA: no barrier pending
+    for (int64_t t = S0 + tid; t < S1; t += blockDim.x) out[t] = static_cast<int32_t>(t);
     return;
   }
   const int64_t lo = 1, hi = T - W;  // middle range [lo, hi)
   const int64_t n_mid = n_kept - 1 - W;
+  // this CTA's slice of the middle range
+  const int64_t sl = (hi - lo + kSelCluster - 1) / kSelCluster;
+  const int64_t A0 = min64(hi, lo + rank * sl), A1 = min64(hi, A0 + sl);
 
   // --- radix select: the n_mid-th largest key among the middle tokens
   uint64_t prefix = 0;
@@ -158,16 +182,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   if (n_mid > 0) {
     // every candidate key lies in [kmin, kmax], so they share its common prefix
     uint64_t kmin = ~0ull, kmax = 0ull;
-    for (int64_t t0 = lo + tid; t0 < hi; t0 += kUnroll * blockDim.x) {
+    for (int64_t t0 = A0 + tid; t0 < A1; t0 += kUnroll * blockDim.x) {
       double v[kUnroll];
 #pragma unroll
       for (int j = 0; j < kUnroll; ++j) {
         const int64_t t = t0 + j * blockDim.x;
-        v[j] = t < hi ? __ldg(s + t) : 0.0;
+        v[j] = t < A1 ? __ldg(s + t) : 0.0;
       }
 #pragma unroll
       for (int j = 0; j < kUnroll; ++j) {
-        if (t0 + j * blockDim.x < hi) {
+        if (t0 + j * blockDim.x < A1) {
           const uint64_t key = score_key(v[j]);
           kmin = key < kmin ? key : kmin;
           kmax = key > kmax ? key : kmax;
@@ -192,15 +216,20 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
         mn = s_min[w] < mn ? s_min[w] : mn;
         mx = s_max[w] > mx ? s_max[w] : mx;
       }
-      s_min[0] = mn;
-      s_max[0] = mx;
+      c_minmax[0] = mn;
+      c_minmax[1] = mx;
     }
-    __syncthreads();
-    const uint64_t diff = s_min[0] ^ s_max[0];
+    cl.sync();  // every CTA's min/max published
+    uint64_t mn = ~0ull, mx = 0ull;
+    for (int r = 0; r < kSelCluster; ++r) {
+      const uint64_t* mm = cl.map_shared_rank(c_minmax, r);
+      mn = mm[0] < mn ? mm[0] : mn;
+      mx = mm[1] > mx ? mm[1] : mx;
+    }
+    const uint64_t diff = mn ^ mx;
     int rem = diff ? 64 - __clzll(static_cast<long long>(diff)) : 0;  // bits still undecided
-    prefix = s_min[0] & (rem == 64 ? 0ull : ~((1ull << rem) - 1ull));
-    __syncthreads();
-    int64_t ncand = -1;  // >= 0 once the candidates sit in cand[]
+    prefix = mn & (rem == 64 ? 0ull : ~((1ull << rem) - 1ull));
+    int64_t ncand = -1;  // >= 0 once this CTA's candidates sit in cand[]
     while (rem > 0) {
       const int width = rem < kDigitBits ? rem : kDigitBits;
       const int shift = rem - width;
@@ -213,27 +242,30 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
           if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
         }
       } else {
-        // warp-uniform loop bound (lanes past the end are masked by `in`)
-        for (int64_t w0 = lo + (tid & ~31); w0 < hi; w0 += kUnroll * blockDim.x) {
-          const int64_t t0 = w0 + lane;
+        for (int64_t t0 = A0 + tid; t0 < A1; t0 += kUnroll * blockDim.x) {
           double v[kUnroll];
 #pragma unroll
           for (int j = 0; j < kUnroll; ++j) {
             const int64_t t = t0 + j * blockDim.x;
-            v[j] = t < hi ? __ldg(s + t) : 0.0;
+            v[j] = t < A1 ? __ldg(s + t) : 0.0;
           }
 #pragma unroll
           for (int j = 0; j < kUnroll; ++j) {
             const uint64_t key = score_key(v[j]);
-            const bool in = t0 + j * blockDim.x < hi && (key & pmask) == prefix;
+            const bool in = t0 + j * blockDim.x < A1 && (key & pmask) == prefix;
             if (in) atomicAdd(&hist[(key >> shift) & ((1u << width) - 1u)], 1u);
           }
         }
       }
-      __syncthreads();
-      // descending bins: thread t owns bins 2047-2t and 2046-2t
+      cl.sync();  // every CTA's histogram complete
+      // descending bins: thread t owns bins 2047-2t and 2046-2t, summed over the cluster
       const int b0 = kBins - 1 - 2 * tid, b1 = b0 - 1;
-      const unsigned int c0 = hist[b0], c1 = hist[b1];
+      unsigned int c0 = 0, c1 = 0;
+      for (int r = 0; r < kSelCluster; ++r) {
+        const unsigned int* hr = cl.map_shared_rank(hist, r);
+        c0 += hr[b0];
+        c1 += hr[b1];
+      }
       const unsigned int own = c0 + c1;
       unsigned int inc = own;
 #pragma unroll
@@ -266,38 +298,37 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
       k = s_k;
       n_eq = s_eq;
       rem = shift;
-      __syncthreads();
+      cl.sync();  // every CTA has read the cluster's histograms: they may be cleared
       if (ncand < 0 && rem > 0 && n_eq <= kCandCap) {
-        // few keys share the prefix now: copy them to shared memory once, so
-        // the remaining passes read cand[] instead of every score
+        // few keys share the prefix now: copy this CTA's ones to shared memory
+        // once, so the remaining passes read cand[] instead of every score
         if (tid == 0) s_ncand = 0;
         __syncthreads();
         const uint64_t pm = ~((1ull << rem) - 1ull);
-        for (int64_t w0 = lo + (tid & ~31); w0 < hi; w0 += kUnroll * blockDim.x) {
-          const int64_t t0 = w0 + lane;
+        for (int64_t t0 = A0 + tid; t0 < A1; t0 += kUnroll * blockDim.x) {
           double v[kUnroll];
 #pragma unroll
           for (int j = 0; j < kUnroll; ++j) {
             const int64_t t = t0 + j * blockDim.x;
-            v[j] = t < hi ? __ldg(s + t) : 0.0;
+            v[j] = t < A1 ? __ldg(s + t) : 0.0;
           }
 #pragma unroll
           for (int j = 0; j < kUnroll; ++j) {
             const uint64_t key = score_key(v[j]);
-            if (t0 + j * blockDim.x < hi && (key & pm) == prefix) cand[atomicAdd(&s_ncand, 1u)] = key;
+            if (t0 + j * blockDim.x < A1 && (key & pm) == prefix) cand[atomicAdd(&s_ncand, 1u)] = key;
           }
         }
         __syncthreads();
-        ncand = n_eq;  // exactly the keys counted in the chosen bin
+        ncand = s_ncand;
       }
     }
   }
   const uint64_t kstar = prefix;  // threshold key
   const int64_t need_eq = k;      // how many keys equal to kstar are taken, lowest positions first
 
-  // --- ordered compaction: each warp owns a contiguous segment of positions
-  const int64_t seg = ((T + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
-  const int64_t s0 = warp * seg, s1 = min64(T, s0 + seg);
+  // --- ordered compaction: each warp owns a contiguous part of the CTA's segment
+  const int64_t seg = ((S1 - S0 + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
+  const int64_t s0 = min64(S1, S0 + warp * seg), s1 = min64(S1, s0 + seg);
 
   // pass A (only when ties at the threshold must be split by position):
   // keys equal to the threshold, per warp
@@ -321,8 +352,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   }
   if (lane == 0) warp_cnt[warp] = eq;
   __syncthreads();
+  if (tid == 0) {
+    long long tot = 0;
+    for (int w = 0; w < kSelWarps; ++w) tot += warp_cnt[w];
+    c_count[0] = tot;
+  }
   block_exclusive_scan32(warp_cnt);
-  int64_t eq_rank = warp_cnt[warp];
+  cl.sync();  // every CTA's tie count published
+  long long eq_base = 0;
+  for (int r = 0; r < rank; ++r) eq_base += cl.map_shared_rank(c_count, r)[0];
+  int64_t eq_rank = eq_base + warp_cnt[warp];
   __syncthreads();
 
   // pass B: keep flags (bitmask in smem) and per-warp kept counts
@@ -349,22 +388,31 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
                                                            (is_eq && (!rank_ties || r < need_eq)))));
       const uint32_t kb = __ballot_sync(0xffffffffu, keep);
       eq_rank += __popc(eqb);
-      if (lane == 0) flagbits[b >> 5] = kb;
+      if (lane == 0) flagbits[(b - S0) >> 5] = kb;
       cnt += __popc(kb);
     }
   }
   if (lane == 0) warp_cnt[warp] = cnt;
   __syncthreads();
+  if (tid == 0) {
+    long long tot = 0;
+    for (int w = 0; w < kSelWarps; ++w) tot += warp_cnt[w];
+    c_count[1] = tot;
+  }
   block_exclusive_scan32(warp_cnt);
+  cl.sync();  // every CTA's kept count published
+  long long out_base = 0;
+  for (int r = 0; r < rank; ++r) out_base += cl.map_shared_rank(c_count, r)[1];
 
   // pass C: write kept positions in ascending order
-  int64_t o = warp_cnt[warp];
+  int64_t o = out_base + warp_cnt[warp];
   for (int64_t b = s0; b < s1; b += 32) {
-    const uint32_t kb = flagbits[b >> 5];
+    const uint32_t kb = flagbits[(b - S0) >> 5];
     const int64_t idx = o + __popc(kb & ((1u << lane) - 1u));
     if (((kb >> lane) & 1u) && idx < n_kept) out[idx] = static_cast<int32_t>(b + lane);
     o += __popc(kb);
   }
+  cl.sync();  // no CTA leaves while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------- launch
@@ -432,13 +480,28 @@ cudaError_t launch_select(const double* scores, int units, int64_t T, int W, int
                           int64_t n_kept, int32_t* kept, int64_t kept_stride,
                           cudaStream_t stream) {
   (void)evict_pct;
-  // flag words rounded up to an even count (8-byte alignment of the keys), then the keys
-  const size_t smem = static_cast<size_t>((T + 63) / 64) * 2 * sizeof(uint32_t) +
+  // this CTA's flag words rounded up to an even count (8-byte alignment of the
+  // keys), then the keys
+  const int64_t seg_cta = ((T + kSelCluster - 1) / kSelCluster + 31) / 32 * 32;
+  const size_t smem = static_cast<size_t>((seg_cta + 63) / 64) * 2 * sizeof(uint32_t) +
                       static_cast<size_t>(kCandCap) * sizeof(uint64_t);
   cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  select_kernel<<<units, kSelThreads, smem, stream>>>(scores, T, W, n_kept, kept, kept_stride);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units) * kSelCluster);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSelCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, select_kernel, scores, T, W, n_kept, kept, kept_stride);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
