@@ -165,25 +165,6 @@ __device__ __forceinline__ void issue_raw(const CodecArgs& a, int32_t src_lane, 
   }
 }
 
-// Decode's variant: 1024 16-byte chunks spread over all threads (thread c
-// copies chunk c % 32 of row (c / 32) % 2 of slot c / 64, stepping by the
-// CTA size); every warp runs the same number of iterations.
-__device__ __forceinline__ void issue_raw_spread(const CodecArgs& a, int32_t src_lane, uint32_t raw,
-                                                 int tid, int nthreads) {
-  for (int c = tid; c < kSlots * 64; c += nthreads) {
-    const int slot = c >> 6;
-    const int32_t src = __shfl_sync(0xffffffffu, src_lane, slot);
-    if (src < 0) continue;
-    const int64_t pos = a.pos_base + src;
-    int64_t hi = pos >> 8;
-    hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
-    const int which = (c >> 5) & 1, part = c & 31;
-    const float2* row = which ? a.tab + (a.n_a + (pos & 255)) * kHalf : a.tab + hi * kHalf;
-    cp_async16(raw + slot * kRawSlot + which * 512 + part * 16,
-               reinterpret_cast<const char*>(row) + part * 16);
-  }
-}
-
 // cs table of one tile: float4 cs[j][slot] = (c_2j, s_2j, c_2j+1, s_2j+1),
 // c = fmaf(cA, cB, -(sA sB)), s = fmaf(sA, cB, cA sB); a thread of half h
 // later reads j in [16h, 16h+16).
@@ -706,9 +687,9 @@ __global__ void __launch_bounds__(256, 2)
   // prologue: rows of tiles 0 and 1 in flight, table of tile 0 combined
   int32_t src_pref = -1;
   if (ROPE) {
-    if (my_tiles > 0) issue_raw_spread(a, slot_src(a, tile(0), slot_l), raw_of(0), tid, nthreads);
+    if (my_tiles > 0) issue_raw(a, slot_src(a, tile(0), slot_l), raw_of(0), warp, nwarps, lane);
     cp_async_commit();
-    if (my_tiles > 1) issue_raw_spread(a, slot_src(a, tile(1), slot_l), raw_of(1), tid, nthreads);
+    if (my_tiles > 1) issue_raw(a, slot_src(a, tile(1), slot_l), raw_of(1), warp, nwarps, lane);
     cp_async_commit();
     if (my_tiles > 2) src_pref = slot_src(a, tile(2), slot_l);
     cp_async_wait<1>();
@@ -722,7 +703,7 @@ __global__ void __launch_bounds__(256, 2)
       // rows of tile k+1 landed (everyone's), table k combined, tile k-1 decoded
       cp_async_wait<0>();
       __syncthreads();
-      if (k + 2 < my_tiles) issue_raw_spread(a, src_pref, raw_of(k), tid, nthreads);
+      if (k + 2 < my_tiles) issue_raw(a, src_pref, raw_of(k), warp, nwarps, lane);
       cp_async_commit();
       if (k + 3 < my_tiles) src_pref = slot_src(a, tile(k + 3), slot_l);
       if (k + 1 < my_tiles) combine_raw(raw_of(k + 1), cs_of(k + 1), tid, nthreads);
