@@ -17,16 +17,22 @@
 // two lanes of an fp32x2 register hold groups g and g+8, so the E8 search
 // runs two groups per packed instruction (__fadd2_rn / __ffma2_rn /
 // __fmul2_rn: per-lane IEEE round-to-nearest, the same bits as scalar code).
-// A persistent CTA of HG warps (HG heads) walks tiles of 16 slots x HG heads.
+// A persistent CTA of HG warps (HG heads) walks tiles of 16 slots x HG heads
+// (encode: 16 (unit, slot) pairs of the flat pair list, so a tile may span
+// units; decode: 16 slots of one unit).  The E8 decision is taken from the
+// integer coset's rounding alone when the two coset distances are clearly
+// apart, with the full two-coset decision as the exact fallback (e8_choose).
 // Encode stages the input rows with warp-cooperative 16-byte async copies
 // (each warp instruction moves two whole 256-byte rows, gathered through the
 // kept list) into padded shared-memory rows, double buffered, so the loads of
 // tile k+2 overlap the arithmetic of tile k; the RoPE (cos, sin) pairs of a
-// tile are combined once per CTA and shared by its heads.  Decode loads the
-// next tile's codes one tile ahead and writes each warp's 16 reconstructed
-// rows into a 128-byte-swizzled shared tile that one lane stores with two
-// TMA tensor stores (cp.async.bulk.tensor, 4-D map of the output).  Every
-// (bits, RoPE) variant is its own kernel: keys and values are two launches.
+// tile are combined once per CTA from table rows staged a tile ahead and
+// shared by its heads.  Decode loads the next tile's codes one tile ahead,
+// double-buffers the table rows (one CTA barrier per tile) and writes each
+// warp's 16 reconstructed rows into a 128-byte-swizzled shared tile that one
+// lane stores with two TMA tensor stores (cp.async.bulk.tensor, 4-D map of the
+// output).  Every (bits, RoPE) variant is its own kernel: keys and values are
+// two launches.
 #include <cuda.h>
 
 #include <mutex>
