@@ -188,6 +188,8 @@ nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_stride
     return fail(NQ_ERR_INVALID, "need units >= 0, 1 <= heads <= 1024, n >= 0, slot0 >= 0, pos_base >= 0");
   if (units == 0 || n == 0) return NQ_OK;
   if (T_in < 1) return fail(NQ_ERR_INVALID, "T_in must be >= 1");
+  if (static_cast<int64_t>(units) * n >= (int64_t(1) << 31))
+    return fail(NQ_ERR_UNSUPPORTED, "units * n must stay below 2^31 (slot pairs of one call)");
   if (kept) {
     if (!aligned(kept, 4)) return fail(NQ_ERR_INVALID, "kept misaligned");
     if (kept_stride < n) return fail(NQ_ERR_INVALID, "kept_stride < n");

@@ -188,7 +188,8 @@ nq_status nq_select(const double *scores, int units, int64_t T, int W, int evict
  *   written to slot slot0 + i of k_out / v_out.
  * K and/or V may be NULL (then its k_out/v_out is ignored).  bits: K and V
  * may differ (K3V2).  rope_tab: device tables from nq_rope_tables_fill_host
- * (required when K != NULL), positions must be < rope_max_pos. */
+ * (required when K != NULL), positions must be < rope_max_pos.
+ * units * n must stay below 2^31 (NQ_ERR_UNSUPPORTED otherwise). */
 nq_status nq_encode(const void *K, nq_kv_strides ks, const void *V, nq_kv_strides vs, int units,
                     int heads, int64_t T_in, int64_t n, const int32_t *kept, int64_t kept_stride,
                     int64_t pos_base, const float *rope_tab, int64_t rope_max_pos,

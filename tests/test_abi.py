@@ -111,6 +111,8 @@ def test_validation_rejects_bad_arguments(nq):
     assert L.nq_score(fake, ok, 1, 8, 64, 64, fake, fake, 16, None) == nq.NQ_ERR_WORKSPACE
     assert L.nq_score(fake, ok, 1, 129, 64, 64, fake, fake, 1 << 30, None) == nq.NQ_ERR_UNSUPPORTED
     assert L.nq_score_static(fake, ok, 1, 129, 64, 64, fake, None) == nq.NQ_ERR_UNSUPPORTED
+    assert L.nq_encode(fake, ok, None, ok, 1 << 20, 8, 1 << 12, 1 << 12, None, 0, 0, fake, 1 << 12,
+                       ctypes.byref(pk), None, 0, None) == nq.NQ_ERR_UNSUPPORTED
     assert L.nq_e8_quantise(fake, 4, 5, fake, fake, None) == nq.NQ_ERR_INVALID
     assert L.nq_e8_quantise(fake, -1, 3, fake, fake, None) == nq.NQ_ERR_INVALID
     # select: percentage range, stride, size limit
