@@ -16,8 +16,8 @@
  *     (dev.to, section "Como funciona (em 6 passos)", steps 1-5)
  *
  * The pages leave every formula open; the readings taken (fp32 operation
- * order, tie rules, scale rule, packed layout) are listed in the design doc and
- * restated next to each function below.
+ * order, tie rules, scale rule, packed layout) are stated next to each
+ * function below.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
  * (no SIMD intrinsics, no OpenMP).  -ffp-contract=off matters: every fused
