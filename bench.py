@@ -539,8 +539,10 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, world, K.device)
     return {"value": world * in_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
-            "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": Kd.numel() * 2 + Vd.numel() * 2,
-            "ms_per_step": ms, "steps": args.e2e_steps, "chunk_layers": args.e2e_chunk}
+            "h2d_bytes_per_step": rt.h2d_bytes(Kh, Vh),
+            "d2h_bytes_per_step": Kd.numel() * 2 + Vd.numel() * 2,
+            "ms_per_step": ms, "steps": args.e2e_steps, "chunk_layers": args.e2e_chunk,
+            "values_read_in_place": rt.values_in_place}
 
 
 def main():

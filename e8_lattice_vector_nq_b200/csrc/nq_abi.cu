@@ -59,6 +59,26 @@ nq_status check_rope(const float* tab, int64_t max_pos) {
 
 constexpr int64_t kMaxSelectT = int64_t(1) << 20;
 
+// The address at which the device reads p: p itself for device (or managed)
+// memory, the mapped address for pinned host memory; anything the device
+// cannot read (plain host memory) is refused before any launch.
+nq_status device_readable(const void* p, const void** out, const char* name) {
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of the query
+    return fail(NQ_ERR_INVALID, "%s: the device cannot read this pointer", name);
+  }
+  if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) {
+    *out = p;
+    return NQ_OK;
+  }
+  if (attr.type == cudaMemoryTypeHost && attr.devicePointer) {
+    *out = attr.devicePointer;
+    return NQ_OK;
+  }
+  return fail(NQ_ERR_INVALID, "%s is host memory the device cannot read (not pinned/mapped)", name);
+}
+
 }  // namespace
 
 extern "C" {
@@ -208,10 +228,18 @@ nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_stride
     if (nq_status st = check_kv(V, vs, "V")) return st;
     if (nq_status st = check_packed(v_out, "v_out")) return st;
   }
+  // K and V may live in pinned host memory: the kernels then read only the
+  // rows they encode across the bus
+  const void* Kd = nullptr;
+  const void* Vd = nullptr;
+  if (K)
+    if (nq_status st = device_readable(K, &Kd, "K")) return st;
+  if (V)
+    if (nq_status st = device_readable(V, &Vd, "V")) return st;
   nq::EncodeLaunch L{};
-  L.K = K;
+  L.K = Kd;
   L.ks = ks;
-  L.V = V;
+  L.V = Vd;
   L.vs = vs;
   L.units = units;
   L.heads = heads;

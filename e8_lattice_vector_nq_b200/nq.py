@@ -106,6 +106,14 @@ def _require_cuda(*ts):
             raise ValueError("libnq works on CUDA tensors only (no CPU path)")
 
 
+def _require_device_readable(*ts):
+    """CUDA tensors, or pinned host tensors: with unified addressing the
+    kernels read pinned host memory in place over the bus (no CPU arithmetic)."""
+    for t in ts:
+        if t is not None and not (t.is_cuda or t.is_pinned()):
+            raise ValueError("libnq reads CUDA tensors or pinned host tensors only (no CPU path)")
+
+
 def kv_strides(t: torch.Tensor) -> KVStrides:
     """Strides of a [units][heads][tokens][128] bf16 tensor (last dim contiguous)."""
     if t.dim() != 4 or t.shape[-1] != D or t.stride(-1) != 1 or t.dtype != torch.bfloat16:
@@ -211,8 +219,11 @@ def nq_encode(K: torch.Tensor | None, V: torch.Tensor | None, k_out: PackedStore
               v_out: PackedStore | None, n: int, rope_tab: torch.Tensor | None = None,
               rope_max_pos: int = 0, kept: torch.Tensor | None = None, pos_base: int = 0,
               slot0: int = 0, stream=None):
-    """Encode n slots of every (unit, head) into the packed stores (see nq.h, nq_encode)."""
-    _require_cuda(K, V, kept, rope_tab)
+    """Encode n slots of every (unit, head) into the packed stores (see nq.h, nq_encode).
+    K and V may also be pinned host tensors: the kernel then reads only the rows
+    it encodes (the kept ones) across the bus."""
+    _require_device_readable(K, V)
+    _require_cuda(kept, rope_tab)
     ref = K if K is not None else V
     units, heads, T_in, _ = ref.shape
     kd = k_out.desc() if K is not None else None
@@ -377,14 +388,25 @@ class HostRoundTrip:
     current stream, which afterwards waits for the last copy."""
 
     def __init__(self, codec: Codec, K: torch.Tensor, V: torch.Tensor, K_out: torch.Tensor,
-                 V_out: torch.Tensor, chunk_units: int = 4):
+                 V_out: torch.Tensor, chunk_units: int = 4, values_in_place: bool | None = None):
         self.codec, self.K, self.V, self.K_out, self.V_out = codec, K, V, K_out, V_out
+        # With eviction only the kept value rows are needed: the encode kernel
+        # reads them straight from the pinned host cache, so the rows it drops
+        # never cross the bus (keys are copied whole: every key is scored).
+        self.values_in_place = codec.evict if values_in_place is None else values_in_place
         self.chunks = [slice(u, min(u + chunk_units, codec.units))
                        for u in range(0, codec.units, chunk_units)]
         self.h2d, self.comp, self.d2h = (torch.cuda.Stream(K.device) for _ in range(3))
         ev = lambda: [torch.cuda.Event() for _ in self.chunks]  # noqa: E731
         self.in_ready, self.comp_done, self.out_done = ev(), ev(), ev()
         self.ran = False
+
+    def h2d_bytes(self, Kh: torch.Tensor, Vh: torch.Tensor) -> int:
+        """Bytes that cross the bus host-to-device per run."""
+        if not self.values_in_place:
+            return Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size()
+        c = self.codec
+        return Kh.numel() * Kh.element_size() + c.units * c.heads * c.n * 128 * Vh.element_size()
 
     def run(self, Kh: torch.Tensor, Vh: torch.Tensor, K_out_h: torch.Tensor,
             V_out_h: torch.Tensor):
@@ -398,12 +420,13 @@ class HostRoundTrip:
                 if self.ran:  # the previous run's kernels are done reading this chunk
                     self.h2d.wait_event(self.comp_done[c])
                 self.K[u].copy_(Kh[u], non_blocking=True)
-                self.V[u].copy_(Vh[u], non_blocking=True)
+                if not self.values_in_place:
+                    self.V[u].copy_(Vh[u], non_blocking=True)
                 self.in_ready[c].record(self.h2d)
             self.comp.wait_event(self.in_ready[c])
             if self.ran:  # the previous run's copy-out of this chunk is done
                 self.comp.wait_event(self.out_done[c])
-            self.codec.encode(self.K, self.V, self.comp, units=u)
+            self.codec.encode(self.K, Vh if self.values_in_place else self.V, self.comp, units=u)
             self.codec.decode(self.K_out, self.V_out, self.comp, units=u)
             self.comp_done[c].record(self.comp)
             with torch.cuda.stream(self.d2h):

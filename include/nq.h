@@ -16,7 +16,11 @@
  * --------------------------------
  * - Every tensor pointer is a DEVICE pointer that the caller allocates and
  *   owns; the library never allocates, frees or retains memory, except
- *   nq_rope_tables_fill_host, which writes a caller-owned HOST buffer.
+ *   nq_rope_tables_fill_host, which writes a caller-owned HOST buffer.  The
+ *   one exception: nq_encode's K and V inputs may also be pinned host memory
+ *   (cudaHostAlloc / cudaHostRegister), which the kernels read in place, so
+ *   only the rows encoded (the kept tokens) cross the bus; memory the device
+ *   cannot read is refused with NQ_ERR_INVALID before any launch.
  * - Every compute call is asynchronous on the caller's CUDA stream and
  *   returns as soon as its kernels are queued.  Nothing synchronises.
  * - Return value: nq_status.  NQ_ERR_INVALID for bad arguments (checked on the
