@@ -16,7 +16,6 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
 import json
 import os
 import statistics
@@ -63,10 +62,19 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+# The translation unit the encode kernel is compiled from (its source and every
+# header it includes, the public header among them).
+ENCODE_SOURCES = ("e8_lattice_vector_nq_b200/csrc/nq_codec.cu",
+                  "e8_lattice_vector_nq_b200/csrc/nq_codec_math.cuh",
+                  "e8_lattice_vector_nq_b200/csrc/nq_device.cuh",
+                  "e8_lattice_vector_nq_b200/csrc/nq_internal.h",
+                  "include/nq.h")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "e8_lattice_vector_nq_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for f in ENCODE_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]
 
