@@ -334,9 +334,9 @@ nq_status nq_attend(const float* q, int units, int heads, int G, const nq_packed
   const size_t need = nq_attend_workspace_bytes(units, heads, G, n);
   if (ws_bytes < need)
     return fail(NQ_ERR_WORKSPACE, "attend workspace too small: %zu < %zu", ws_bytes, need);
-  if (static_cast<int64_t>(units) * heads * ((n + 255) / 256) > 0x7FFFFFFF ||
+  if (n > 0x7FFFFFFF || nq::attend_ctas(units, heads, n) > 0x7FFFFFFF ||
       static_cast<int64_t>(units) * heads * G > 0x7FFFFFFF)
-    return fail(NQ_ERR_UNSUPPORTED, "units * heads * chunks too large for one launch");
+    return fail(NQ_ERR_UNSUPPORTED, "n or units * heads * chunks too large for one launch");
   nq::AttendLaunch L{};
   L.q = q;
   L.units = units;

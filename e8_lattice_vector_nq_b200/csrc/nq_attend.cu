@@ -9,18 +9,24 @@
 // decode kernel rounds to bf16 (keys re-rotated at their positions).
 //
 // Design (B200).  Split-K over the tokens (flash decoding): a CTA takes one
-// (unit, KV head, chunk of kChunk tokens) and all G query heads of the group.
-//   pass 1: two threads per token rebuild the key half by half (the decode
-//           kernel's arithmetic: unpack, Hadamard, kappa, RoPE with the
-//           two-level table rows read through L1) and dot it with the G
-//           queries held in shared memory as (q_i, q_{i+64}) pairs;
-//   softmax: one warp per query head: chunk max m, l = sum exp(s - m), and
-//           the weights w_t = exp(s_t - m) * kappa_t in place;
-//   pass 2: values stay in the code domain: since v_t = kappa_t * H t_t (H the
-//           unnormalised Hadamard matrix, t_t the 2q integers), the chunk
-//           accumulates a = sum_t w_t t_t per coordinate (thread = coordinate,
-//           two token streams), and H is applied once per query head when the
-//           chunks are combined (o = H A / L).
+// (unit, group of up to 8 KV heads, chunk of tokens), one warp per KV head
+// with all G query heads of that KV head, and walks the chunk in tiles of 16
+// tokens.  All heads of a unit share the tokens' positions, so:
+//   - the RoPE table rows of a tile are staged two tiles ahead (cp.async) and
+//     combined once into a cos/sin table that every warp of the CTA reads;
+//   - keys: two lanes per token rebuild the key half by half exactly as the
+//     decode kernel does (unpack, Hadamard, kappa, RoPE from the shared
+//     table) and dot it with the warp's queries, held in shared memory as
+//     (q_i, q_{i+64}) pairs;
+//   - online softmax per query head: running max m and sum l, the sums
+//     rescaled by exp(m_old - m_new) when the max grows; token weights
+//     w_t = exp(s_t - m) * kappa_t;
+//   - values stay in the code domain: since v_t = kappa_t * H t_t (H the
+//     unnormalised Hadamard matrix, t_t the 2q integers), the warp
+//     accumulates a = sum_t w_t t_t, lane l owning coordinates 4l..4l+3 (half
+//     a coset group), from value codes staged one tile ahead; H is applied
+//     once per query head when the chunks are merged (o = H A / L).
+// One CTA barrier per tile (the shared table); everything else is per warp.
 // The combine kernel merges the chunks' (m, l, a) with the usual rescaling,
 // applies the 128-point Hadamard transform across one warp and writes o, lse.
 #include "nq_codec_math.cuh"
@@ -28,248 +34,296 @@
 
 namespace nq {
 
-constexpr int kChunk = 512;         // tokens per CTA
-constexpr int kAttThreads = 256;
-constexpr int kMaxGroup = 8;        // query heads per KV head
 constexpr int kPartFloats = 2 + kD;  // m, l, a[128]
+constexpr int kMinChunk = 64;        // tokens per CTA at least
+// Splits are chosen so that a launch has about this many CTAs: four waves of
+// two 256-thread CTAs per SM on 148 SMs.
+constexpr int64_t kTargetCtas = 8 * 148;
 
 struct AttendArgs {
   const float* q;  // [units][heads * G][128]
   const uint32_t *kc, *km, *vc, *vm;
   int64_t kpu, kph, vpu, vph;  // vector strides of the packed stores
-  int heads, G, GT;  // GT: query heads computed per CTA (G rounded up to 1, 2, 4 or 8)
+  int heads, hg, ngroups;      // KV heads, KV heads per CTA, CTAs per (unit, split)
+  int G, GT;  // GT: query heads computed per warp (G rounded up to 1, 2, 4 or 8)
   int64_t n, slot0;
   const int32_t* pos;
   int64_t pos_stride, pos_base;
   const float2* tab;
   int64_t n_a;
   float scale;
-  int64_t nsplit;
-  float* part;  // [units][heads][nsplit][G][kPartFloats]
+  int64_t chunk, nsplit;  // tokens per CTA (a multiple of 16), chunks per (unit, head)
+  float* part;            // [units][heads][nsplit][GT][kPartFloats]
 };
 
-constexpr int kStreams = 8;  // token streams of pass 2 (one per warp)
-
-// Dynamic shared memory of the partial kernel for GT query heads per CTA.
+// Dynamic shared memory of the partial kernel: per CTA the raw RoPE rows and
+// the cos/sin tables of two tiles; per warp its queries, the key and value
+// codes of two tiles, and the current tile's weights and value meta.  Key
+// codes sit at a stride of 48 bytes per token (3 bits: exactly the codes;
+// 2 bits: padded), so the 16-byte reads of 8 consecutive tokens hit
+// distinct bank groups.
+constexpr int kKStride = 48;
 template <int BV, int GT>
 struct AttSmem {
-  static constexpr int kQ = GT * 64 * 8;          // float2 qp[GT][64]
-  static constexpr int kSc = kChunk * GT * 4;     // float sc[kChunk][GT]
-  static constexpr int kVw = kChunk * 4 * BV * 4;  // uint32 vw[kChunk][4 BV]
-  static constexpr int kMeta = kChunk * 4;        // uint32 vmeta[kChunk]
-  static constexpr int kAcc = kStreams * GT * kD * 4;  // float acc[kStreams][GT][128]
-  static constexpr int kRed = GT * 2 * 4;         // float red[GT][2]
-  static constexpr int bytes = kQ + kSc + kVw + kMeta + kAcc + kRed;
+  static constexpr int kRaw = 2 * kRawBytes;
+  static constexpr int kCs = 2 * kCsBytes;
+  static constexpr int kQ = GT * 64 * 8;               // float2 qp[GT][64]
+  static constexpr int kKc = 2 * kSlots * kKStride;    // key codes [2][16][48 bytes]
+  static constexpr int kVc = 2 * kSlots * 4 * BV * 4;  // uint32 codes[2][16][4 BV]
+  static constexpr int kW = kSlots * GT * 4;           // float w[16][GT]
+  static constexpr int kVm = kSlots * 4;               // uint32 vmeta[16]
+  static constexpr int kWarp = kQ + kKc + kVc + kW + kVm;
+  static constexpr int bytes(int warps) { return kRaw + kCs + warps * kWarp; }
 };
 
 template <int BK, int BV, int GT>
-__global__ void __launch_bounds__(kAttThreads, 2) attend_partial_kernel(const AttendArgs a) {
+__global__ void __launch_bounds__(256, 2) attend_partial_kernel(const AttendArgs a) {
   extern __shared__ __align__(16) unsigned char att_smem[];
   using S = AttSmem<BV, GT>;
-  float2(*qp)[64] = reinterpret_cast<float2(*)[64]>(att_smem);                     // (q_i, q_{i+64})
-  float* sc = reinterpret_cast<float*>(att_smem + S::kQ);                          // [kChunk][GT]
-  uint32_t* vw = reinterpret_cast<uint32_t*>(att_smem + S::kQ + S::kSc);           // value codes
-  uint32_t* vmeta = reinterpret_cast<uint32_t*>(att_smem + S::kQ + S::kSc + S::kVw);
-  float* accs = reinterpret_cast<float*>(att_smem + S::kQ + S::kSc + S::kVw + S::kMeta);
-  float* red = accs + kStreams * GT * kD;                                          // [GT][2]
-
+  constexpr int GP = (GT + 1) / 2;  // query heads in fp32x2 pairs (GT = 1: one lane unused)
+  constexpr int kVWords = 4 * BV;   // value code words per token
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int slot_l = lane & 15, half = lane >> 4;
+
   const int64_t split = blockIdx.x % a.nsplit;
-  const int64_t uh = blockIdx.x / a.nsplit;
-  const int h = static_cast<int>(uh % a.heads);
-  const int64_t u = uh / a.heads;
-  const int G = a.G;  // G <= GT; heads G..GT-1 of the CTA are zero queries
-  const int64_t t0 = split * kChunk;
-  const int nt = static_cast<int>(min64(kChunk, a.n - t0));
+  const int64_t ug = blockIdx.x / a.nsplit;
+  const int h = static_cast<int>(ug % a.ngroups) * a.hg + warp;
+  const int64_t u = ug / a.ngroups;
+  const int64_t t0 = split * a.chunk;
+  const int nt = static_cast<int>(min64(a.chunk, a.n - t0));  // >= 1
+  const int ntiles = (nt + kSlots - 1) / kSlots;
 
-  // queries of the group, and the chunk's value codes (cp.async) and meta
-  const float* qg = a.q + (u * a.heads * G + static_cast<int64_t>(h) * G) * kD;
-  for (int e = tid; e < GT * 64; e += kAttThreads) {
+  const uint32_t raw0 = smem_u32(att_smem);
+  unsigned char* cs0 = att_smem + S::kRaw;
+  unsigned char* wsm = att_smem + S::kRaw + S::kCs + warp * S::kWarp;
+  float2(*qp)[64] = reinterpret_cast<float2(*)[64]>(wsm);
+  const uint32_t kcb = smem_u32(wsm + S::kQ);
+  uint32_t* vcb = reinterpret_cast<uint32_t*>(wsm + S::kQ + S::kKc);
+  float* wts = reinterpret_cast<float*>(wsm + S::kQ + S::kKc + S::kVc);
+  uint32_t* vmb = reinterpret_cast<uint32_t*>(wsm + S::kQ + S::kKc + S::kVc + S::kW);
+  auto raw_of = [&](int k) { return raw0 + static_cast<uint32_t>(k & 1) * kRawBytes; };
+  auto cs_of = [&](int k) { return reinterpret_cast<float4*>(cs0 + (k & 1) * kCsBytes); };
+
+  // position minus pos_base of this lane's token in tile k, -1 past the chunk
+  // (out-of-contract negative positions are taken as 0)
+  auto src_of = [&](int k) -> int32_t {
+    const int tt = k * kSlots + slot_l;
+    if (tt >= nt) return -1;
+    const int32_t p =
+        a.pos ? __ldg(a.pos + u * a.pos_stride + t0 + tt) : static_cast<int32_t>(t0 + tt);
+    return p < 0 ? 0 : p;
+  };
+  const int64_t kv0 = u * a.kpu + h * a.kph + a.slot0 + t0;  // first key vector of the chunk
+  const int64_t vv0 = u * a.vpu + h * a.vph + a.slot0 + t0;  // first value vector
+  // key and value codes of tile k (its valid tokens) into the warp's buffers k & 1
+  auto issue_codes = [&](int k) {
+    const int nv = min(kSlots, nt - k * kSlots);
+    const char* ks = reinterpret_cast<const char*>(a.kc + (kv0 + k * kSlots) * (4 * BK));
+    const uint32_t kd = kcb + (k & 1) * (kSlots * kKStride);
+    for (int c = lane; c < nv * BK; c += 32) {
+      const int tok = c / BK;
+      cp_async16(kd + tok * kKStride + (c - tok * BK) * 16, ks + c * 16);
+    }
+    const char* vs = reinterpret_cast<const char*>(a.vc + (vv0 + k * kSlots) * kVWords);
+    const uint32_t vd = smem_u32(vcb + (k & 1) * (kSlots * kVWords));
+    for (int c = lane; c < nv * BV; c += 32) cp_async16(vd + c * 16, vs + c * 16);
+  };
+  // key and value meta of this lane's token in tile k (zero past the chunk)
+  uint32_t kmeta = 0, vmeta = 0;
+  auto load_meta = [&](int k) {
+    const int tt = k * kSlots + slot_l;
+    kmeta = tt < nt ? __ldg(a.km + kv0 + tt) : 0u;
+    vmeta = tt < nt ? __ldg(a.vm + vv0 + tt) : 0u;
+  };
+
+  // the warp's queries (heads G..GT-1 are zero)
+  const float* qg = a.q + (u * a.heads + h) * static_cast<int64_t>(a.G) * kD;
+  for (int e = lane; e < GT * 64; e += 32) {
     const int g = e >> 6, i = e & 63;
-    qp[g][i] = g < G ? make_float2(__ldg(qg + g * kD + i), __ldg(qg + g * kD + i + 64))
-                     : make_float2(0.f, 0.f);
+    qp[g][i] = g < a.G ? make_float2(__ldg(qg + g * kD + i), __ldg(qg + g * kD + i + 64))
+                       : make_float2(0.f, 0.f);
   }
-  const int64_t vbase = u * a.vpu + h * a.vph + a.slot0 + t0;
-  {
-    const char* src = reinterpret_cast<const char*>(a.vc + vbase * (4 * BV));
-    const uint32_t dst = smem_u32(vw);
-    for (int c = tid; c < nt * BV; c += kAttThreads) cp_async16(dst + c * 16, src + c * 16);
-    cp_async_commit();
-  }
-  for (int t = tid; t < nt; t += kAttThreads) vmeta[t] = __ldg(a.vm + vbase + t);
-  __syncthreads();  // qp ready
 
-  // ---- pass 1: keys and scores (16 tokens per warp per round); each round's
-  // codes, meta and position are loaded one round ahead
-  uint32_t wn_[4 * BK];
-  uint32_t meta_n = 0;
-  int64_t pos_n = 0;
-  auto load_round = [&](int r) {
-    const int tt = r * 128 + warp * 16 + slot_l;
+  // prologue: rows of tiles 0 and 1 and the value codes of tile 0 in flight,
+  // the table of tile 0 combined
+  int32_t src_pref = -1;
+  issue_rope_rows(a.tab, a.n_a, a.pos_base, src_of(0), raw_of(0), warp, nwarps, lane);
+  issue_codes(0);
+  cp_async_commit();
+  if (ntiles > 1)
+    issue_rope_rows(a.tab, a.n_a, a.pos_base, src_of(1), raw_of(1), warp, nwarps, lane);
+  cp_async_commit();
+  if (ntiles > 2) src_pref = src_of(2);
+  load_meta(0);
+  cp_async_wait<1>();
+  __syncthreads();
+  combine_rope_rows(raw_of(0), cs_of(0), tid, nthreads);
+
+  // running max and sum of query head g live in lane g
+  float m_lane = -INFINITY, l_lane = 0.f;
+  float2 acc[GP][4];
 #pragma unroll
-    for (int i = 0; i < 4 * BK; ++i) wn_[i] = 0;
-    meta_n = 0;
-    pos_n = 0;
-    if (tt < nt) {
-      const int64_t vec = u * a.kpu + h * a.kph + a.slot0 + t0 + tt;
-      const uint4* src = reinterpret_cast<const uint4*>(a.kc + vec * (4 * BK));
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[g][c] = make_float2(0.f, 0.f);
+
+  // Lane l's value coordinates 4l..4l+3: codes at bits BV*4l.. of the token's
+  // words, coset group l/2.  2q = 2 (2^22 + j) - 2^23 - (2^b - 2) - h, with
+  // 2^22 + j built by one LOP3 (the code at mantissa bit 1: the fp32 spacing
+  // at 2^22 is 1/2) and every constant an integer below 2^24: exact.
+  const int bitpos = BV * 4 * lane;
+  const int wi = bitpos >> 5, off = bitpos & 31;
+  const int wn = wi + 1 < kVWords ? wi + 1 : wi;
+  const int vgrp = lane >> 1;
+  constexpr float kBase = -8388608.0f - static_cast<float>((1 << BV) - 2);
+  constexpr uint32_t kMask2 = ((1u << BV) - 1u) << 1;
+
+  for (int k = 0; k < ntiles; ++k) {
+    // rows of tile k+1 and codes of tile k landed (everyone's), table k
+    // combined, tile k-1 done by every warp
+    cp_async_wait<0>();
+    __syncthreads();
+    if (k + 2 < ntiles)
+      issue_rope_rows(a.tab, a.n_a, a.pos_base, src_pref, raw_of(k), warp, nwarps, lane);
+    if (k + 1 < ntiles) issue_codes(k + 1);
+    cp_async_commit();
+    if (k + 3 < ntiles) src_pref = src_of(k + 3);
+    if (k + 1 < ntiles) combine_rope_rows(raw_of(k + 1), cs_of(k + 1), tid, nthreads);
+
+    const bool valid = k * kSlots + slot_l < nt;
+    const uint32_t kmc = kmeta, vmc = vmeta;
+    if (k + 1 < ntiles) load_meta(k + 1);
+
+    // ---- keys and scores (a token past the chunk has kappa 0 and score -inf)
+    float sc[GT];
+    {
+      uint32_t wc[4 * BK];
+      const uint32_t kt = kcb + (k & 1) * (kSlots * kKStride) + slot_l * kKStride;
 #pragma unroll
       for (int c = 0; c < BK; ++c) {
-        const uint4 x = __ldg(src + c);
-        wn_[4 * c] = x.x;
-        wn_[4 * c + 1] = x.y;
-        wn_[4 * c + 2] = x.z;
-        wn_[4 * c + 3] = x.w;
+        const uint4 x = lds128(kt + c * 16);
+        wc[4 * c] = x.x;
+        wc[4 * c + 1] = x.y;
+        wc[4 * c + 2] = x.z;
+        wc[4 * c + 3] = x.w;
       }
-      meta_n = __ldg(a.km + vec);
-      pos_n = a.pos_base + (a.pos ? static_cast<int64_t>(__ldg(a.pos + u * a.pos_stride + t0 + tt))
-                                  : t0 + tt);
-    }
-  };
-  load_round(0);
-  for (int r = 0; r < kChunk / 128; ++r) {
-    const int tt = r * 128 + warp * 16 + slot_l;
-    const bool valid = tt < nt;
-    uint32_t w[4 * BK];
+      float2 v[32];
+      reconstruct_half<BK>(wc, kmc, half, v);
+      rope_half(v, smem_u32(cs_of(k)) + (16 * half * kSlots + slot_l) * 16);
 #pragma unroll
-    for (int i = 0; i < 4 * BK; ++i) w[i] = wn_[i];
-    const uint32_t meta = meta_n;
-    const int64_t pos = pos_n;
-    if (r + 1 < kChunk / 128 && (r + 1) * 128 < nt) load_round(r + 1);
-    float2 v[32];
-    reconstruct_half<BK>(w, meta, half, v);
-    // RoPE: o_i = fmaf(x_i, c, -(x_{i+64} s)), o_{i+64} = fmaf(x_{i+64}, c, x_i s) with
-    // c = fmaf(cA, cB, -(sA sB)), s = fmaf(sA, cB, cA sB) from the table rows of
-    // p = 256 hi + lo (clamped into the table for out-of-contract positions)
-    int64_t hi = pos >> 8;
-    hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);
-    const float4* rowA = reinterpret_cast<const float4*>(a.tab + hi * kHalf + 32 * half);
-    const float4* rowB =
-        reinterpret_cast<const float4*>(a.tab + (a.n_a + (pos & 255)) * kHalf + 32 * half);
+      for (int g = 0; g < GT; ++g) {
+        float2 d0 = make_float2(0.f, 0.f), d1 = d0;
+        const float4* qh = reinterpret_cast<const float4*>(&qp[g][32 * half]);
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const float4 A = __ldg(rowA + jj), B = __ldg(rowB + jj);
-#pragma unroll
-      for (int ww = 0; ww < 2; ++ww) {
-        const float cA = ww ? A.z : A.x, sA = ww ? A.w : A.y;
-        const float cB = ww ? B.z : B.x, sB = ww ? B.w : B.y;
-        const float c = __fmaf_rn(cA, cB, -__fmul_rn(sA, sB));
-        const float s = __fmaf_rn(sA, cB, __fmul_rn(cA, sB));
-        const float2 P = v[2 * jj + ww];
-        const float2 Q = mul2(P, make_float2(s, s));
-        v[2 * jj + ww] = make_float2(__fmaf_rn(P.x, c, -Q.y), __fmaf_rn(P.y, c, Q.x));
+        for (int j = 0; j < 16; ++j) {
+          const float4 qq = qh[j];
+          d0 = fma2(v[2 * j], make_float2(qq.x, qq.y), d0);
+          d1 = fma2(v[2 * j + 1], make_float2(qq.z, qq.w), d1);
+        }
+        float d = (d0.x + d0.y) + (d1.x + d1.y);
+        d += __shfl_xor_sync(0xffffffffu, d, 16);
+        sc[g] = valid ? a.scale * d : -INFINITY;
       }
     }
+
+    // ---- online softmax over the tile (lanes l and l+16 hold the same token)
+    const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(vmc >> 16)));
+    const float kappa = __fmul_rn(__fmul_rn(sig, 0.5f), __uint_as_float(kCBits));
+    float wt[GT], al[GT];
 #pragma unroll
     for (int g = 0; g < GT; ++g) {
-      float2 d0 = make_float2(0.f, 0.f), d1 = d0;
-      const float4* qh = reinterpret_cast<const float4*>(&qp[g][32 * half]);
+      float mt = sc[g];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float4 qq = qh[j];
-        d0 = fma2(v[2 * j], make_float2(qq.x, qq.y), d0);
-        d1 = fma2(v[2 * j + 1], make_float2(qq.z, qq.w), d1);
+      for (int o = 8; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+      const float mo = __shfl_sync(0xffffffffu, m_lane, g);
+      const float mn = fmaxf(mo, mt);  // finite: every tile holds a valid token
+      al[g] = __expf(mo - mn);         // 0 on the first tile
+      const float p = valid ? __expf(sc[g] - mn) : 0.f;
+      float ps = p;
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+      const float lo = __shfl_sync(0xffffffffu, l_lane, g);
+      if (lane == g) {
+        m_lane = mn;
+        l_lane = __fmaf_rn(lo, al[g], ps);
       }
-      float d = (d0.x + d0.y) + (d1.x + d1.y);
-      d += __shfl_xor_sync(0xffffffffu, d, 16);
-      if (half == 0 && valid) sc[tt * GT + g] = a.scale * d;
+      wt[g] = valid ? p * kappa : 0.f;
     }
-  }
-  cp_async_wait<0>();
-  __syncthreads();
+    if (half == 0) {
+      float* wd = wts + slot_l * GT;
+      if (GT >= 4) {
+#pragma unroll
+        for (int g = 0; g < GT; g += 4)
+          *reinterpret_cast<float4*>(wd + g) = make_float4(wt[g], wt[g + 1], wt[g + 2], wt[g + 3]);
+      } else if (GT == 2) {
+        *reinterpret_cast<float2*>(wd) = make_float2(wt[0], wt[1]);
+      } else {
+        wd[0] = wt[0];
+      }
+      vmb[slot_l] = vmc;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float2 a2 = make_float2(al[2 * g], al[2 * g + 1 < GT ? 2 * g + 1 : 2 * g]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[g][c] = mul2(acc[g][c], a2);
+    }
 
-  // ---- softmax statistics per query head (warp g), weights in place
-  if (warp < GT) {
-    const int g = warp;
-    float m = -INFINITY;
-    for (int t = lane; t < nt; t += 32) m = fmaxf(m, sc[t * GT + g]);
+    // ---- values: a[g][4l + c] += w[t][g] * t_{t, 4l + c}; tokens past the
+    // chunk carry weight 0 (their staged codes are stale but decode to finite values)
+    const uint32_t* vcur = vcb + (k & 1) * (kSlots * kVWords);
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.f;
-    for (int t = lane; t < nt; t += 32) {
-      const float p = __expf(sc[t * GT + g] - m);
-      l += p;
-      const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(vmeta[t] >> 16)));
-      const float kappa = __fmul_rn(__fmul_rn(sig, 0.5f), __uint_as_float(kCBits));
-      sc[t * GT + g] = p * kappa;
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      red[2 * g] = m;
-      red[2 * g + 1] = l;
-    }
-  }
-  __syncthreads();
-
-  // ---- pass 2: a[g][i] = sum_t w[t][g] * t_{t,i}.  Thread (stream, quad) owns
-  // coordinates 4 quad .. 4 quad + 3 (one coset group) for tokens t = stream mod 8.
-  // Code k of the quad sits at bits BV*(4 quad + k) of the token's words;
-  // 2q = 2 (2^22 + j) - 2^23 - (2^b - 2) - h, with 2^22 + j built by one LOP3
-  // (the code at mantissa bit 1: the fp32 spacing at 2^22 is 1/2) and every
-  // constant an integer below 2^24: exact.
-  {
-    const int quad = lane, strm = warp;
-    const int bitpos = BV * 4 * quad;
-    const int wi = bitpos >> 5, off = bitpos & 31;
-    const int wn = wi + 1 < 4 * BV ? wi + 1 : wi;
-    const int grp = quad >> 1;
-    constexpr float kBase = -8388608.0f - static_cast<float>((1 << BV) - 2);
-    constexpr uint32_t kMask2 = ((1u << BV) - 1u) << 1;
-    // heads in pairs as fp32x2 lanes (GT = 1: one lane unused)
-    constexpr int GP = (GT + 1) / 2;
-    float2 acc[GP][4];
-#pragma unroll
-    for (int g = 0; g < GP; ++g)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(0.f, 0.f);
-    for (int t = strm; t < nt; t += kStreams) {
-      const uint32_t* ww = vw + t * (4 * BV);
+    for (int t = 0; t < kSlots; ++t) {
+      const uint32_t* ww = vcur + t * kVWords;
       const uint32_t x =
           (off + 4 * BV <= 32 ? (ww[wi] >> off) : __funnelshift_r(ww[wi], ww[wn], off)) << 1;
-      const float kg = ((vmeta[t] >> grp) & 1u) ? kBase - 1.0f : kBase;
-      float2 wt[GP];
+      const float kg = ((vmb[t] >> vgrp) & 1u) ? kBase - 1.0f : kBase;
+      float2 wp[GP];
       if (GT >= 4) {
 #pragma unroll
         for (int g = 0; g < GP; g += 2) {
-          const float4 w4 = *reinterpret_cast<const float4*>(sc + t * GT + 2 * g);
-          wt[g] = make_float2(w4.x, w4.y);
-          wt[g + 1 < GP ? g + 1 : g] = make_float2(w4.z, w4.w);
+          const float4 w4 = *reinterpret_cast<const float4*>(wts + t * GT + 2 * g);
+          wp[g] = make_float2(w4.x, w4.y);
+          wp[g + 1 < GP ? g + 1 : g] = make_float2(w4.z, w4.w);
         }
       } else if (GT == 2) {
-        wt[0] = *reinterpret_cast<const float2*>(sc + t * GT);
+        wp[0] = *reinterpret_cast<const float2*>(wts + t * GT);
       } else {
-        wt[0] = make_float2(sc[t * GT], 0.f);
+        wp[0] = make_float2(wts[t], 0.f);
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float J = __uint_as_float(((x >> (BV * k)) & kMask2) | 0x4A800000u);
-        const float tq = __fmaf_rn(J, 2.0f, kg);
+      for (int cp = 0; cp < 2; ++cp) {
+        const float J0 = __uint_as_float(((x >> (BV * 2 * cp)) & kMask2) | 0x4A800000u);
+        const float J1 = __uint_as_float(((x >> (BV * (2 * cp + 1))) & kMask2) | 0x4A800000u);
+        const float2 tq = fma2(make_float2(J0, J1), make_float2(2.0f, 2.0f), make_float2(kg, kg));
 #pragma unroll
-        for (int g = 0; g < GP; ++g) acc[g][k] = fma2(wt[g], make_float2(tq, tq), acc[g][k]);
+        for (int g = 0; g < GP; ++g) {
+          acc[g][2 * cp] = fma2(wp[g], make_float2(tq.x, tq.x), acc[g][2 * cp]);
+          acc[g][2 * cp + 1] = fma2(wp[g], make_float2(tq.y, tq.y), acc[g][2 * cp + 1]);
+        }
       }
     }
+  }
+
+  // the chunk's (m, l, a) for each query head of the warp
+  float* out = a.part + ((u * a.heads + h) * a.nsplit + split) * (GT * kPartFloats);
 #pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      *reinterpret_cast<float4*>(accs + (strm * GT + 2 * g) * kD + 4 * quad) =
-          make_float4(acc[g][0].x, acc[g][1].x, acc[g][2].x, acc[g][3].x);
-      if (2 * g + 1 < GT)
-        *reinterpret_cast<float4*>(accs + (strm * GT + 2 * g + 1) * kD + 4 * quad) =
-            make_float4(acc[g][0].y, acc[g][1].y, acc[g][2].y, acc[g][3].y);
+  for (int g = 0; g < GP; ++g) {
+    float* o0 = out + (2 * g) * kPartFloats + 2 + 4 * lane;
+    *reinterpret_cast<float2*>(o0) = make_float2(acc[g][0].x, acc[g][1].x);
+    *reinterpret_cast<float2*>(o0 + 2) = make_float2(acc[g][2].x, acc[g][3].x);
+    if (2 * g + 1 < GT) {
+      float* o1 = o0 + kPartFloats;
+      *reinterpret_cast<float2*>(o1) = make_float2(acc[g][0].y, acc[g][1].y);
+      *reinterpret_cast<float2*>(o1 + 2) = make_float2(acc[g][2].y, acc[g][3].y);
     }
   }
-  __syncthreads();
-  // sum the streams in a fixed order and write the chunk's (m, l, a)
-  float* out = a.part + (uh * a.nsplit + split) * GT * kPartFloats;
-  for (int e = tid; e < GT * kD; e += kAttThreads) {
-    const int g = e / kD, i = e % kD;
-    float sum = 0.f;
-#pragma unroll
-    for (int st = 0; st < kStreams; ++st) sum += accs[(st * GT + g) * kD + i];
-    out[g * kPartFloats + 2 + i] = sum;
+  if (lane < GT) {
+    out[lane * kPartFloats] = m_lane;
+    out[lane * kPartFloats + 1] = l_lane;
   }
-  if (tid < 2 * GT) out[(tid >> 1) * kPartFloats + (tid & 1)] = red[tid];
 }
 
 // One warp per (unit, query head): merge the chunks, o = H A / L, lse = M + log L.
@@ -323,18 +377,39 @@ __global__ void __launch_bounds__(32) attend_combine_kernel(const AttendArgs a, 
 
 static int group_tile(int G) { return G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8)); }
 
+// Tokens per CTA: about kTargetCtas CTAs per launch, a multiple of the tile,
+// at least kMinChunk.
+static int64_t attend_chunk(int units, int heads, int64_t n) {
+  int64_t per_split = static_cast<int64_t>(units) * (heads / pick_head_group(heads));
+  if (per_split < 1) per_split = 1;
+  const int64_t want = (kTargetCtas + per_split - 1) / per_split;
+  int64_t chunk = (n + want - 1) / want;
+  chunk = (chunk + kSlots - 1) / kSlots * kSlots;
+  return chunk < kMinChunk ? kMinChunk : chunk;
+}
+
+static int64_t attend_nsplit(int units, int heads, int64_t n) {
+  const int64_t c = attend_chunk(units, heads, n);
+  return (n + c - 1) / c;
+}
+
 size_t attend_workspace_floats(int units, int heads, int G, int64_t n) {
-  const int64_t nsplit = (n + kChunk - 1) / kChunk;
-  return static_cast<size_t>(units) * heads * nsplit * group_tile(G) * kPartFloats;
+  return static_cast<size_t>(units) * heads * attend_nsplit(units, heads, n) * group_tile(G) *
+         kPartFloats;
+}
+
+int64_t attend_ctas(int units, int heads, int64_t n) {
+  return static_cast<int64_t>(units) * (heads / pick_head_group(heads)) *
+         attend_nsplit(units, heads, n);
 }
 
 template <int BK, int BV, int GT>
 static cudaError_t launch_partial_gt(const AttendArgs& a, int64_t grid, cudaStream_t stream) {
-  constexpr int smem = AttSmem<BV, GT>::bytes;
+  const int smem = AttSmem<BV, GT>::bytes(a.hg);
   cudaError_t err = cudaFuncSetAttribute(attend_partial_kernel<BK, BV, GT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  attend_partial_kernel<BK, BV, GT><<<static_cast<unsigned>(grid), kAttThreads, smem, stream>>>(a);
+  attend_partial_kernel<BK, BV, GT><<<static_cast<unsigned>(grid), 32 * a.hg, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -360,6 +435,8 @@ cudaError_t launch_attend(const AttendLaunch& L, cudaStream_t stream) {
   a.vpu = L.v_in.unit_stride;
   a.vph = L.v_in.head_stride;
   a.heads = L.heads;
+  a.hg = pick_head_group(L.heads);
+  a.ngroups = L.heads / a.hg;
   a.G = L.G;
   a.GT = group_tile(L.G);
   a.n = L.n;
@@ -370,9 +447,11 @@ cudaError_t launch_attend(const AttendLaunch& L, cudaStream_t stream) {
   a.tab = reinterpret_cast<const float2*>(L.rope_tab);
   a.n_a = (L.rope_max_pos + 255) / 256;
   a.scale = L.scale;
-  a.nsplit = (L.n + kChunk - 1) / kChunk;
+  a.chunk = attend_chunk(L.units, L.heads, L.n);
+  a.nsplit = (L.n + a.chunk - 1) / a.chunk;
   a.part = static_cast<float*>(L.ws);
-  const int64_t grid = static_cast<int64_t>(L.units) * L.heads * a.nsplit;
+  const int64_t grid = static_cast<int64_t>(L.units) * a.ngroups * a.nsplit;
+  if (grid >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
   const int bk = L.k_in.bits, bv = L.v_in.bits;
   cudaError_t err;
   if (bk == 3 && bv == 2) err = launch_partial<3, 2>(a, grid, stream);

@@ -42,9 +42,6 @@
 
 namespace nq {
 
-constexpr int kSlots = 16;                  // slots per tile: one warp = 16 slots x 2 halves
-constexpr int kCsBytes = 32 * kSlots * 16;  // float4 cs[32][16]
-
 // Division by a fixed divisor for numerators below 2^31 (round-up method of
 // Granlund and Montgomery): q = (n * m) >> (31 + l), l = ceil(log2 d),
 // m = floor(2^(31+l) / d) + 1.
@@ -146,46 +143,6 @@ __device__ __forceinline__ EncPair enc_pair(const CodecArgs& a, int64_t p0, int 
 __device__ __forceinline__ int32_t enc_src(const CodecArgs& a, const EncPair& e) {
   if (!e.valid) return -1;
   return a.idx ? __ldg(a.idx + e.unit * a.idx_stride + e.slot) : static_cast<int32_t>(e.slot);
-}
-
-// RoPE table rows of a tile, staged raw: for each of the 16 slots the A row
-// (angle 256a) and the B row (angle b) of its position p = 256a + b, 512
-// bytes each, at a padded stride of kRawSlot bytes per slot.  Warp w copies
-// the rows of slots w, w + nwarps, ...: one 16-byte chunk per lane per row.
-constexpr int kRawSlot = 1024 + 16;
-constexpr int kRawBytes = kSlots * kRawSlot;
-
-__device__ __forceinline__ void issue_raw(const CodecArgs& a, int32_t src_lane, uint32_t raw,
-                                          int warp, int nwarps, int lane) {
-  for (int slot = warp; slot < kSlots; slot += nwarps) {  // warp-uniform
-    const int32_t src = __shfl_sync(0xffffffffu, src_lane, slot);
-    if (src < 0) continue;
-    const int64_t pos = a.pos_base + src;
-    int64_t hi = pos >> 8;
-    hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
-    const char* rowA = reinterpret_cast<const char*>(a.tab + hi * kHalf);
-    const char* rowB = reinterpret_cast<const char*>(a.tab + (a.n_a + (pos & 255)) * kHalf);
-    const uint32_t dst = raw + slot * kRawSlot + lane * 16;
-    cp_async16(dst, rowA + lane * 16);
-    cp_async16(dst + 512, rowB + lane * 16);
-  }
-}
-
-// cs table of one tile: float4 cs[j][slot] = (c_2j, s_2j, c_2j+1, s_2j+1),
-// c = fmaf(cA, cB, -(sA sB)), s = fmaf(sA, cB, cA sB); a thread of half h
-// later reads j in [16h, 16h+16).
-__device__ __forceinline__ void combine_raw(uint32_t raw, float4* cs, int tid, int nthreads) {
-  for (int e = tid; e < 32 * kSlots; e += nthreads) {
-    const int slot = e & 15, j = e >> 4;
-    const float4 A = lds128f(raw + slot * kRawSlot + j * 16);
-    const float4 B = lds128f(raw + slot * kRawSlot + 512 + j * 16);
-    float4 v;
-    v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
-    v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
-    v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
-    v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
-    cs[j * kSlots + slot] = v;
-  }
 }
 
 // ---------------------------------------------------------- E8 (fp32x2)
@@ -536,19 +493,19 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
     const EncTile t0 = tile(0);
     const EncPair p0 = enc_pair(a, t0.p0, slot_l);
     const int32_t s0 = enc_src(a, p0);
-    if (ROPE) issue_raw(a, s0, raw, warp, nthreads / 32, lane);
+    if (ROPE) issue_rope_rows(a.tab, a.n_a, a.pos_base, s0, raw, warp, nthreads / 32, lane);
     issue_rows(t0, p0, s0, 0);
   }
   cp_async_commit();
   cp_async_wait<0>();
   sync();
-  if (ROPE && my_tiles > 0) combine_raw(raw, reinterpret_cast<float4*>(smem + rows_bytes), tid, nthreads);
+  if (ROPE && my_tiles > 0) combine_rope_rows(raw, reinterpret_cast<float4*>(smem + rows_bytes), tid, nthreads);
   sync();
   if (my_tiles > 1) {
     const EncTile t1 = tile(1);
     const EncPair p1 = enc_pair(a, t1.p0, slot_l);
     const int32_t s1 = enc_src(a, p1);
-    if (ROPE) issue_raw(a, s1, raw, warp, nthreads / 32, lane);
+    if (ROPE) issue_rope_rows(a.tab, a.n_a, a.pos_base, s1, raw, warp, nthreads / 32, lane);
     cp_async_commit();
     issue_rows(t1, p1, s1, 1);
     cp_async_commit();
@@ -578,11 +535,11 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
     load_half<ROPE>(v, smem_u32(st + row_idx * kRowPad),
                     smem_u32(st + rows_bytes) + (16 * half * kSlots + slot_l) * 16, half);
     if (ROPE && k + 1 < my_tiles)  // RoPE table of tile k+1 into the other stage
-      combine_raw(raw, reinterpret_cast<float4*>(smem + (s ^ 1) * stage_bytes + rows_bytes), tid,
+      combine_rope_rows(raw, reinterpret_cast<float4*>(smem + (s ^ 1) * stage_bytes + rows_bytes), tid,
                   nthreads);
     sync();  // stage s and the raw rows are free
     if (k + 2 < my_tiles) {
-      if (ROPE) issue_raw(a, src_pref, raw, warp, nthreads / 32, lane);
+      if (ROPE) issue_rope_rows(a.tab, a.n_a, a.pos_base, src_pref, raw, warp, nthreads / 32, lane);
       cp_async_commit();
       issue_rows(tile(k + 2), pp_pref, src_pref, s);
       cp_async_commit();
@@ -606,20 +563,7 @@ __device__ __forceinline__ void decode_half(const uint32_t (&w)[4 * BITS], uint3
                                             uint32_t csa, uint32_t row, int rsw, int half) {
   float2 v[32];
   reconstruct_half<BITS>(w, meta, half, v);
-  if (ROPE) {
-    // o_i = fmaf(x_i, c, -(x_{i+64} s)),  o_{i+64} = fmaf(x_{i+64}, c, x_i s)
-#pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const float4 t = lds128f(csa + jj * (kSlots * 16));
-#pragma unroll
-      for (int ww = 0; ww < 2; ++ww) {
-        const float c = ww ? t.z : t.x, s = ww ? t.w : t.y;
-        const float2 P = v[2 * jj + ww];
-        const float2 Q = mul2(P, make_float2(s, s));
-        v[2 * jj + ww] = make_float2(__fmaf_rn(P.x, c, -Q.y), __fmaf_rn(P.y, c, Q.x));
-      }
-    }
-  }
+  if (ROPE) rope_half(v, csa);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint32_t A[4], B[4];
@@ -693,14 +637,14 @@ __global__ void __launch_bounds__(256, 2)
   // prologue: rows of tiles 0 and 1 in flight, table of tile 0 combined
   int32_t src_pref = -1;
   if (ROPE) {
-    if (my_tiles > 0) issue_raw(a, slot_src(a, tile(0), slot_l), raw_of(0), warp, nwarps, lane);
+    if (my_tiles > 0) issue_rope_rows(a.tab, a.n_a, a.pos_base, slot_src(a, tile(0), slot_l), raw_of(0), warp, nwarps, lane);
     cp_async_commit();
-    if (my_tiles > 1) issue_raw(a, slot_src(a, tile(1), slot_l), raw_of(1), warp, nwarps, lane);
+    if (my_tiles > 1) issue_rope_rows(a.tab, a.n_a, a.pos_base, slot_src(a, tile(1), slot_l), raw_of(1), warp, nwarps, lane);
     cp_async_commit();
     if (my_tiles > 2) src_pref = slot_src(a, tile(2), slot_l);
     cp_async_wait<1>();
     __syncthreads();
-    if (my_tiles > 0) combine_raw(raw_of(0), cs_of(0), tid, nthreads);
+    if (my_tiles > 0) combine_rope_rows(raw_of(0), cs_of(0), tid, nthreads);
   }
   if (my_tiles > 0) load_codes<BITS>(a, first, warp, slot_l, w, meta);
 
@@ -709,10 +653,10 @@ __global__ void __launch_bounds__(256, 2)
       // rows of tile k+1 landed (everyone's), table k combined, tile k-1 decoded
       cp_async_wait<0>();
       __syncthreads();
-      if (k + 2 < my_tiles) issue_raw(a, src_pref, raw_of(k), warp, nwarps, lane);
+      if (k + 2 < my_tiles) issue_rope_rows(a.tab, a.n_a, a.pos_base, src_pref, raw_of(k), warp, nwarps, lane);
       cp_async_commit();
       if (k + 3 < my_tiles) src_pref = slot_src(a, tile(k + 3), slot_l);
-      if (k + 1 < my_tiles) combine_raw(raw_of(k + 1), cs_of(k + 1), tid, nthreads);
+      if (k + 1 < my_tiles) combine_rope_rows(raw_of(k + 1), cs_of(k + 1), tid, nthreads);
     }
     const Tile tl = tile(k);
     const int h = tl.group * a.hg + warp;
@@ -740,12 +684,6 @@ __global__ void __launch_bounds__(256, 2)
 }
 
 // ---------------------------------------------------------------- launch
-static int pick_head_group(int heads) {
-  for (int g = 8; g >= 1; --g)
-    if (heads % g == 0) return g;
-  return 1;
-}
-
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against the driver library).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -1,7 +1,8 @@
-// nq_codec_math.cuh -- the codec arithmetic shared by the decode kernel and
-// the attention kernel (sm_100a): the in-thread Walsh-Hadamard transform of a
-// half vector, code unpacking, and the reconstruction x = fp32(w * kappa) of
-// one thread's 64 coordinates from a packed vector.
+// nq_codec_math.cuh -- the codec arithmetic shared by the encode, decode and
+// attention kernels (sm_100a): the in-thread Walsh-Hadamard transform of a
+// half vector, code unpacking, the reconstruction x = fp32(w * kappa) of one
+// thread's 64 coordinates from a packed vector, and the staging of the
+// two-level RoPE table for tiles of 16 vectors.
 //
 // Thread layout: two threads own one 128-vector; half h holds the coordinate
 // pairs (x_i, x_{i+64}) for i in [32h, 32h+32) as packed fp32x2 registers.
@@ -10,6 +11,72 @@
 #include "nq_device.cuh"
 
 namespace nq {
+
+constexpr int kSlots = 16;                  // vectors per tile: one warp = 16 slots x 2 halves
+constexpr int kCsBytes = 32 * kSlots * 16;  // float4 cs[32][16]
+
+// ------------------------------------------------------ RoPE table rows
+// The table holds cos/sin of the angles 256a * theta_i (rows a < n_a) and
+// b * theta_i (rows n_a + b, b < 256) as 64 (c, s) pairs per row.  The rows of
+// a tile are staged raw: for each of the 16 slots the A row of its position
+// p = 256a + b and its B row, 512 bytes each, at a padded stride of kRawSlot
+// bytes per slot.  Warp w copies the rows of slots w, w + nwarps, ...: one
+// 16-byte chunk per lane per row.  src_lane is the position minus pos_base of
+// the lane's slot (lanes l and l+16 share slot l % 16), -1 for an empty slot.
+constexpr int kRawSlot = 1024 + 16;
+constexpr int kRawBytes = kSlots * kRawSlot;
+
+__device__ __forceinline__ void issue_rope_rows(const float2* tab, int64_t n_a, int64_t pos_base,
+                                                int32_t src_lane, uint32_t raw, int warp,
+                                                int nwarps, int lane) {
+  for (int slot = warp; slot < kSlots; slot += nwarps) {  // warp-uniform
+    const int32_t src = __shfl_sync(0xffffffffu, src_lane, slot);
+    if (src < 0) continue;
+    const int64_t pos = pos_base + src;
+    int64_t hi = pos >> 8;
+    hi = hi < 0 ? 0 : (hi >= n_a ? n_a - 1 : hi);  // out-of-contract positions stay in bounds
+    const char* rowA = reinterpret_cast<const char*>(tab + hi * kHalf);
+    const char* rowB = reinterpret_cast<const char*>(tab + (n_a + (pos & 255)) * kHalf);
+    const uint32_t dst = raw + slot * kRawSlot + lane * 16;
+    cp_async16(dst, rowA + lane * 16);
+    cp_async16(dst + 512, rowB + lane * 16);
+  }
+}
+
+// cs table of one tile from its raw rows: float4 cs[j][slot] = (c_2j, s_2j,
+// c_2j+1, s_2j+1) with c = fmaf(cA, cB, -(sA sB)), s = fmaf(sA, cB, cA sB)
+// (the angle-sum rule); a thread of half h later reads j in [16h, 16h+16).
+__device__ __forceinline__ void combine_rope_rows(uint32_t raw, float4* cs, int tid,
+                                                  int nthreads) {
+  for (int e = tid; e < 32 * kSlots; e += nthreads) {
+    const int slot = e & 15, j = e >> 4;
+    const float4 A = lds128f(raw + slot * kRawSlot + j * 16);
+    const float4 B = lds128f(raw + slot * kRawSlot + 512 + j * 16);
+    float4 v;
+    v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
+    v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
+    v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
+    v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
+    cs[j * kSlots + slot] = v;
+  }
+}
+
+// Rotation of this thread's half vector at its position:
+// o_i = fmaf(x_i, c, -(x_{i+64} s)), o_{i+64} = fmaf(x_{i+64}, c, x_i s), with
+// (c, s) read from the cs table at csa = cs + (16 half * kSlots + slot) * 16.
+__device__ __forceinline__ void rope_half(float2 (&v)[32], uint32_t csa) {
+#pragma unroll
+  for (int jj = 0; jj < 16; ++jj) {
+    const float4 t = lds128f(csa + jj * (kSlots * 16));
+#pragma unroll
+    for (int ww = 0; ww < 2; ++ww) {
+      const float c = ww ? t.z : t.x, s = ww ? t.w : t.y;
+      const float2 P = v[2 * jj + ww];
+      const float2 Q = mul2(P, make_float2(s, s));
+      v[2 * jj + ww] = make_float2(__fmaf_rn(P.x, c, -Q.y), __fmaf_rn(P.y, c, Q.x));
+    }
+  }
+}
 
 // ------------------------------------------------------ Hadamard (fp32)
 // Unnormalised Sylvester transform, stages h = 1, 2, ..., 64 in this order.

@@ -11,6 +11,14 @@
 
 namespace nq {
 
+// Heads per CTA of the tiled kernels (one warp per head): the largest divisor
+// of the head count up to 8.
+inline int pick_head_group(int heads) {
+  for (int g = 8; g >= 1; --g)
+    if (heads % g == 0) return g;
+  return 1;
+}
+
 struct EncodeLaunch {
   const void* K;
   nq_kv_strides ks;
@@ -62,6 +70,7 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 
 cudaError_t codec_read_clear_error(uint32_t* flags);
 size_t attend_workspace_floats(int units, int heads, int G, int64_t n);
+int64_t attend_ctas(int units, int heads, int64_t n);  // CTAs of the partial kernel
 cudaError_t launch_attend(const AttendLaunch& L, cudaStream_t stream);
 cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
                                uint8_t* coset, cudaStream_t stream);

@@ -233,9 +233,11 @@ nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int
  * sums), so results agree with an exact evaluation to about 1e-5 relative,
  * not bit for bit.  q: fp32 [units][heads*G][128], 16-byte aligned.
  * out: fp32 [units][heads*G][128].  k_in/v_in: packed stores as for
- * nq_decode (any bits 2/3).  1 <= G <= 8, n >= 1.  ws: device workspace of
+ * nq_decode (any bits 2/3).  1 <= G <= 8, 1 <= n < 2^31 (larger n returns
+ * NQ_ERR_UNSUPPORTED).  ws: device workspace of
  * nq_attend_workspace_bytes(units, heads, G, n) bytes, 16-byte aligned
- * (per-chunk partial results).  rope_tab as for nq_decode. */
+ * (per-chunk partial results; the token chunk per CTA depends on units,
+ * heads and n only).  rope_tab as for nq_decode. */
 size_t nq_attend_workspace_bytes(int units, int heads, int G, int64_t n);
 nq_status nq_attend(const float *q, int units, int heads, int G, const nq_packed *k_in,
                     const nq_packed *v_in, int64_t n, int64_t slot0, const int32_t *positions,

@@ -2,14 +2,15 @@
 
 The kernel reconstructs keys and values in fp32 exactly as the decode path
 does before its bf16 rounding, but scores, exponentials and sums run in fp32
-in the kernel's own order (chunks of 256 tokens, values accumulated in the
-Hadamard code domain and transformed once per query head).  Bound used here,
+in the kernel's own order (online softmax over tiles of 16 tokens within
+chunks of at least 64, values accumulated in the Hadamard code domain and
+transformed once per query head).  Bound used here,
 per output vector (the per-vector relative form of the reconstruction bound
 on K/V, ten times tighter): ||out - out_ref||_2 <= 1e-4 ||out_ref||_2, and
 |lse - lse_ref| <= 1e-4 (1 + |lse_ref|).  Sources of error: a 128-term fp32
 dot product per score (relative error of order sqrt(128) 2^-24 of
-sum |q_i k_i|), the fp32 exponential (2^-21 relative), 128-term fp32 sums of
-weighted codes per token stream, and the fp32 Hadamard transform of the
+sum |q_i k_i|), the fp32 exponential (2^-21 relative), fp32 running sums of
+weighted codes over each chunk, and the fp32 Hadamard transform of the
 merged sums (128 terms per output); together of order 1e-6 of ||out||, so
 the bound leaves two orders of magnitude of margin for cancellation in
 averaged outputs.
@@ -84,6 +85,18 @@ def test_attend_ragged_lengths_and_formats(nq, oq, n, G, bits_k, bits_v):
     wl = synth.WORKLOADS["qwen25_7b_64k"]
     k, v = synth.gen_layer(wl, 5, "cuda", tokens=n)
     check(nq, oq, k[None], v[None], None, n, G, bits_k, bits_v, wl.theta, pos_base=300, seed=n)
+
+
+def test_attend_two_head_groups_several_units(nq, oq):
+    """12 KV heads (two CTAs of 6 warps per chunk), 3 units, 700 tokens."""
+    wl = synth.WORKLOADS["tiny"]
+    K, V = [], []
+    for u in range(3):
+        k0, v0 = synth.gen_layer(wl, 2 * u, "cuda", tokens=700)
+        k1, v1 = synth.gen_layer(wl, 2 * u + 1, "cuda", tokens=700)
+        K.append(torch.cat([k0, k1[:4]]))
+        V.append(torch.cat([v0, v1[:4]]))
+    check(nq, oq, torch.stack(K), torch.stack(V), None, 700, 2, 3, 2, wl.theta, seed=5)
 
 
 def test_attend_sharp_and_flat_softmax(nq, oq):
