@@ -78,6 +78,11 @@ def _load():
             "oq_rope_apply_batch": (None, [P, P, P, i64, i32]),
             "oq_encode_batch": (i64, [P, i64, i32, P, P, i32, P, P]),
             "oq_decode_batch": (None, [P, P, i64, i32, P, P, i32, P]),
+            "oq_ans_table": (None, [P, i32, P]),
+            "oq_ans_encode": (i64, [P, i64, P, i32, P, i64]),
+            "oq_ans_decode": (i64, [P, i64, P, i32, P, i64]),
+            "oq_entropy_encode_store": (i64, [P, i64, i32, i64, i32, i32, P, P, P, i64]),
+            "oq_entropy_decode_store": (i32, [P, P, P, i64, i32, i64, i32, i32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -301,3 +306,72 @@ def attend_unit(k_codes, k_meta, v_codes, v_meta, q, G: int, scale: float, posit
     _load().oq_attend_unit(_p(kc), _p(km), _p(vc), _p(vm), H, G, n, _p(pp), int(pos_base),
                            float(theta), bits_k, bits_v, _p(q), float(scale), _p(out), _p(lse))
     return out, lse
+
+
+# ------------------------------------------------- delta + entropy stage
+ANS_M = 4096
+ANS_SEG = 2048  # tokens per stream segment
+
+
+def ans_table(counts) -> np.ndarray:
+    """Quantised rANS frequencies (sum 4096) of symbol counts."""
+    counts = np.ascontiguousarray(counts, dtype=np.uint64)
+    F = np.empty(counts.size, np.uint16)
+    _load().oq_ans_table(_p(counts), counts.size, _p(F))
+    return F
+
+
+def ans_encode(sym, F) -> np.ndarray:
+    """One rANS stream of 16-bit words (final state first)."""
+    sym = np.ascontiguousarray(sym, dtype=np.uint8)
+    F = np.ascontiguousarray(F, dtype=np.uint16)
+    cap = sym.size + 2
+    out = np.empty(cap, np.uint16)
+    n = _load().oq_ans_encode(_p(sym), sym.size, _p(F), F.size, _p(out), cap)
+    if n < 0:
+        raise ValueError("oq_ans_encode failed (%d)" % n)
+    return out[:n].copy()
+
+
+def ans_decode(words, F, count: int) -> tuple[np.ndarray, int]:
+    """Decode count symbols; returns (symbols, words read or -1)."""
+    words = np.ascontiguousarray(words, dtype=np.uint16)
+    F = np.ascontiguousarray(F, dtype=np.uint16)
+    sym = np.empty(count, np.uint8)
+    used = _load().oq_ans_decode(_p(words), words.size, _p(F), F.size, _p(sym), count)
+    return sym, int(used)
+
+
+def entropy_streams(units: int, heads: int, n: int) -> int:
+    return units * heads * ((n + ANS_SEG - 1) // ANS_SEG) * D
+
+
+def entropy_encode_store(codes, bits: int, delta: bool):
+    """codes: uint32 [units][heads][n][4*bits].  Returns (freq [units][heads][2^bits]
+    uint16, offsets [streams + 1] uint32, words uint16)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    units, heads, n = codes.shape[:3]
+    S = entropy_streams(units, heads, n)
+    cap = S * (ANS_SEG + 2)
+    freq = np.empty((units, heads, 1 << bits), np.uint16)
+    offsets = np.empty(S + 1, np.uint32)
+    words = np.empty(cap, np.uint16)
+    tot = _load().oq_entropy_encode_store(_p(codes), units, heads, n, bits, int(delta), _p(freq),
+                                          _p(offsets), _p(words), cap)
+    if tot < 0:
+        raise ValueError("oq_entropy_encode_store failed")
+    return freq, offsets, words[:tot].copy()
+
+
+def entropy_decode_store(words, offsets, freq, units: int, heads: int, n: int, bits: int,
+                         delta: bool) -> np.ndarray:
+    """Inverse of entropy_encode_store: uint32 codes [units][heads][n][4*bits]."""
+    words = np.ascontiguousarray(words, dtype=np.uint16)
+    offsets = np.ascontiguousarray(offsets, dtype=np.uint32)
+    freq = np.ascontiguousarray(freq, dtype=np.uint16)
+    codes = np.empty((units, heads, n, 4 * bits), np.uint32)
+    rc = _load().oq_entropy_decode_store(_p(words), _p(offsets), _p(freq), units, heads, n, bits,
+                                         int(delta), _p(codes))
+    if rc != 0:
+        raise ValueError("oq_entropy_decode_store: inconsistent stream")
+    return codes

@@ -616,3 +616,214 @@ void oq_decode_batch(const uint32_t *words, const uint32_t *meta, int64_t n, int
         oq_decode_vector(words + 4 * bits * i, meta[i], rope, c + OQ_HALF * i, s + OQ_HALF * i,
                          bits, out + OQ_D * i);
 }
+
+/* ------------------------------------------------- delta + entropy stage */
+
+/* The lattice indices (the b-bit codes) of a packed store, coded the way the
+ * NexusQuant pages describe their last step: consecutive tokens give similar
+ * lattice indices, so the difference to the previous token is stored and the
+ * result compressed ("Implementation details" of the zingnex.cn page; step 6
+ * of the dev.to page, which names zstd).  zstd is a third-party library, so
+ * the compressor here is range-variant asymmetric numeral systems (rANS,
+ * J. Duda, "Asymmetric numeral systems", 2013) with a static frequency table;
+ * streams, table rule and word format are the library's reading:
+ *
+ *   streams  one per (unit, head, segment of OQ_SEG tokens, coordinate c),
+ *            in that order (coordinate fastest); symbols
+ *            d_t = (j_t - j_{t-1}) mod 2^b inside the segment, d = j at the
+ *            segment's first token (or d_t = j_t when the difference is off);
+ *   table    per (unit, head), over the symbols of all its streams:
+ *            F_s = 0 for an absent symbol, else max(1, floor(count_s M / total))
+ *            with M = 4096, and the remainder M - sum F added to the largest F
+ *            (the lowest symbol on ties); C_s = sum_{r<s} F_r;
+ *   encoder  state x in [2^16, 2^32), starting at 2^16, symbols taken last to
+ *            first: if x >= F_s 2^20, emit x mod 2^16 and x = floor(x / 2^16);
+ *            then x = floor(x / F_s) M + (x mod F_s) + C_s;
+ *   stream   the final state (low 16 bits, high 16 bits), then the emitted
+ *            words from the last emitted to the first;
+ *   decoder  slot = x mod M; s = the symbol with C_s <= slot < C_s + F_s;
+ *            x = F_s floor(x / M) + slot - C_s; if x < 2^16, x = x 2^16 + the
+ *            next word. */
+#define OQ_ANS_M 4096u
+#define OQ_ANS_L 65536u
+#define OQ_SEG 2048
+
+void oq_ans_table(const uint64_t *counts, int A, uint16_t *F)
+{
+    uint64_t total = 0;
+    for (int s = 0; s < A; s++) total += counts[s];
+    int64_t sum = 0;
+    for (int s = 0; s < A; s++) {
+        uint64_t f = 0;
+        if (counts[s]) {
+            f = counts[s] * OQ_ANS_M / total;
+            if (f < 1) f = 1;
+        }
+        F[s] = (uint16_t)f;
+        sum += (int64_t)f;
+    }
+    int best = 0;
+    for (int s = 1; s < A; s++)
+        if (F[s] > F[best]) best = s;
+    F[best] = (uint16_t)((int64_t)F[best] + ((int64_t)OQ_ANS_M - sum));
+}
+
+static void oq_ans_cum(const uint16_t *F, int A, uint32_t *C)
+{
+    C[0] = 0;
+    for (int s = 0; s < A; s++) C[s + 1] = C[s] + F[s];
+}
+
+/* One stream: returns its length in 16-bit words (written to out[0..len)),
+ * -1 when cap words do not suffice, -2 for a symbol of frequency 0. */
+int64_t oq_ans_encode(const uint8_t *sym, int64_t count, const uint16_t *F, int A, uint16_t *out,
+                      int64_t cap)
+{
+    uint32_t C[257];
+    oq_ans_cum(F, A, C);
+    int64_t p = cap; /* emitted words fill out[] from the end */
+    uint32_t x = OQ_ANS_L;
+    for (int64_t t = count - 1; t >= 0; t--) {
+        uint32_t s = sym[t], f = F[s];
+        if (f == 0) return -2;
+        if ((uint64_t)x >= ((uint64_t)f << 20)) {
+            if (p == 0) return -1;
+            out[--p] = (uint16_t)(x & 0xFFFFu);
+            x >>= 16;
+        }
+        x = (x / f) * OQ_ANS_M + (x % f) + C[s];
+    }
+    if (p < 2) return -1;
+    out[--p] = (uint16_t)(x >> 16);
+    out[--p] = (uint16_t)(x & 0xFFFFu);
+    int64_t len = cap - p;
+    memmove(out, out + p, (size_t)len * sizeof(uint16_t));
+    return len;
+}
+
+/* Inverse of oq_ans_encode: count symbols from a stream of len words;
+ * returns the words read, -1 if the stream ends early. */
+int64_t oq_ans_decode(const uint16_t *in, int64_t len, const uint16_t *F, int A, uint8_t *sym,
+                      int64_t count)
+{
+    uint32_t C[257];
+    oq_ans_cum(F, A, C);
+    if (len < 2) return -1;
+    uint32_t x = (uint32_t)in[0] | ((uint32_t)in[1] << 16);
+    int64_t i = 2;
+    for (int64_t t = 0; t < count; t++) {
+        uint32_t slot = x & (OQ_ANS_M - 1u);
+        int s = 0;
+        while (s + 1 < A && C[s + 1] <= slot) s++;
+        sym[t] = (uint8_t)s;
+        x = F[s] * (x >> 12) + slot - C[s];
+        if (x < OQ_ANS_L) {
+            if (i >= len) return -1;
+            x = (x << 16) | in[i++];
+        }
+    }
+    return i;
+}
+
+static uint32_t oq_get_code(const uint32_t *words, int bits, int c)
+{
+    uint32_t j = 0;
+    int bitpos = bits * c;
+    for (int k = 0; k < bits; k++)
+        j |= ((words[(bitpos + k) >> 5] >> ((bitpos + k) & 31)) & 1u) << k;
+    return j;
+}
+
+static void oq_put_code(uint32_t *words, int bits, int c, uint32_t j)
+{
+    int bitpos = bits * c;
+    for (int k = 0; k < bits; k++)
+        if (j & (1u << k)) words[(bitpos + k) >> 5] |= 1u << ((bitpos + k) & 31);
+}
+
+/* Symbols of the stream (segment g, coordinate c) of one (unit, head):
+ * codes holds its n vectors of 4*bits words. */
+static int64_t oq_stream_symbols(const uint32_t *codes, int64_t n, int bits, int delta, int64_t g,
+                                 int c, uint8_t *sym)
+{
+    int64_t t0 = g * OQ_SEG, t1 = t0 + OQ_SEG < n ? t0 + OQ_SEG : n;
+    uint32_t mask = (1u << bits) - 1u, prev = 0;
+    for (int64_t t = t0; t < t1; t++) {
+        uint32_t j = oq_get_code(codes + 4 * bits * t, bits, c);
+        sym[t - t0] = (uint8_t)(delta ? ((j - prev) & mask) : j);
+        prev = j;
+    }
+    return t1 - t0;
+}
+
+/* Encode the codes of units x heads x n vectors (codes: [units][heads][n][4 bits]
+ * contiguous): freq [units][heads][2^bits], offsets [streams + 1] (stream i
+ * occupies words[offsets[i] .. offsets[i+1])).  Returns the total words, -1
+ * if cap words do not suffice. */
+int64_t oq_entropy_encode_store(const uint32_t *codes, int64_t units, int heads, int64_t n,
+                                int bits, int delta, uint16_t *freq, uint32_t *offsets,
+                                uint16_t *words, int64_t cap)
+{
+    int A = 1 << bits;
+    int64_t nseg = (n + OQ_SEG - 1) / OQ_SEG, stream = 0, off = 0;
+    uint8_t *sym = malloc(OQ_SEG);
+    for (int64_t uh = 0; uh < units * heads; uh++) {
+        const uint32_t *cu = codes + uh * n * 4 * bits;
+        uint64_t counts[8] = {0};
+        for (int64_t g = 0; g < nseg; g++)
+            for (int c = 0; c < OQ_D; c++) {
+                int64_t m = oq_stream_symbols(cu, n, bits, delta, g, c, sym);
+                for (int64_t t = 0; t < m; t++) counts[sym[t]]++;
+            }
+        uint16_t *F = freq + uh * A;
+        oq_ans_table(counts, A, F);
+        for (int64_t g = 0; g < nseg; g++)
+            for (int c = 0; c < OQ_D; c++) {
+                int64_t m = oq_stream_symbols(cu, n, bits, delta, g, c, sym);
+                int64_t len = oq_ans_encode(sym, m, F, A, words + off, cap - off);
+                if (len < 0) {
+                    free(sym);
+                    return -1;
+                }
+                offsets[stream++] = (uint32_t)off;
+                off += len;
+            }
+    }
+    offsets[stream] = (uint32_t)off;
+    free(sym);
+    return off;
+}
+
+/* Inverse of oq_entropy_encode_store: rebuilds the code words (meta is not
+ * part of the streams).  Returns 0, or -1 if a stream is inconsistent. */
+int oq_entropy_decode_store(const uint16_t *words, const uint32_t *offsets, const uint16_t *freq,
+                            int64_t units, int heads, int64_t n, int bits, int delta,
+                            uint32_t *codes)
+{
+    int A = 1 << bits;
+    uint32_t mask = (1u << bits) - 1u;
+    int64_t nseg = (n + OQ_SEG - 1) / OQ_SEG, stream = 0;
+    uint8_t *sym = malloc(OQ_SEG);
+    memset(codes, 0, (size_t)(units * heads * n * 4 * bits) * sizeof(uint32_t));
+    for (int64_t uh = 0; uh < units * heads; uh++) {
+        uint32_t *cu = codes + uh * n * 4 * bits;
+        const uint16_t *F = freq + uh * A;
+        for (int64_t g = 0; g < nseg; g++)
+            for (int c = 0; c < OQ_D; c++, stream++) {
+                int64_t t0 = g * OQ_SEG, t1 = t0 + OQ_SEG < n ? t0 + OQ_SEG : n;
+                int64_t len = (int64_t)offsets[stream + 1] - (int64_t)offsets[stream];
+                int64_t used = oq_ans_decode(words + offsets[stream], len, F, A, sym, t1 - t0);
+                if (used != len) {
+                    free(sym);
+                    return -1;
+                }
+                uint32_t j = 0;
+                for (int64_t t = t0; t < t1; t++) {
+                    j = delta ? ((j + sym[t - t0]) & mask) : sym[t - t0];
+                    oq_put_code(cu + 4 * bits * t, bits, c, j);
+                }
+            }
+    }
+    free(sym);
+    return 0;
+}

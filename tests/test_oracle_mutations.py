@@ -55,6 +55,16 @@ MUTATIONS = [
      "tests/test_oracle_attend.py::test_attention_equals_library_softmax"),
     ("attend-lse", "lse[h * G + g] = m + log(l);", "lse[h * G + g] = log(l);",
      "tests/test_oracle_attend.py::test_attention_equals_library_softmax"),
+    ("ans-table-tie", "if (F[s] > F[best]) best = s;", "if (F[s] >= F[best]) best = s;",
+     "tests/test_oracle_entropy.py::test_table_rule_worked_examples"),
+    ("ans-renorm-threshold", "if ((uint64_t)x >= ((uint64_t)f << 20)) {",
+     "if ((uint64_t)x >= ((uint64_t)f << 21)) {",
+     "tests/test_oracle_entropy.py::test_round_trip_and_size_bound"),
+    ("ans-cumulative-offset", "x = (x / f) * OQ_ANS_M + (x % f) + C[s];",
+     "x = (x / f) * OQ_ANS_M + (x % f) + C[s] + 1;",
+     "tests/test_oracle_entropy.py::test_round_trip_and_size_bound"),
+    ("entropy-delta-reference", "        prev = j;\n", "        prev = 0;\n",
+     "tests/test_oracle_entropy.py::test_store_layout_matches_a_numpy_restatement"),
 ]
 
 
