@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-attend", action="store_true", help="skip the decode-attention timing")
+    ap.add_argument("--no-entropy", action="store_true",
+                    help="skip the delta + entropy stage timing")
     ap.add_argument("--layers", type=int, default=0, help="override layer count (small runs)")
     ap.add_argument("--tokens", type=int, default=0, help="override token count (small runs)")
     return ap.parse_args()
@@ -460,6 +462,9 @@ def run_ours(args, world, rank, local):
 
     if not args.no_attend:
         line["decode_attention"] = attend_timing(args, codec, Kd, Vd, stream, world)
+    if not args.no_entropy:
+        line["entropy_stage"] = entropy_timing(args, codec, stream, world,
+                                               K.numel() + V.numel())
     if not args.no_e2e:
         line["e2e"] = e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes)
     if not args.no_cpu_baseline and rank == 0:
@@ -518,6 +523,65 @@ def attend_timing(args, codec, Kd, Vd, stream, world, G: int = 4):
             "fused_ms": f_ms, "decode_then_sdpa_ms": u_ms, "sdpa_on_bf16_ms": s_ms,
             "speedup_vs_decode_then_sdpa": u_ms / f_ms,
             "fused_packed_read_gbs": packed / (f_ms * 1e-3) / 1e9}
+
+
+def entropy_timing(args, codec, stream, world, total_elems):
+    """The delta + rANS stage over the lattice indices of the whole packed
+    cache (keys and values, every layer in one call each): coded size and
+    encode / decode time, with and without the token difference.  Code bits
+    are per kept element; the cache figure (coded codes + raw meta) is per
+    element of the bf16 input cache, like bits_per_elem.  CUDA events, max
+    over ranks."""
+    from e8_lattice_vector_nq_b200 import nq
+
+    res = {}
+    elems = 0
+    for name, st in (("k", codec.k_store), ("v", codec.v_store)):
+        elems += st.meta.numel() * 128
+    dev = codec.k_store.codes.device
+    out = {"k": nq.PackedStore.empty(codec.units, codec.heads, codec.n, codec.k_store.bits, dev),
+           "v": nq.PackedStore.empty(codec.units, codec.heads, codec.n, codec.v_store.bits, dev)}
+    ws = nq.entropy_workspace(codec.units, codec.heads, codec.n, dev)
+    coded = {}
+    for delta in (True, False):
+
+        def enc():
+            for name, st in (("k", codec.k_store), ("v", codec.v_store)):
+                coded[name] = nq.nq_entropy_encode(st, codec.n, delta=delta, ws=ws,
+                                                   coded=coded.get(name))
+
+        def dec():
+            for name in ("k", "v"):
+                nq.nq_entropy_decode(coded[name], out[name])
+
+        def t(fn, reps=5):
+            fn()
+            torch.cuda.synchronize()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            for _ in range(reps):
+                fn()
+            e.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(s.elapsed_time(e) / reps, world, dev)
+
+        enc_ms = t(enc)
+        dec_ms = t(dec)
+        exact = all(torch.equal(out[nm].codes, st.codes)
+                    for nm, st in (("k", codec.k_store), ("v", codec.v_store)))
+        coded_bytes = sum(c.coded_bytes() for c in coded.values())
+        code_bytes = codec.k_store.codes.numel() * 4 + codec.v_store.codes.numel() * 4
+        meta_bytes = codec.k_store.meta.numel() * 4 + codec.v_store.meta.numel() * 4
+        res["delta" if delta else "plain"] = {
+            "encode_ms": enc_ms, "decode_ms": dec_ms,
+            "codes_bits_per_elem_raw": code_bytes * 8 / elems,
+            "codes_bits_per_elem_coded": coded_bytes * 8 / elems,
+            "codes_ratio": code_bytes / coded_bytes,
+            "cache_bits_per_elem_with_meta": (coded_bytes + meta_bytes) * 8 / total_elems,
+            "encode_gbs_codes_in": code_bytes / (enc_ms * 1e-3) / 1e9,
+            "decode_gbs_codes_out": code_bytes / (dec_ms * 1e-3) / 1e9,
+            "round_trip_exact": bool(exact)}
+    return res
 
 
 def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):

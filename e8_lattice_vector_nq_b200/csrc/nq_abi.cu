@@ -372,6 +372,70 @@ nq_status nq_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* cod
                      "nq_e8_quantise launch");
 }
 
+int64_t nq_entropy_streams(int units, int heads, int64_t n) {
+  if (units < 0 || heads < 1 || n < 1) return 0;
+  return nq::entropy_streams(units, heads, n);
+}
+
+int64_t nq_entropy_max_words(int units, int heads, int64_t n) {
+  if (units < 0 || heads < 1 || n < 1) return 0;
+  return nq::entropy_max_words(units, heads, n);
+}
+
+size_t nq_entropy_workspace_bytes(int units, int heads, int64_t n) {
+  if (units < 0 || heads < 1 || n < 1) return 0;
+  return nq::entropy_workspace_bytes(units, heads, n);
+}
+
+static nq_status check_entropy_shape(int units, int heads, int64_t n, int64_t slot0, int delta) {
+  if (units < 0 || heads < 1 || heads > 1024)
+    return fail(NQ_ERR_INVALID, "need units >= 0 and 1 <= heads <= 1024");
+  if (n < 1 || n >= (int64_t(1) << 25))
+    return fail(NQ_ERR_INVALID, "need 1 <= n < 2^25 (got %lld)", static_cast<long long>(n));
+  if (slot0 < 0) return fail(NQ_ERR_INVALID, "slot0 must be >= 0");
+  if (delta != 0 && delta != 1) return fail(NQ_ERR_INVALID, "delta must be 0 or 1");
+  if (nq::entropy_max_words(units, heads, n) > 0xFFFFFFFFll)
+    return fail(NQ_ERR_UNSUPPORTED, "units * heads * n too large for 32-bit stream offsets");
+  return NQ_OK;
+}
+
+nq_status nq_entropy_encode(const nq_packed* in, int units, int heads, int64_t n, int64_t slot0,
+                            int delta, uint16_t* freq, uint32_t* offsets, uint16_t* words,
+                            int64_t words_cap, void* ws, size_t ws_bytes, nq_stream_t stream) {
+  if (nq_status st = check_entropy_shape(units, heads, n, slot0, delta)) return st;
+  if (nq_status st = check_packed(in, "in")) return st;
+  if (units == 0) return NQ_OK;
+  if (!freq || !offsets || !words || !ws)
+    return fail(NQ_ERR_INVALID, "freq, offsets, words and ws must be non-NULL");
+  if (!aligned(freq, 2) || !aligned(offsets, 4) || !aligned(words, 2) || !aligned(ws, 16))
+    return fail(NQ_ERR_INVALID, "freq/words 2-byte, offsets 4-byte, ws 16-byte aligned");
+  if (words_cap < nq::entropy_max_words(units, heads, n))
+    return fail(NQ_ERR_WORKSPACE, "words_cap %lld < nq_entropy_max_words %lld",
+                static_cast<long long>(words_cap),
+                static_cast<long long>(nq::entropy_max_words(units, heads, n)));
+  const size_t need = nq::entropy_workspace_bytes(units, heads, n);
+  if (ws_bytes < need)
+    return fail(NQ_ERR_WORKSPACE, "entropy workspace too small: %zu < %zu", ws_bytes, need);
+  return cuda_status(nq::launch_entropy_encode(*in, units, heads, n, slot0, delta, freq, offsets,
+                                               words, ws, reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_entropy_encode launch");
+}
+
+nq_status nq_entropy_decode(const uint16_t* words, const uint32_t* offsets, const uint16_t* freq,
+                            int units, int heads, int64_t n, int delta, const nq_packed* out,
+                            int64_t slot0, nq_stream_t stream) {
+  if (nq_status st = check_entropy_shape(units, heads, n, slot0, delta)) return st;
+  if (nq_status st = check_packed(out, "out")) return st;
+  if (units == 0) return NQ_OK;
+  if (!freq || !offsets || !words)
+    return fail(NQ_ERR_INVALID, "words, offsets and freq must be non-NULL");
+  if (!aligned(freq, 2) || !aligned(offsets, 4) || !aligned(words, 2))
+    return fail(NQ_ERR_INVALID, "freq/words 2-byte, offsets 4-byte aligned");
+  return cuda_status(nq::launch_entropy_decode(words, offsets, freq, units, heads, n, delta, *out,
+                                               slot0, reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_entropy_decode launch");
+}
+
 nq_status nq_device_error(uint32_t* flags_out) {
   if (!flags_out) return fail(NQ_ERR_INVALID, "flags_out is NULL");
   return cuda_status(nq::codec_read_clear_error(flags_out), "nq_device_error");

@@ -75,6 +75,17 @@ cudaError_t launch_attend(const AttendLaunch& L, cudaStream_t stream);
 cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
                                uint8_t* coset, cudaStream_t stream);
 
+int64_t entropy_streams(int units, int heads, int64_t n);
+int64_t entropy_max_words(int units, int heads, int64_t n);
+size_t entropy_workspace_bytes(int units, int heads, int64_t n);
+cudaError_t launch_entropy_encode(const nq_packed& in, int units, int heads, int64_t n,
+                                  int64_t slot0, int delta, uint16_t* freq, uint32_t* offsets,
+                                  uint16_t* words, void* ws, cudaStream_t stream);
+cudaError_t launch_entropy_decode(const uint16_t* words, const uint32_t* offsets,
+                                  const uint16_t* freq, int units, int heads, int64_t n,
+                                  int delta, const nq_packed& out, int64_t slot0,
+                                  cudaStream_t stream);
+
 cudaError_t launch_score(const void* K, nq_kv_strides ks, int units, int heads, int64_t T, int W,
                          double* scores, float* mean_ws, cudaStream_t stream);
 cudaError_t launch_score_static(const void* K, nq_kv_strides ks, int units, int heads, int64_t T,

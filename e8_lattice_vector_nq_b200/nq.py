@@ -43,7 +43,8 @@ EXPORTS = (
     "nq_rope_tables_fill_host", "nq_score_workspace_bytes", "nq_score", "nq_score_static",
     "nq_kept_count",
     "nq_select", "nq_encode", "nq_decode", "nq_e8_quantise", "nq_attend_workspace_bytes",
-    "nq_attend", "nq_device_error",
+    "nq_attend", "nq_device_error", "nq_entropy_streams", "nq_entropy_max_words",
+    "nq_entropy_workspace_bytes", "nq_entropy_encode", "nq_entropy_decode",
 )
 
 
@@ -77,6 +78,11 @@ def lib() -> ctypes.CDLL:
         "nq_attend": (i32, [P, i32, i32, i32, PK, PK, i64, i64, P, i64, i64, P, i64,
                             ctypes.c_float, P, P, P, sz, P]),
         "nq_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32)]),
+        "nq_entropy_streams": (i64, [i32, i32, i64]),
+        "nq_entropy_max_words": (i64, [i32, i32, i64]),
+        "nq_entropy_workspace_bytes": (sz, [i32, i32, i64]),
+        "nq_entropy_encode": (i32, [PK, i32, i32, i64, i64, i32, P, P, P, i64, P, sz, P]),
+        "nq_entropy_decode": (i32, [P, P, P, i32, i32, i64, i32, PK, i64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -317,6 +323,71 @@ def nq_e8_quantise(y: torch.Tensor, bits: int, stream=None):
     coset = torch.empty(g, dtype=torch.uint8, device=y.device)
     _check(lib().nq_e8_quantise(_ptr(y), g, int(bits), _ptr(codes), _ptr(coset), _stream(stream)))
     return codes, coset
+
+
+class EntropyCoded:
+    """Output of nq_entropy_encode (device tensors; see nq.h): words (uint16 in
+    an int16 tensor of capacity nq_entropy_max_words), offsets (uint32 in an
+    int32 tensor, [streams + 1]) and freq ([units][heads][2^bits], uint16 in
+    int16)."""
+
+    def __init__(self, words, offsets, freq, units, heads, n, bits, delta):
+        self.words, self.offsets, self.freq = words, offsets, freq
+        self.units, self.heads, self.n, self.bits, self.delta = units, heads, n, bits, delta
+
+    def total_words(self) -> int:
+        """Coded length in 16-bit words (reads offsets[streams]: synchronises)."""
+        return int(self.offsets[-1].item()) & 0xFFFFFFFF
+
+    def coded_bytes(self) -> int:
+        """Stream words plus offsets and tables, as stored."""
+        return 2 * self.total_words() + 4 * self.offsets.numel() + 2 * self.freq.numel()
+
+
+def entropy_workspace(units: int, heads: int, n: int, device="cuda") -> torch.Tensor:
+    need = lib().nq_entropy_workspace_bytes(units, heads, int(n))
+    return torch.empty(max(need, 16) // 4 + 4, dtype=torch.int32, device=device)
+
+
+def nq_entropy_encode(store: PackedStore, n: int, delta: bool = True, slot0: int = 0,
+                      ws: torch.Tensor | None = None, coded: EntropyCoded | None = None,
+                      stream=None) -> EntropyCoded:
+    """Delta + rANS coding of the codes of slots slot0 .. slot0+n-1 of every
+    (unit, head) of a packed store (see nq.h, nq_entropy_encode).  ws and
+    coded (a previous result of the same shape) may be given to reuse memory."""
+    _require_cuda(store.codes)
+    units, heads = store.meta.shape[0], store.meta.shape[1]
+    dev = store.codes.device
+    L = lib()
+    S = L.nq_entropy_streams(units, heads, int(n))
+    cap = L.nq_entropy_max_words(units, heads, int(n))
+    need = L.nq_entropy_workspace_bytes(units, heads, int(n))
+    if (coded is not None and coded.words.numel() >= cap and coded.offsets.numel() == S + 1
+            and tuple(coded.freq.shape) == (units, heads, 1 << store.bits)):
+        words, offsets, freq = coded.words, coded.offsets, coded.freq
+    else:
+        words = torch.empty(max(cap, 1), dtype=torch.int16, device=dev)
+        offsets = torch.empty(S + 1, dtype=torch.int32, device=dev)
+        freq = torch.empty(units, heads, 1 << store.bits, dtype=torch.int16, device=dev)
+    if ws is None or ws.numel() * ws.element_size() < need:
+        ws = entropy_workspace(units, heads, n, dev)
+    d = store.desc()
+    _check(L.nq_entropy_encode(ctypes.byref(d), units, heads, int(n), int(slot0), int(delta),
+                               _ptr(freq), _ptr(offsets), _ptr(words), cap, _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)))
+    return EntropyCoded(words, offsets, freq, units, heads, int(n), store.bits, bool(delta))
+
+
+def nq_entropy_decode(coded: EntropyCoded, out: PackedStore, slot0: int = 0, stream=None):
+    """Write the codes of slots slot0 .. slot0+n-1 of `out` from an
+    EntropyCoded (meta untouched; see nq.h, nq_entropy_decode)."""
+    _require_cuda(out.codes, coded.words)
+    if out.bits != coded.bits or out.meta.shape[0] != coded.units or out.meta.shape[1] != coded.heads:
+        raise ValueError("output store does not match the coded shape / bits")
+    d = out.desc()
+    _check(lib().nq_entropy_decode(_ptr(coded.words), _ptr(coded.offsets), _ptr(coded.freq),
+                                   coded.units, coded.heads, coded.n, int(coded.delta),
+                                   ctypes.byref(d), int(slot0), _stream(stream)))
 
 
 def device_error() -> int:

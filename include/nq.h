@@ -245,6 +245,45 @@ nq_status nq_attend(const float *q, int units, int heads, int G, const nq_packed
                     int64_t rope_max_pos, float scale, float *out, float *lse, void *ws,
                     size_t ws_bytes, nq_stream_t stream);
 
+/* --------------------------------------------- delta + entropy coding
+ * Lossless coding of the lattice indices (the b-bit codes) of a packed store,
+ * the last step of the NexusQuant pipeline: consecutive tokens give similar
+ * lattice indices, so the difference to the previous token is stored and the
+ * result compressed ([NQ-zh] "Implementation details"; [NQ-pt] step 6, which
+ * names zstd).  The coder is rANS (Duda, "Asymmetric numeral systems", 2013)
+ * with a static table per (unit, head); this format is the library's:
+ *   streams: one per (unit, head, segment of 2048 slots, coordinate c), in
+ *     that order (coordinate fastest), over slots slot0 .. slot0+n-1;
+ *     symbols d_t = (j_t - j_{t-1}) mod 2^b inside the segment, d = j at the
+ *     segment's first slot (delta = 1), or d_t = j_t (delta = 0);
+ *   freq [units][heads][2^b] uint16: F_s = 0 for an absent symbol, else
+ *     max(1, floor(count_s * 4096 / total)), the remainder 4096 - sum F added
+ *     to the largest F (lowest symbol on ties);
+ *   words: stream i is words[offsets[i] .. offsets[i+1]) (uint16): the final
+ *     coder state (low, high 16 bits) then the emitted words from the last
+ *     emitted to the first; offsets [streams + 1] uint32, offsets[streams] =
+ *     the total words.
+ * Meta words (coset bits, fp16 scale) are not part of the streams.
+ * nq_entropy_encode reads the code words of `in` and writes freq, offsets and
+ * words (capacity words_cap >= nq_entropy_max_words, the worst case of one
+ * word per symbol plus two per stream); ws: device workspace of
+ * nq_entropy_workspace_bytes, 16-byte aligned.  nq_entropy_decode writes the
+ * code words of `out` (slots slot0 .. slot0+n-1; meta untouched) from the
+ * output of nq_entropy_encode with the same units, heads, n, bits and delta;
+ * other inputs are out of contract (no fault: a stream never reads past its
+ * offsets, but the codes are then unspecified).  All arrays are device
+ * memory owned by the caller.  1 <= n < 2^25; units * heads * streams must
+ * keep the worst case below 2^32 words (else NQ_ERR_UNSUPPORTED). */
+int64_t nq_entropy_streams(int units, int heads, int64_t n);
+int64_t nq_entropy_max_words(int units, int heads, int64_t n);
+size_t nq_entropy_workspace_bytes(int units, int heads, int64_t n);
+nq_status nq_entropy_encode(const nq_packed *in, int units, int heads, int64_t n, int64_t slot0,
+                            int delta, uint16_t *freq, uint32_t *offsets, uint16_t *words,
+                            int64_t words_cap, void *ws, size_t ws_bytes, nq_stream_t stream);
+nq_status nq_entropy_decode(const uint16_t *words, const uint32_t *offsets, const uint16_t *freq,
+                            int units, int heads, int64_t n, int delta, const nq_packed *out,
+                            int64_t slot0, nq_stream_t stream);
+
 /* ------------------------------------------------------ E8 quantiser
  * The lattice step of nq_encode on its own ([NQ-zh] "E8 lattice
  * quantisation"; [NQ-pt] step 4), for coordinates that are already rotated

@@ -123,6 +123,25 @@ def test_validation_rejects_bad_arguments(nq):
     assert L.nq_decode(None, None, 1, 8, 64, 0, None, 0, 0, fake, 64, None, ok, None, ok, None) == nq.NQ_ERR_INVALID
     assert L.nq_decode(None, ctypes.byref(bad_bits), 1, 8, 64, 0, None, 0, 0, fake, 64, None, ok,
                        fake, ok, None) == nq.NQ_ERR_INVALID
+    # entropy stage: shape, flag, capacity and workspace checks
+    assert L.nq_entropy_encode(ctypes.byref(pk), 1, 8, 0, 0, 1, fake, fake, fake, 1 << 30, fake,
+                               1 << 30, None) == nq.NQ_ERR_INVALID
+    assert L.nq_entropy_encode(ctypes.byref(pk), 1, 8, 64, 0, 2, fake, fake, fake, 1 << 30, fake,
+                               1 << 30, None) == nq.NQ_ERR_INVALID
+    assert L.nq_entropy_encode(ctypes.byref(bad_bits), 1, 8, 64, 0, 1, fake, fake, fake, 1 << 30,
+                               fake, 1 << 30, None) == nq.NQ_ERR_INVALID
+    cap = L.nq_entropy_max_words(1, 8, 64)
+    assert cap == L.nq_entropy_streams(1, 8, 64) * 2050 == 8 * 128 * 2050
+    assert L.nq_entropy_encode(ctypes.byref(pk), 1, 8, 64, 0, 1, fake, fake, fake, cap - 1, fake,
+                               1 << 30, None) == nq.NQ_ERR_WORKSPACE
+    assert L.nq_entropy_encode(ctypes.byref(pk), 1, 8, 64, 0, 1, fake, fake, fake, cap, fake,
+                               16, None) == nq.NQ_ERR_WORKSPACE
+    assert L.nq_entropy_encode(ctypes.byref(pk), 1 << 12, 1024, 1 << 20, 0, 1, fake, fake, fake,
+                               1 << 62, fake, 1 << 62, None) == nq.NQ_ERR_UNSUPPORTED
+    assert L.nq_entropy_decode(fake, fake, fake, 1, 8, 1 << 25, 1, ctypes.byref(pk), 0,
+                               None) == nq.NQ_ERR_INVALID
+    assert L.nq_entropy_decode(None, fake, fake, 1, 8, 64, 1, ctypes.byref(pk), 0,
+                               None) == nq.NQ_ERR_INVALID
     # rope table fill: bad theta, small buffer
     buf = np.zeros(16, np.float32)
     assert L.nq_rope_tables_fill_host(0.5, 10, buf.ctypes.data, 64) == nq.NQ_ERR_INVALID
@@ -135,3 +154,7 @@ def test_empty_work_is_ok_without_device(nq):
     fake = ctypes.c_void_p(0x10000)
     assert L.nq_encode(fake, S, None, S, 0, 8, 64, 64, None, 0, 0, fake, 64, None, None, 0, None) == 0
     assert L.nq_score(fake, S, 0, 8, 64, 64, fake, fake, 0, None) == 0
+    pk = nq.Packed(0x20000, 0x30000, 64, 64, 2)
+    assert L.nq_entropy_encode(ctypes.byref(pk), 0, 8, 64, 0, 1, None, None, None, 0, None, 0,
+                               None) == 0
+    assert L.nq_entropy_decode(None, None, None, 0, 8, 64, 0, ctypes.byref(pk), 0, None) == 0
