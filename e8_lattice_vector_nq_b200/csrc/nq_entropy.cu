@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(128) entropy_count_kernel(const EntArgs a, uin
     __syncthreads();
     const uint32_t* buf = stage[k & 1];
     const int nt = min(kChunk, p.m - k * kChunk);
+#pragma unroll 4
     for (int t = 0; t < nt; ++t) {
       const uint32_t j = code_of<BITS>(buf + t * VW, at);
       const uint32_t s = a.delta ? ((j - prev) & kMask) : j;
@@ -227,6 +228,7 @@ __global__ void __launch_bounds__(128) entropy_encode_kernel(const EntArgs a, co
     __syncthreads();
     const uint32_t* buf = stage[k & 1];
     const int nt = min(kChunk, p.m - k * kChunk);
+#pragma unroll 4
     for (int t = nt - 1; t >= 0; --t) {
       const uint32_t j = code_of<BITS>(buf + t * VW, at);
       if (a.delta) {
@@ -401,6 +403,7 @@ __global__ void __launch_bounds__(128) entropy_decode_kernel(const EntArgs a, co
   uint32_t j = 0;
   for (int k = 0; k < nch; ++k) {
     const int nt = min(kChunk, p.m - k * kChunk);
+#pragma unroll 4
     for (int t = 0; t < nt; ++t) {
       const uint32_t slot = x & (kAnsM - 1u);
       uint32_t s = 0;

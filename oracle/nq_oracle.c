@@ -257,6 +257,24 @@ static uint32_t oq_code(int32_t t, int half, int bits, int *clamped)
     return (uint32_t)((tc + lim) / 2);
 }
 
+/* The b-bit code of coordinate c sits at bits [b*c, b*c + b) of a vector's
+ * little-endian stream of 32-bit words. */
+static uint32_t oq_get_code(const uint32_t *words, int bits, int c)
+{
+    uint32_t j = 0;
+    int bitpos = bits * c;
+    for (int k = 0; k < bits; k++)
+        j |= ((words[(bitpos + k) >> 5] >> ((bitpos + k) & 31)) & 1u) << k;
+    return j;
+}
+
+static void oq_put_code(uint32_t *words, int bits, int c, uint32_t j)
+{
+    int bitpos = bits * c;
+    for (int k = 0; k < bits; k++)
+        if (j & (1u << k)) words[(bitpos + k) >> 5] |= 1u << ((bitpos + k) & 31);
+}
+
 /* --------------------------------------------------------------- encode */
 
 /* Encode one 128-vector (NexusQuant steps 3-5 plus packing):
@@ -300,12 +318,8 @@ int oq_encode_vector(const uint16_t *x, int rope, const float *c, const float *s
         int32_t t[8];
         int half = oq_e8_nearest(y, t, NULL);
         if (half) cmask |= 1u << g;
-        for (int i = 0; i < 8; i++) {
-            uint32_t j = oq_code(t[i], half, bits, &clamped);
-            int bitpos = bits * (8 * g + i);
-            for (int k = 0; k < bits; k++)
-                if (j & (1u << k)) words[(bitpos + k) >> 5] |= 1u << ((bitpos + k) & 31);
-        }
+        for (int i = 0; i < 8; i++)
+            oq_put_code(words, bits, 8 * g + i, oq_code(t[i], half, bits, &clamped));
     }
     *meta = cmask | ((uint32_t)sig16 << 16);
     return clamped;
@@ -325,10 +339,7 @@ void oq_reconstruct_vector(const uint32_t *words, uint32_t meta, int rope, const
                            const float *s, int bits, float *w)
 {
     for (int cidx = 0; cidx < OQ_D; cidx++) {
-        uint32_t j = 0;
-        int bitpos = bits * cidx;
-        for (int k = 0; k < bits; k++)
-            j |= ((words[(bitpos + k) >> 5] >> ((bitpos + k) & 31)) & 1u) << k;
+        uint32_t j = oq_get_code(words, bits, cidx);
         int h = (meta >> (cidx >> 3)) & 1u;
         int32_t t = 2 * (int32_t)j - (1 << bits) + 2 - h;
         w[cidx] = (float)t;
@@ -723,22 +734,6 @@ int64_t oq_ans_decode(const uint16_t *in, int64_t len, const uint16_t *F, int A,
         }
     }
     return i;
-}
-
-static uint32_t oq_get_code(const uint32_t *words, int bits, int c)
-{
-    uint32_t j = 0;
-    int bitpos = bits * c;
-    for (int k = 0; k < bits; k++)
-        j |= ((words[(bitpos + k) >> 5] >> ((bitpos + k) & 31)) & 1u) << k;
-    return j;
-}
-
-static void oq_put_code(uint32_t *words, int bits, int c, uint32_t j)
-{
-    int bitpos = bits * c;
-    for (int k = 0; k < bits; k++)
-        if (j & (1u << k)) words[(bitpos + k) >> 5] |= 1u << ((bitpos + k) & 31);
 }
 
 /* Symbols of the stream (segment g, coordinate c) of one (unit, head):
