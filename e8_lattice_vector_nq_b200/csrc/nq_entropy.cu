@@ -28,12 +28,12 @@
 // move between HBM and shared memory in chunks of 64 tokens (16-byte cp.async
 // loads, 16-byte stores), so the 32 lanes of a warp read a token's words with
 // one broadcast LDS and, decoding, build them back with one warp
-// OR-reduction per word.  Encode passes: count
-// (16-bit field counters in two 64-bit registers per thread, warp sums, one
-// atomic per symbol and warp), table (a thread per (unit, head)), encode into
-// fixed slots of kSeg + 2 words per stream in the workspace (a step emits at
-// most one word), an exclusive scan of the stream lengths (tile sums, their
-// scan, per-tile scans), and a copy to the dense output (a warp per stream).  The division by F_s uses
+// OR-reduction per word.  Encode passes: count (per-lane counters in shared
+// memory, warp sums, one atomic per symbol and warp), table (a thread per
+// (unit, head)), encode into fixed slots of kSeg + 2 words per stream in the
+// workspace (a step emits at most one word), an exclusive scan of the stream
+// lengths (tile sums, their scan, per-tile scans), and a copy to the dense
+// output (a warp per stream).  The division by F_s uses
 // floor(x * floor(2^32 / F_s) / 2^32), which is floor(x / F_s) or one less,
 // and one correction step.
 #include "nq_internal.h"
@@ -112,14 +112,17 @@ __global__ void __launch_bounds__(128) entropy_count_kernel(const EntArgs a, uin
   constexpr int VW = 4 * BITS;
   constexpr uint32_t kMask = A - 1;
   __shared__ __align__(16) uint32_t stage[2][kChunk * VW];
-  const int c = threadIdx.x, lane = c & 31;
+  __shared__ uint32_t cnt[4][A][32];  // per warp, symbol and lane: the bank is the lane
+  const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
   const StreamPos p = stream_pos(a);
   const CodeAt at = code_at<BITS>(c);
   const uint32_t* seg = a.codes + p.vec0 * VW;
   const int nch = (p.m + kChunk - 1) / kChunk;
   issue_chunk<BITS>(smem_u32(stage[0]), seg, 0, p.m, c);
   cp_async_commit();
-  uint64_t lo = 0, hi = 0;  // 16-bit counters: symbols 0-3 in lo, 4-7 in hi
+  uint32_t* my = &cnt[warp][0][lane];  // this thread's counter of symbol s: my[32 s]
+#pragma unroll
+  for (int s = 0; s < A; ++s) my[32 * s] = 0;
   uint32_t prev = 0;
   for (int k = 0; k < nch; ++k) {
     if (k + 1 < nch) issue_chunk<BITS>(smem_u32(stage[(k + 1) & 1]), seg, k + 1, p.m, c);
@@ -133,16 +136,13 @@ __global__ void __launch_bounds__(128) entropy_count_kernel(const EntArgs a, uin
       const uint32_t j = code_of<BITS>(buf + t * VW, at);
       const uint32_t s = a.delta ? ((j - prev) & kMask) : j;
       prev = j;
-      const uint64_t inc = 1ull << (16 * (s & 3u));
-      if (s < 4) lo += inc;
-      else hi += inc;
+      my[32 * s] += 1u;
     }
     __syncthreads();  // the buffer is refilled next iteration
   }
 #pragma unroll
   for (int s = 0; s < A; ++s) {
-    const uint32_t v = static_cast<uint32_t>(((s < 4 ? lo : hi) >> (16 * (s & 3))) & 0xFFFFu);
-    const uint32_t sum = __reduce_add_sync(0xffffffffu, v);
+    const uint32_t sum = __reduce_add_sync(0xffffffffu, my[32 * s]);
     if (lane == 0 && sum) atomicAdd(counts + p.uh * 8 + s, sum);
   }
 }
@@ -361,6 +361,7 @@ __global__ void __launch_bounds__(256) entropy_compact_kernel(const uint16_t* sc
   const uint32_t len = sizes[s];
   const uint16_t* src = scratch + s * kCap + (kCap - len);
   uint16_t* dst = words + offsets[s];
+#pragma unroll 4
   for (uint32_t i = lane; i < len; i += 32) dst[i] = src[i];
 }
 
