@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mistral7b_32k")
     ap.add_argument("--e2e-steps", type=int, default=2)
-    ap.add_argument("--e2e-chunk", type=int, default=2, help="layers per pipelined chunk (e2e)")
+    ap.add_argument("--e2e-chunk", type=int, default=1, help="layers per pipelined chunk (e2e)")
     ap.add_argument("--cpu-layers", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -610,11 +610,62 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     e.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, world, K.device)
-    return {"value": world * in_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
-            "h2d_bytes_per_step": rt.h2d_bytes(Kh, Vh),
+    link = link_rates(Kh, K, Kd, Koh)
+    h2d = rt.h2d_bytes(Kh, Vh)
+    bound = in_bytes / (h2d / (link["h2d_gbs"] * 1e9)) / 1e9  # GB/s of KV in, H2D-bound
+    value = world * in_bytes / (ms * 1e-3) / 1e9
+    return {"value": value, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": Kd.numel() * 2 + Vd.numel() * 2,
             "ms_per_step": ms, "steps": args.e2e_steps, "chunk_layers": args.e2e_chunk,
-            "values_read_in_place": rt.values_in_place}
+            "values_read_in_place": rt.values_in_place, "link": link,
+            "h2d_bound_gbs": world * bound, "frac_of_h2d_bound": value / (world * bound)}
+
+
+def link_rates(Kh, K, Kd, Koh, reps: int = 3):
+    """Pinned copy rates of this GPU's host link with the run's own buffers:
+    host-to-device (Kh -> K), device-to-host (Kd -> Koh) and both at once on
+    two streams with equal byte counts (aggregate).  CUDA events on the
+    current stream, which joins the two copy streams before the stop event."""
+    dev = K.device
+    s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+
+    def h2d():
+        s1.wait_stream(cur)
+        with torch.cuda.stream(s1):
+            K.copy_(Kh, non_blocking=True)
+
+    def d2h():
+        s2.wait_stream(cur)
+        with torch.cuda.stream(s2):
+            Koh.copy_(Kd, non_blocking=True)
+
+    m = Kd.numel()  # equal byte counts both ways for the duplex figure
+    Kh_m, K_m = Kh.view(-1)[:m], K.view(-1)[:m]
+
+    def both():
+        s1.wait_stream(cur)
+        with torch.cuda.stream(s1):
+            K_m.copy_(Kh_m, non_blocking=True)
+        d2h()
+
+    def t(fn):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(cur)
+        for _ in range(reps):
+            fn()
+        cur.wait_stream(s1)
+        cur.wait_stream(s2)
+        b.record(cur)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e-3
+
+    nh, nd = Kh.numel() * Kh.element_size(), Kd.numel() * Kd.element_size()
+    return {"h2d_gbs": nh / t(h2d) / 1e9, "d2h_gbs": nd / t(d2h) / 1e9,
+            "both_ways_gbs": 2 * nd / t(both) / 1e9}
 
 
 def main():
