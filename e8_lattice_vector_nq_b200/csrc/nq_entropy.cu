@@ -33,7 +33,8 @@
 // (unit, head)), encode into fixed slots of kSeg + 2 words per stream in the
 // workspace (a step emits at most one word), an exclusive scan of the stream
 // lengths (tile sums, their scan, per-tile scans), and a copy to the dense
-// output (a warp per stream).  The division by F_s uses
+// output (a warp per stream).  Decoding looks the symbol of a slot up in a
+// per-CTA table of 4096 16-bit entries (s | F_s << 3).  The division by F_s uses
 // floor(x * floor(2^32 / F_s) / 2^32), which is floor(x / F_s) or one less,
 // and one correction step.
 #include "nq_internal.h"
@@ -195,16 +196,14 @@ __global__ void __launch_bounds__(128) entropy_encode_kernel(const EntArgs a, co
   constexpr int VW = 4 * BITS;
   constexpr uint32_t kMask = A - 1;
   __shared__ __align__(16) uint32_t stage[2][kChunk * VW];
-  __shared__ uint32_t fc[A];   // F << 16 | C
-  __shared__ uint32_t rcp[A];  // floor(2^32 / F) for F >= 2
+  __shared__ uint2 sym_tab[A];  // (F << 16 | C, floor(2^32 / F) for F >= 2): one 64-bit load
   const int c = threadIdx.x;
   const StreamPos p = stream_pos(a);
   if (c == 0) {
     uint32_t C = 0;
     for (int s = 0; s < A; ++s) {
       const uint32_t F = freq[p.uh * A + s];
-      fc[s] = (F << 16) | C;
-      rcp[s] = F > 1 ? static_cast<uint32_t>(0x100000000ull / F) : 0u;
+      sym_tab[s] = make_uint2((F << 16) | C, F > 1 ? static_cast<uint32_t>(0x100000000ull / F) : 0u);
       C += F;
     }
   }
@@ -233,17 +232,18 @@ __global__ void __launch_bounds__(128) entropy_encode_kernel(const EntArgs a, co
       const uint32_t j = code_of<BITS>(buf + t * VW, at);
       if (a.delta) {
         if (k * kChunk + t < p.m - 1) {
-          const uint32_t s = (jn - j) & kMask;
-          x = ans_put(x, fc[s], rcp[s], out, pos);
+          const uint2 e = sym_tab[(jn - j) & kMask];
+          x = ans_put(x, e.x, e.y, out, pos);
         }
         jn = j;
       } else {
-        x = ans_put(x, fc[j], rcp[j], out, pos);
+        const uint2 e = sym_tab[j];
+        x = ans_put(x, e.x, e.y, out, pos);
       }
     }
     __syncthreads();  // the buffer is refilled next iteration
   }
-  if (a.delta) x = ans_put(x, fc[jn], rcp[jn], out, pos);
+  if (a.delta) x = ans_put(x, sym_tab[jn].x, sym_tab[jn].y, out, pos);
   out[--pos] = static_cast<uint16_t>(x >> 16);
   out[--pos] = static_cast<uint16_t>(x & 0xFFFFu);
   sizes[stream] = static_cast<uint32_t>(kCap - pos);
@@ -373,7 +373,8 @@ __global__ void __launch_bounds__(128) entropy_decode_kernel(const EntArgs a, co
   constexpr int VW = 4 * BITS;
   constexpr uint32_t kMask = A - 1;
   __shared__ __align__(16) uint32_t stage[kChunk * VW];
-  __shared__ uint32_t fc[A];  // F << 16 | C
+  __shared__ uint32_t fc[A];             // F << 16 | C
+  __shared__ uint16_t slot_tab[kAnsM];   // slot -> s | F_s << 3 (the symbol whose range holds it)
   const int c = threadIdx.x, lane = c & 31, blk32 = c >> 5;
   const StreamPos p = stream_pos(a);
   if (c == 0) {
@@ -385,9 +386,20 @@ __global__ void __launch_bounds__(128) entropy_decode_kernel(const EntArgs a, co
     }
   }
   __syncthreads();
-  uint32_t cum[A];  // C_1 .. C_{A-1} (cum[0] unused)
+  {
+    uint32_t cum[A];  // C_1 .. C_{A-1} (cum[0] unused)
 #pragma unroll
-  for (int s = 0; s < A; ++s) cum[s] = fc[s] & 0xFFFFu;
+    for (int s = 0; s < A; ++s) cum[s] = fc[s] & 0xFFFFu;
+    // thread c fills slots 32c .. 32c+31: s = the number of C_q <= slot, q >= 1
+    for (int q = 0; q < static_cast<int>(kAnsM) / 128; ++q) {
+      const uint32_t slot = static_cast<uint32_t>(c) * (kAnsM / 128) + q;
+      uint32_t s = 0;
+#pragma unroll
+      for (int k = 1; k < A; ++k) s += slot >= cum[k] ? 1u : 0u;
+      slot_tab[slot] = static_cast<uint16_t>(s | ((fc[s] >> 16) << 3));
+    }
+  }
+  __syncthreads();
   const int64_t stream = static_cast<int64_t>(blockIdx.x) * 128 + c;
   const uint32_t o0 = offsets[stream];
   const uint32_t len = offsets[stream + 1] - o0;
@@ -407,11 +419,9 @@ __global__ void __launch_bounds__(128) entropy_decode_kernel(const EntArgs a, co
 #pragma unroll 4
     for (int t = 0; t < nt; ++t) {
       const uint32_t slot = x & (kAnsM - 1u);
-      uint32_t s = 0;
-#pragma unroll
-      for (int q = 1; q < A; ++q) s += slot >= cum[q] ? 1u : 0u;
-      const uint32_t e = fc[s];
-      x = (e >> 16) * (x >> 12) + slot - (e & 0xFFFFu);
+      const uint32_t e = slot_tab[slot];
+      const uint32_t s = e & 7u;
+      x = (e >> 3) * (x >> 12) + slot - (fc[s] & 0xFFFFu);
       if (x < kAnsL) {
         x = (x << 16) | nxt;
         nxt = i < len ? in[i] : 0u;
