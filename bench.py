@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--no-attend", action="store_true", help="skip the decode-attention timing")
     ap.add_argument("--no-entropy", action="store_true",
                     help="skip the delta + entropy stage timing")
+    ap.add_argument("--layerwise", action="store_true",
+                    help="also time score -> select -> encode layer by layer (keys stay in L2 "
+                         "between score and encode) against the all-layer calls")
     ap.add_argument("--layers", type=int, default=0, help="override layer count (small runs)")
     ap.add_argument("--tokens", type=int, default=0, help="override token count (small runs)")
     return ap.parse_args()
@@ -462,6 +465,8 @@ def run_ours(args, world, rank, local):
 
     if not args.no_attend:
         line["decode_attention"] = attend_timing(args, codec, Kd, Vd, stream, world)
+    if args.layerwise:
+        line["layerwise_encode"] = layerwise_timing(codec, K, V, stream, world)
     if not args.no_entropy:
         line["entropy_stage"] = entropy_timing(args, codec, stream, world,
                                                K.numel() + V.numel())
@@ -523,6 +528,33 @@ def attend_timing(args, codec, Kd, Vd, stream, world, G: int = 4):
             "fused_ms": f_ms, "decode_then_sdpa_ms": u_ms, "sdpa_on_bf16_ms": s_ms,
             "speedup_vs_decode_then_sdpa": u_ms / f_ms,
             "fused_packed_read_gbs": packed / (f_ms * 1e-3) / 1e9}
+
+
+def layerwise_timing(codec, K, V, stream, world, reps: int = 10):
+    """score -> select -> encode over all layers in one call each, against the
+    same calls one layer at a time (the order in which a layer's keys are still
+    in L2 when encode re-reads the kept rows).  CUDA events, max over ranks."""
+
+    def batched():
+        codec.encode(K, V, stream)
+
+    def per_layer():
+        for l in range(codec.units):
+            codec.encode(K, V, stream, units=slice(l, l + 1))
+
+    def t(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) / reps, world, K.device)
+
+    return {"all_layers_ms": t(batched), "layer_by_layer_ms": t(per_layer)}
 
 
 def entropy_timing(args, codec, stream, world, total_elems):
