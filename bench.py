@@ -435,7 +435,9 @@ def run_ours(args, world, rank, local):
     achieved = alg[dom] / (per_stage[dom] * 1e-3) / 1e9
     kernel_name = {"score": "score_kernel", "select": "select_kernel", "encode": "encode_kernel",
                    "decode": "decode_kernel"}[dom]
-    traffic = recorded_traffic(kernel_name, wl.name)
+    # the recorded figure belongs to the named workload at its full size only
+    full_size = wl == synth.WORKLOADS[args.workload]
+    traffic = recorded_traffic(kernel_name, wl.name) if full_size else None
 
     enc_ms = sum(per_stage[s] for s in stages if s != "decode")
     out_bytes = Kd.numel() * 2 + Vd.numel() * 2

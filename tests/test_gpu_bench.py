@@ -1,0 +1,66 @@
+"""bench.py's JSON line on a small cache (2 layers of the Mistral-shaped
+workload): every key the benchmark contract asks for is present and
+consistent, and the optional blocks (attention, entropy, layer-by-layer
+encode) run."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def line():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    res = subprocess.run([sys.executable, "bench.py", "--layers", "2", "--steps", "3", "--warmup",
+                          "3", "--e2e-steps", "1", "--cpu-layers", "1", "--layerwise"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [x for x in res.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, res.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_contract_keys(line):
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "roofline", "cpu_baseline", "e2e", "clocks", "gpu_launches"):
+        assert k in line, k
+    assert line["n_gpus"] == 1 and line["steps"] == 3 and line["warmup"] == 3
+    assert line["higher_is_better"] is True and line["scaling"] == "weak"
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    assert line["config"]["workload"] == "mistral7b_32k" and line["config"]["layers"] == 2
+    assert line["gpu_launches"] == 3 * 7
+
+
+def test_roofline_and_baselines(line):
+    r = line["roofline"]
+    assert r["bound"] in ("hbm", "tensor", "alu") and r["unit"] == "GB/s"
+    assert 0 < r["achieved"] and 0 < r["peak"]
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    assert r["traffic"] is None  # recorded for the full 32-layer launch only
+    c = line["cpu_baseline"]
+    assert c["kind"] == "oracle" and c["cores"] >= 1 and c["value"] > 0 and c["sample"]
+    e = line["e2e"]
+    assert e["value"] > 0 and e["unit"] == line["unit"]
+    assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    assert e["link"]["h2d_gbs"] > 0 and 0 < e["frac_of_h2d_bound"] <= 1.5
+    assert line["clocks"]["sm_mhz"] > 0 and isinstance(line["clocks"]["reasons"], list)
+
+
+def test_optional_blocks(line):
+    a = line["decode_attention"]
+    assert a["fused_ms"] > 0 and a["decode_then_sdpa_ms"] > 0
+    for mode in ("delta", "plain"):
+        s = line["entropy_stage"][mode]
+        assert s["round_trip_exact"] is True
+        assert 0 < s["codes_bits_per_elem_coded"] < 4
+    w = line["layerwise_encode"]
+    assert w["all_layers_ms"] > 0 and w["layer_by_layer_ms"] > 0
