@@ -137,6 +137,9 @@ class ClockSampler:
             reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
                 pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
             self._stop = threading.Event()
+            # one sample now, so that even a sub-millisecond region has one
+            self.samples.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                 int(reasons_fn(h))))
 
             def run():
                 while not self._stop.is_set():
