@@ -451,15 +451,16 @@ class Codec:
 
 class HostRoundTrip:
     """Compress a cache that lives in pinned host memory and write its
-    reconstruction back to pinned host memory, in chunks of units on three
-    streams: the host-to-device copy of chunk c+1, the kernels of chunk c and
-    the device-to-host copy of chunk c-1 run at the same time (the two copy
+    reconstruction back to pinned host memory, in chunks of units (one by
+    default: the finest pipeline measured fastest) on three streams: the
+    host-to-device copy of chunk c+1, the kernels of chunk c and the
+    device-to-host copy of chunk c-1 run at the same time (the two copy
     directions share nothing on a full-duplex link).  The device tensors are
     the codec's working copies; every run() is asynchronous on the caller's
     current stream, which afterwards waits for the last copy."""
 
     def __init__(self, codec: Codec, K: torch.Tensor, V: torch.Tensor, K_out: torch.Tensor,
-                 V_out: torch.Tensor, chunk_units: int = 4, values_in_place: bool | None = None):
+                 V_out: torch.Tensor, chunk_units: int = 1, values_in_place: bool | None = None):
         self.codec, self.K, self.V, self.K_out, self.V_out = codec, K, V, K_out, V_out
         # With eviction only the kept value rows are needed: the encode kernel
         # reads them straight from the pinned host cache, so the rows it drops
