@@ -148,3 +148,25 @@ def test_rope_undo_recovers_prerope_keys(oq):
         # plus fp32 table error
         tol = 2.0 ** -8 * np.abs(pre[h]).max(-1, keepdims=True) + 1e-5
         assert np.all(np.abs(u - pre[h]) <= tol)
+
+
+def test_hadamard_spreads_outlier_channels(oq):
+    """The rotation spreads outliers ([NQ-pt] step 4: an outlier would otherwise
+    dominate the scale): on keys with 4 of 128 channels scaled x8 (the
+    synthetic generator's outlier channels), the absmax-to-RMS ratio of each
+    vector drops after the normalised Walsh-Hadamard transform.  The transform
+    is orthogonal up to its 1/sqrt(128), so the RMS is unchanged and only the
+    peak falls."""
+    wl = synth.WORKLOADS["tiny"]
+    pre = synth.gen_prerope_keys(wl, 0, "cpu", tokens=256).numpy().reshape(-1, 128)
+    x = pre.astype(np.float32)
+    y = oq.fwht(x) / np.float32(np.sqrt(128.0))
+
+    def peak_to_rms(a):
+        return np.abs(a).max(-1) / np.sqrt((a.astype(np.float64) ** 2).mean(-1))
+
+    before, after = peak_to_rms(x), peak_to_rms(y)
+    assert np.allclose(np.sqrt((y.astype(np.float64) ** 2).mean(-1)),
+                       np.sqrt((x.astype(np.float64) ** 2).mean(-1)), rtol=1e-5)
+    assert np.median(before) > 1.5 * np.median(after)
+    assert np.mean(after < before) > 0.95
