@@ -470,6 +470,7 @@ def run_ours(args, world, rank, local):
 
     if not args.no_attend:
         line["decode_attention"] = attend_timing(args, codec, Kd, Vd, stream, world)
+    line["reconstruction"] = reconstruction_quality(K, V, Kd, Vd, codec)
     if args.layerwise:
         line["layerwise_encode"] = layerwise_timing(codec, K, V, stream, world)
     if not args.no_entropy:
@@ -533,6 +534,26 @@ def attend_timing(args, codec, Kd, Vd, stream, world, G: int = 4):
             "fused_ms": f_ms, "decode_then_sdpa_ms": u_ms, "sdpa_on_bf16_ms": s_ms,
             "speedup_vs_decode_then_sdpa": u_ms / f_ms,
             "fused_packed_read_gbs": packed / (f_ms * 1e-3) / 1e9}
+
+
+def reconstruction_quality(K, V, Kd, Vd, codec, layers=(0, 15, 31)):
+    """Diagnostic (outside the timed region): the decoded cache against its
+    input rows (the kept ones), per vector: mean cosine similarity and mean
+    relative L2 error, on a few layers.  Keys are compared with RoPE applied on
+    both sides (the decoder re-applies it)."""
+    import torch.nn.functional as F
+
+    sample = [l for l in layers if l < codec.units]
+    res = {"layers_sampled": sample}
+    for name, X, Xd in (("k", K, Kd), ("v", V, Vd)):
+        cos, rel = [], []
+        for l in sample:
+            x = X[l] if codec.kept is None else X[l][:, codec.kept[l].long()]
+            x, xd = x.float(), Xd[l].float()
+            cos.append(F.cosine_similarity(x, xd, dim=-1).mean().item())
+            rel.append(((x - xd).norm(dim=-1) / x.norm(dim=-1).clamp_min(1e-30)).mean().item())
+        res[name] = {"cosine_mean": sum(cos) / len(cos), "rel_l2_mean": sum(rel) / len(rel)}
+    return res
 
 
 def layerwise_timing(codec, K, V, stream, world, reps: int = 10):
