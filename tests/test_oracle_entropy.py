@@ -12,9 +12,12 @@ static table, so the pins come from its definition and from arithmetic:
   bits, so 16 * words <= sum_t log2(M / F_{s_t}) + n log2(17/16) + 32;
 * a stream of one symbol with F = M never changes the state (closed form);
 * round trips, and a numpy restatement of the stream layout (segments,
-  coordinate order, differences mod 2^b) and of the per-(unit, head) counts.
+  coordinate order, differences mod 2^b) and of the per-(unit, head) counts;
+* streams worked out by hand from the coder's definition
+  (tests/golden/rans_examples.txt).
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -180,3 +183,27 @@ def test_differences_pay_off_on_correlated_codes():
     _, _, w_delta = oq.entropy_encode_store(codes, 3, True)
     _, _, w_plain = oq.entropy_encode_store(codes, 3, False)
     assert w_delta.size < 0.5 * w_plain.size
+
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "rans_examples.txt")
+
+
+def load_rans_golden():
+    rows = []
+    for line in open(GOLDEN):
+        line = line.split("#", 1)[0].strip()
+        if not line:
+            continue
+        f, s, w = (part.split() for part in line.split("|"))
+        rows.append((np.array(f, np.uint16), np.array(s, np.uint8), [int(x) for x in w]))
+    return rows
+
+
+def test_hand_worked_streams():
+    rows = load_rans_golden()
+    assert len(rows) == 3
+    for F, sym, words in rows:
+        w = oq.ans_encode(sym, F)
+        assert w.tolist() == words
+        back, used = oq.ans_decode(np.array(words, np.uint16), F, sym.size)
+        assert used == len(words) and np.array_equal(back, sym)
