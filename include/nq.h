@@ -7,7 +7,8 @@
  *            (zingnex.cn), sections "Token eviction", "E8 lattice
  *            quantisation", "Implementation details";
  *   [NQ-pt]  "Como comprimir o KV cache do seu LLM em 33x sem treino"
- *            (dev.to), section "Como funciona (em 6 passos)", steps 1-5.
+ *            (dev.to), section "Como funciona (em 6 passos)", steps 1-6
+ *            (step 6, the coding of the lattice indices: nq_entropy_*).
  * The pages give no formulas or code; the concrete arithmetic below (fp32
  * operation order, tie rules, scale rule, packed layout) is this library's
  * reading and is restated next to each call.
@@ -229,9 +230,10 @@ nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int
  *                                          positions[u*pos_stride + t] : t))
  *     out[u][j] = sum_t softmax(s)_t v_t   v_t: the fp32 value before bf16
  *     lse[u][j] = log(sum_t exp(s_t))      (natural log; lse may be NULL)
- * fp32 arithmetic in the kernels' own order (scores, fp32 exp, chunked
- * sums), so results agree with an exact evaluation to about 1e-5 relative,
- * not bit for bit.  q: fp32 [units][heads*G][128], 16-byte aligned.
+ * fp32 arithmetic in the kernels' own order (scores, fp32 exp, a running
+ * max and sum over tiles of 16 tokens within each chunk, chunks merged at
+ * the end), so results agree with an exact evaluation to about 1e-5
+ * relative, not bit for bit.  q: fp32 [units][heads*G][128], 16-byte aligned.
  * out: fp32 [units][heads*G][128].  k_in/v_in: packed stores as for
  * nq_decode (any bits 2/3).  1 <= G <= 8, 1 <= n < 2^31 (larger n returns
  * NQ_ERR_UNSUPPORTED).  ws: device workspace of
