@@ -77,10 +77,18 @@ ENCODE_SOURCES = ("e8_lattice_vector_nq_b200/csrc/nq_codec.cu",
 
 
 def kernel_source_hash() -> str:
+    """Hash of the encode kernel's sources with comments and whitespace
+    removed, so that only a change of code (not of its documentation) retires
+    a recorded traffic figure."""
+    import re
+
     h = hashlib.sha256()
     for f in ENCODE_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:12]
 
 
