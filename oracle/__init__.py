@@ -78,6 +78,9 @@ def _load():
             "oq_rope_apply_batch": (None, [P, P, P, i64, i32]),
             "oq_encode_batch": (i64, [P, i64, i32, P, P, i32, P, P]),
             "oq_decode_batch": (None, [P, P, i64, i32, P, P, i32, P]),
+            "oq_e8_box_code_batch": (None, [P, i64, i32, P, P, P]),
+            "oq_exact_pack_group": (ctypes.c_uint32, [P, i32, i32]),
+            "oq_exact_unpack_group": (None, [ctypes.c_uint32, i32, P, P]),
             "oq_ans_table": (None, [P, i32, P]),
             "oq_ans_encode": (i64, [P, i64, P, i32, P, i64]),
             "oq_ans_decode": (i64, [P, i64, P, i32, P, i64]),
@@ -375,3 +378,31 @@ def entropy_decode_store(words, offsets, freq, units: int, heads: int, n: int, b
     if rc != 0:
         raise ValueError("oq_entropy_decode_store: inconsistent stream")
     return codes
+
+
+# ------------------------------------------- E8 within the code box (exact packing)
+def e8_box_codes(y, bits: int):
+    """Box-constrained nearest E8 points of [n][8] fp32 groups: (codes uint32
+    [n] with code i at bits [b i, b i + b), coset int32 [n], distance fp32 [n])."""
+    y = np.ascontiguousarray(y, dtype=np.float32).reshape(-1, 8)
+    n = y.shape[0]
+    codes = np.empty(n, np.uint32)
+    coset = np.empty(n, np.int32)
+    dist = np.empty(n, np.float32)
+    _load().oq_e8_box_code_batch(_p(y), n, bits, _p(codes), _p(coset), _p(dist))
+    return codes, coset, dist
+
+
+def exact_pack(j8, half: int, bits: int) -> int:
+    """One group's 8 codes and coset bit in 8*bits bits (coset in the low bit of j_7)."""
+    j = np.ascontiguousarray(j8, dtype=np.uint32)
+    return int(_load().oq_exact_pack_group(_p(j), int(half), bits))
+
+
+def exact_unpack(w: int, bits: int):
+    """Inverse of exact_pack: (codes uint32 [8], coset)."""
+    j = np.empty(8, np.uint32)
+    h = ctypes.c_int(0)
+    _load().oq_exact_unpack_group(ctypes.c_uint32(w), bits, _p(j), ctypes.byref(h))
+    return j, h.value
+

@@ -245,6 +245,120 @@ int oq_e8_nearest(const float *y, int32_t *t, float *dist)
     return 0;
 }
 
+/* ---------------------------------------------- E8 within the code box
+ * The nearest point of E8 restricted to the b-bit code box, this library's
+ * parity-preserving reading of the clamp, which the exact (coset bit folded)
+ * packing below needs.  The pages give no clamp rule; the encoder's own rule
+ * (nearest E8 point, then each 2q clamped) can leave E8 when it clamps.
+ * Box: the integer coset q in [-(2^(b-1) - 1), 2^(b-1) - 1], the half coset
+ * q in [-(2^(b-1) - 1/2), 2^(b-1) - 1/2] (the code ranges of oq_code).
+ * Per coset (shift 0 or 1/2, f = q - shift integers in [lo, hi]): each
+ * coordinate takes f = clamp(rint(u), lo, hi) (u = y - shift, ties to even),
+ * e = u - f; an odd sum of f moves the one coordinate whose move to the
+ * nearest in-range value of the other parity (toward u when that is in
+ * range, else away) costs least, cost (e - dir)^2 - e^2 = 1 - 2 dir e, the
+ * first index on ties.  The costs are separable and non-negative, so this is
+ * the nearest point of the coset inside the box (Conway-Sloane's D8 step
+ * with the box).  Distance: e0^2 then an fmaf chain, plus the move's cost;
+ * the half coset wins only when strictly closer.  When the unconstrained
+ * decoder's point lies in the box, this returns the same point. */
+static float oq_d8_box_decode(const float *y, float shift, int32_t lo, int32_t hi, int32_t *g)
+{
+    float u[8], e[8];
+    int32_t f[8];
+    int32_t sum = 0;
+    for (int i = 0; i < 8; i++) {
+        u[i] = y[i] - shift;
+        int32_t r = (int32_t)rintf(u[i]);
+        f[i] = r < lo ? lo : (r > hi ? hi : r);
+        e[i] = u[i] - (float)f[i];
+        sum += f[i];
+    }
+    float d = e[0] * e[0];
+    for (int i = 1; i < 8; i++) d = fmaf(e[i], e[i], d);
+    if (sum & 1) {
+        int k = -1, kdir = 0;
+        float best = 0.0f;
+        for (int i = 0; i < 8; i++) {
+            int32_t dir = (e[i] >= 0.0f) ? 1 : -1;
+            if (f[i] + dir > hi || f[i] + dir < lo) dir = -dir;
+            float cost = fmaf(-2.0f * (float)dir, e[i], 1.0f);
+            if (k < 0 || cost < best) {
+                best = cost;
+                k = i;
+                kdir = dir;
+            }
+        }
+        f[k] += kdir;
+        d = d + best;
+    }
+    for (int i = 0; i < 8; i++) g[i] = f[i];
+    return d;
+}
+
+/* Box-constrained nearest E8 point: t[i] = 2 q_i; returns the coset (0
+ * integer, 1 half), the fp32 distance in *dist. */
+int oq_e8_box_nearest(const float *y, int bits, int32_t *t, float *dist)
+{
+    int32_t g0[8], g1[8];
+    int32_t h = 1 << (bits - 1);
+    float d0 = oq_d8_box_decode(y, 0.0f, -(h - 1), h - 1, g0);
+    float d1 = oq_d8_box_decode(y, 0.5f, -h, h - 1, g1);
+    if (d1 < d0) {
+        for (int i = 0; i < 8; i++) t[i] = 2 * g1[i] + 1;
+        if (dist) *dist = d1;
+        return 1;
+    }
+    for (int i = 0; i < 8; i++) t[i] = 2 * g0[i];
+    if (dist) *dist = d0;
+    return 0;
+}
+
+/* Exact packing of one group of a box-constrained point.  The codes are
+ * j = q + 2^(b-1) - 1 (integer coset) and j = (q - 1/2) + 2^(b-1) (half
+ * coset); a point of E8 has sum q even (integer coset) or sum (q - 1/2) even
+ * (half coset: D8 + 1/2), so sum j is even in both, the low bit of j_7 is the
+ * parity of j_0 .. j_6, and its place carries the coset bit:
+ * bits [b i, b i + b) hold j_i for i < 7, bit 7b the coset, bits
+ * [7b + 1, 8b) the high bits of j_7. */
+uint32_t oq_exact_pack_group(const uint32_t *j, int half, int bits)
+{
+    uint32_t w = 0;
+    for (int i = 0; i < 7; i++) w |= j[i] << (bits * i);
+    w |= ((j[7] & ~1u) | (uint32_t)(half & 1)) << (7 * bits);
+    return w;
+}
+
+void oq_exact_unpack_group(uint32_t w, int bits, uint32_t *j, int *half)
+{
+    uint32_t mask = (1u << bits) - 1u, par = 0;
+    for (int i = 0; i < 7; i++) {
+        j[i] = (w >> (bits * i)) & mask;
+        par ^= j[i] & 1u;
+    }
+    uint32_t last = (w >> (7 * bits)) & mask;
+    *half = (int)(last & 1u);
+    j[7] = (last & ~1u) | par;
+}
+
+/* Batch: box-constrained codes of n groups of 8 (codes packed plainly, code
+ * i at bits [b i, b i + b)), coset flags and distances. */
+void oq_e8_box_code_batch(const float *y, int64_t n, int bits, uint32_t *codes, int32_t *coset,
+                          float *dist)
+{
+    for (int64_t g = 0; g < n; g++) {
+        int32_t t[8];
+        float d;
+        int half = oq_e8_box_nearest(y + 8 * g, bits, t, &d);
+        int32_t lim = (1 << bits) - (half ? 1 : 2);
+        uint32_t w = 0;
+        for (int i = 0; i < 8; i++) w |= (uint32_t)((t[i] + lim) / 2) << (bits * i);
+        codes[g] = w;
+        coset[g] = half;
+        dist[g] = d;
+    }
+}
+
 /* Clamp 2q to the b-bit symmetric code range and return the code:
  *   half coset (t odd):     t in [-(2^b-1), 2^b-1],  j = (t + 2^b - 1)/2
  *   integer coset (t even): t in [-(2^b-2), 2^b-2],  j = (t + 2^b - 2)/2

@@ -65,6 +65,10 @@ MUTATIONS = [
      "tests/test_oracle_entropy.py::test_round_trip_and_size_bound"),
     ("entropy-delta-reference", "        prev = j;\n", "        prev = 0;\n",
      "tests/test_oracle_entropy.py::test_store_layout_matches_a_numpy_restatement"),
+    ("box-move-direction", "if (f[i] + dir > hi || f[i] + dir < lo) dir = -dir;", ";",
+     "tests/test_oracle_box.py::test_points_are_in_e8_and_in_the_box"),
+    ("exact-unpack-parity", "par ^= j[i] & 1u;", "par ^= j[i] & 0u;",
+     "tests/test_oracle_box.py::test_exact_packing_round_trip"),
 ]
 
 
