@@ -304,14 +304,10 @@ int oq_e8_box_nearest(const float *y, int bits, int32_t *t, float *dist)
     int32_t h = 1 << (bits - 1);
     float d0 = oq_d8_box_decode(y, 0.0f, -(h - 1), h - 1, g0);
     float d1 = oq_d8_box_decode(y, 0.5f, -h, h - 1, g1);
-    if (d1 < d0) {
-        for (int i = 0; i < 8; i++) t[i] = 2 * g1[i] + 1;
-        if (dist) *dist = d1;
-        return 1;
-    }
-    for (int i = 0; i < 8; i++) t[i] = 2 * g0[i];
-    if (dist) *dist = d0;
-    return 0;
+    const int half = d1 < d0; /* the half coset only when strictly closer */
+    for (int i = 0; i < 8; i++) t[i] = half ? 2 * g1[i] + 1 : 2 * g0[i];
+    if (dist) *dist = half ? d1 : d0;
+    return half;
 }
 
 /* Exact packing of one group of a box-constrained point.  The codes are
@@ -350,9 +346,9 @@ void oq_e8_box_code_batch(const float *y, int64_t n, int bits, uint32_t *codes, 
         int32_t t[8];
         float d;
         int half = oq_e8_box_nearest(y + 8 * g, bits, t, &d);
-        int32_t lim = (1 << bits) - (half ? 1 : 2);
+        const int32_t offs = half ? (1 << bits) - 1 : (1 << bits) - 2; /* the code range */
         uint32_t w = 0;
-        for (int i = 0; i < 8; i++) w |= (uint32_t)((t[i] + lim) / 2) << (bits * i);
+        for (int i = 0; i < 8; i++) w |= (uint32_t)((t[i] + offs) / 2) << (bits * i);
         codes[g] = w;
         coset[g] = half;
         dist[g] = d;
