@@ -79,6 +79,9 @@ def _load():
             "oq_encode_batch": (i64, [P, i64, i32, P, P, i32, P, P]),
             "oq_decode_batch": (None, [P, P, i64, i32, P, P, i32, P]),
             "oq_e8_box_code_batch": (None, [P, i64, i32, P, P, P]),
+            "oq_encode_box_batch": (i64, [P, i64, i32, P, P, i32, P, P]),
+            "oq_fold_exact_batch": (None, [P, P, i64, i32, P, P]),
+            "oq_unfold_exact_batch": (None, [P, P, i64, i32, P, P]),
             "oq_exact_pack_group": (ctypes.c_uint32, [P, i32, i32]),
             "oq_exact_unpack_group": (None, [ctypes.c_uint32, i32, P, P]),
             "oq_ans_table": (None, [P, i32, P]),
@@ -405,4 +408,42 @@ def exact_unpack(w: int, bits: int):
     h = ctypes.c_int(0)
     _load().oq_exact_unpack_group(ctypes.c_uint32(w), bits, _p(j), ctypes.byref(h))
     return j, h.value
+
+
+def encode_vectors_box(x_bf16, bits: int, rope: bool = False, c=None, s=None):
+    """Encode [n][128] bf16 vectors with the box-constrained E8 step (regular
+    layout); returns (words [n][4b] u32, meta [n] u32)."""
+    x = _u16(x_bf16).reshape(-1, D)
+    n = x.shape[0]
+    if c is None:
+        c = np.zeros((n, D // 2), np.float32)
+        s = np.zeros((n, D // 2), np.float32)
+    c = np.ascontiguousarray(c, dtype=np.float32).reshape(n, D // 2)
+    s = np.ascontiguousarray(s, dtype=np.float32).reshape(n, D // 2)
+    w = np.empty((n, 4 * bits), np.uint32)
+    m = np.empty(n, np.uint32)
+    _load().oq_encode_box_batch(_p(x), n, int(rope), _p(c), _p(s), bits, _p(w), _p(m))
+    return w, m
+
+
+def fold_exact(words, meta, bits: int):
+    """Regular layout -> exact layout: (words [n][4b] u32, sigma [n] u16)."""
+    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, 4 * bits)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32).ravel()
+    n = words.shape[0]
+    out = np.empty_like(words)
+    sig = np.empty(n, np.uint16)
+    _load().oq_fold_exact_batch(_p(words), _p(meta), n, bits, _p(out), _p(sig))
+    return out, sig
+
+
+def unfold_exact(words, sig16, bits: int):
+    """Exact layout -> regular layout: (words [n][4b] u32, meta [n] u32)."""
+    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, 4 * bits)
+    sig16 = np.ascontiguousarray(sig16, dtype=np.uint16).ravel()
+    n = words.shape[0]
+    out = np.empty_like(words)
+    meta = np.empty(n, np.uint32)
+    _load().oq_unfold_exact_batch(_p(words), _p(sig16), n, bits, _p(out), _p(meta))
+    return out, meta
 

@@ -397,9 +397,11 @@ static void oq_put_code(uint32_t *words, int bits, int c, uint32_t j)
  *  5. pack: the b-bit code of coordinate c sits at bits [b*c, b*c + b) of the
  *     vector's little-endian stream of 4*b 32-bit words; meta word =
  *     coset mask (bit g = group g in the half coset) | fp16(sigma) << 16.
- * Returns the number of clamped coordinates. */
-int oq_encode_vector(const uint16_t *x, int rope, const float *c, const float *s,
-                     int bits, uint32_t *words, uint32_t *meta)
+ * Returns the number of clamped coordinates.  With box set, step 4 takes the
+ * nearest E8 point inside the code box instead (oq_e8_box_nearest; nothing
+ * is clamped then). */
+static int oq_encode_vector_mode(const uint16_t *x, int rope, const float *c, const float *s,
+                                 int bits, int box, uint32_t *words, uint32_t *meta)
 {
     float v[OQ_D];
     for (int i = 0; i < OQ_D; i++) v[i] = oq_bf16_to_f32(x[i]);
@@ -426,13 +428,57 @@ int oq_encode_vector(const uint16_t *x, int rope, const float *c, const float *s
             y[i] = (p == 0.0f) ? 0.0f : p;
         }
         int32_t t[8];
-        int half = oq_e8_nearest(y, t, NULL);
+        int half = box ? oq_e8_box_nearest(y, bits, t, NULL) : oq_e8_nearest(y, t, NULL);
         if (half) cmask |= 1u << g;
         for (int i = 0; i < 8; i++)
             oq_put_code(words, bits, 8 * g + i, oq_code(t[i], half, bits, &clamped));
     }
     *meta = cmask | ((uint32_t)sig16 << 16);
     return clamped;
+}
+
+int oq_encode_vector(const uint16_t *x, int rope, const float *c, const float *s,
+                     int bits, uint32_t *words, uint32_t *meta)
+{
+    return oq_encode_vector_mode(x, rope, c, s, bits, 0, words, meta);
+}
+
+int oq_encode_vector_box(const uint16_t *x, int rope, const float *c, const float *s,
+                         int bits, uint32_t *words, uint32_t *meta)
+{
+    return oq_encode_vector_mode(x, rope, c, s, bits, 1, words, meta);
+}
+
+/* The exact layout of a vector of box-constrained points from the regular one:
+ * group g's codes occupy bits [8b g, 8b g + 8b) of the vector's words in both;
+ * the exact layout holds the coset bit h_g where the regular one holds the low
+ * bit of j_{8g+7} (the parity of j_{8g} .. j_{8g+6} for a point of E8), and of
+ * the meta word it keeps only sigma. */
+void oq_fold_exact(const uint32_t *words, uint32_t meta, int bits, uint32_t *out,
+                   uint16_t *sig16)
+{
+    for (int w = 0; w < 4 * bits; w++) out[w] = words[w];
+    for (int g = 0; g < 16; g++) {
+        int pos = bits * (8 * g + 7);
+        uint32_t h = (meta >> g) & 1u;
+        out[pos >> 5] = (out[pos >> 5] & ~(1u << (pos & 31))) | (h << (pos & 31));
+    }
+    *sig16 = (uint16_t)(meta >> 16);
+}
+
+void oq_unfold_exact(const uint32_t *in, uint16_t sig16, int bits, uint32_t *words,
+                     uint32_t *meta)
+{
+    uint32_t cmask = 0;
+    for (int w = 0; w < 4 * bits; w++) words[w] = in[w];
+    for (int g = 0; g < 16; g++) {
+        int pos = bits * (8 * g + 7);
+        cmask |= ((in[pos >> 5] >> (pos & 31)) & 1u) << g;
+        uint32_t par = 0;
+        for (int i = 0; i < 7; i++) par ^= oq_get_code(words, bits, 8 * g + i) & 1u;
+        words[pos >> 5] = (words[pos >> 5] & ~(1u << (pos & 31))) | (par << (pos & 31));
+    }
+    *meta = cmask | ((uint32_t)sig16 << 16);
 }
 
 /* --------------------------------------------------------------- decode */
@@ -736,6 +782,31 @@ void oq_decode_batch(const uint32_t *words, const uint32_t *meta, int64_t n, int
     for (int64_t i = 0; i < n; i++)
         oq_decode_vector(words + 4 * bits * i, meta[i], rope, c + OQ_HALF * i, s + OQ_HALF * i,
                          bits, out + OQ_D * i);
+}
+
+/* Batches of the box-constrained encoder and of the exact-layout conversions. */
+int64_t oq_encode_box_batch(const uint16_t *x, int64_t n, int rope, const float *c,
+                            const float *s, int bits, uint32_t *words, uint32_t *meta)
+{
+    int64_t clamped = 0;
+    for (int64_t i = 0; i < n; i++)
+        clamped += oq_encode_vector_box(x + OQ_D * i, rope, c + OQ_HALF * i, s + OQ_HALF * i, bits,
+                                        words + 4 * bits * i, meta + i);
+    return clamped;
+}
+
+void oq_fold_exact_batch(const uint32_t *words, const uint32_t *meta, int64_t n, int bits,
+                         uint32_t *out, uint16_t *sig16)
+{
+    for (int64_t i = 0; i < n; i++)
+        oq_fold_exact(words + 4 * bits * i, meta[i], bits, out + 4 * bits * i, sig16 + i);
+}
+
+void oq_unfold_exact_batch(const uint32_t *in, const uint16_t *sig16, int64_t n, int bits,
+                           uint32_t *words, uint32_t *meta)
+{
+    for (int64_t i = 0; i < n; i++)
+        oq_unfold_exact(in + 4 * bits * i, sig16[i], bits, words + 4 * bits * i, meta + i);
 }
 
 /* ------------------------------------------------- delta + entropy stage */

@@ -14,14 +14,19 @@ point of E8 inside the b-bit code box.  Pins from the mathematics:
 * when the unconstrained decoder's point lies inside the box, both agree;
 * the exact packing is a bijection on these points (pack then unpack is the
   identity), and it would lose information for points off E8 (the encoder's
-  clamp), which is why the box rule is needed.
+  clamp), which is why the box rule is needed;
+* at the vector level the box encoder equals the codec wherever the codec
+  clamps nothing, and the exact layout (coset bit folded, sigma alone in the
+  meta) converts to the regular one and back without loss.
 """
 import itertools
 
 import numpy as np
 import pytest
+import torch
 
 import oracle as oq
+from e8_lattice_vector_nq_b200 import synth
 
 
 def unpack_codes(c, bits):
@@ -142,3 +147,44 @@ def test_the_encoder_clamp_can_leave_e8():
     assert broken > 0
     cb, hb, _ = oq.e8_box_codes(y, 3)
     assert all(int(np.sum(unpack_codes(cb[g], 3))) % 2 == 0 for g in range(len(y)))
+
+
+def synthetic_vectors(seed, n):
+    """n synthetic key vectors (bf16 bits, [n][128]) of the tiny workload."""
+    wl = synth.WORKLOADS["tiny"]
+    k, _ = synth.gen_layer(wl, seed % 4, "cpu", tokens=n // 8)
+    return k.contiguous().view(torch.int16).numpy().view(np.uint16).reshape(-1, 128)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_vector_encoder_matches_the_codec_where_nothing_clamps(bits):
+    """Vectors whose regular encode clamps no coordinate: the box encoder gives
+    the same words and meta (the box then contains the decoder's points)."""
+    x = synthetic_vectors(bits, 2048)
+    same = 0
+    for i in range(0, x.shape[0], 64):
+        blk = x[i:i + 64]
+        w0, m0, _ = oq.encode_vectors(blk, bits)
+        w1, m1 = oq.encode_vectors_box(blk, bits)
+        for r in range(blk.shape[0]):
+            _, _, cl = oq.encode_vectors(blk[r:r + 1], bits)
+            if cl == 0:
+                assert np.array_equal(w0[r], w1[r]) and m0[r] == m1[r]
+                same += 1
+    assert same > 100
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_exact_layout_round_trip_and_decode(bits):
+    """fold then unfold restores the box encoder's words and meta; the exact
+    layout differs from the regular one in at most one bit per group; and
+    decoding the unfolded vectors gives the box encoder's reconstruction."""
+    x = synthetic_vectors(10 + bits, 2048)
+    w, m = oq.encode_vectors_box(x, bits)
+    ew, sig = oq.fold_exact(w, m, bits)
+    assert np.array_equal(sig, (m >> 16).astype(np.uint16))
+    diff = np.unpackbits((ew ^ w).view(np.uint8), axis=1).sum(axis=1)
+    assert np.all(diff <= 16)
+    w2, m2 = oq.unfold_exact(ew, sig, bits)
+    assert np.array_equal(w2, w) and np.array_equal(m2, m)
+    assert np.array_equal(oq.decode_vectors(w2, m2, bits), oq.decode_vectors(w, m, bits))
