@@ -188,3 +188,27 @@ def test_exact_layout_round_trip_and_decode(bits):
     w2, m2 = oq.unfold_exact(ew, sig, bits)
     assert np.array_equal(w2, w) and np.array_equal(m2, m)
     assert np.array_equal(oq.decode_vectors(w2, m2, bits), oq.decode_vectors(w, m, bits))
+
+
+@pytest.mark.parametrize("name,bits", [("k", 3), ("v", 2)])
+def test_box_rule_costs_little_reconstruction_error(name, bits):
+    """The price of the parity-preserving clamp: on 2048 tokens of layer 0 of the
+    Mistral-shaped cache the box-constrained points differ from the codec's on
+    about a fifth of the vectors, and the mean relative reconstruction error
+    rises by under 1 % (0.1977 -> 0.1981 for 3-bit keys, 0.5037 -> 0.5051 for
+    2-bit values): the clamped codec point is not bound to E8 and can sit a
+    little closer."""
+    wl = synth.WORKLOADS["mistral7b_32k"]
+    k, v = synth.gen_layer(wl, 0, "cpu", tokens=2048)
+    X = k if name == "k" else v
+    x = X.contiguous().view(torch.int16).numpy().view(np.uint16).reshape(-1, 128)
+    w0, m0, _ = oq.encode_vectors(x, bits)
+    w1, m1 = oq.encode_vectors_box(x, bits)
+    xx = oq.bf16_bits_to_f32(x).astype(np.float64)
+
+    def err(w, m):
+        r = oq.reconstruct_vectors(w, m, bits).astype(np.float64)
+        return np.mean(np.linalg.norm(xx - r, axis=1) / np.linalg.norm(xx, axis=1))
+
+    e_clamp, e_box = err(w0, m0), err(w1, m1)
+    assert e_clamp <= e_box < 1.01 * e_clamp
