@@ -13,7 +13,7 @@ the method description it follows:
   sections "Token eviction", "E8 lattice quantisation", "Implementation
   details";
 * "Como comprimir o KV cache do seu LLM em 33x sem treino" (dev.to), section
-  "Como funciona (em 6 passos)", steps 1-5.
+  "Como funciona (em 6 passos)", steps 1-6.
 
 Parity unpinned: end-to-end model quality (perplexity) -- it needs trained
 models and datasets.  Every other function is pinned by ``tests/test_oracle_*``.

@@ -2,7 +2,9 @@
  * nq_oracle.c -- plain, slow, single-threaded CPU oracle of the NexusQuant
  * KV-cache hot path: key-key token scoring, eviction, RoPE removal, Hadamard
  * rotation, per-vector fp16 scale, E8 lattice quantisation, bit packing and
- * the inverse path.
+ * the inverse path; decode attention on the packed cache; the delta + rANS
+ * coding of the lattice indices; and the nearest E8 point inside the code box
+ * with the exact (coset bit folded) packing.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the CPU
  * baseline of the benchmark may load this file.  It shares no code, header,
@@ -13,7 +15,7 @@
  *     (zingnex.cn, sections "Token eviction", "E8 lattice quantisation",
  *     "Implementation details")
  *   - "Como comprimir o KV cache do seu LLM em 33x sem treino"
- *     (dev.to, section "Como funciona (em 6 passos)", steps 1-5)
+ *     (dev.to, section "Como funciona (em 6 passos)", steps 1-6)
  *
  * The pages leave every formula open; the readings taken (fp32 operation
  * order, tie rules, scale rule, packed layout) are stated next to each
