@@ -2,10 +2,14 @@
 """Benchmark of the KV-cache eviction + E8 lattice codec hot path on B200.
 
 One step = one pass of the whole path over one synthetic KV cache held in
-HBM: key-key scores -> token selection -> E8 encode (K3V2) -> decode back to
-bf16, all layers batched into one call per stage.  Default workload: the
-Mistral-7B-shaped cache (32 layers x 8 KV heads x 32768 tokens x 128, bf16,
-theta 1e6, 60% eviction with BOS + 64-token window), inputs 4.3 GB > L2.
+HBM: key-key scores -> token selection (when the workload evicts) -> E8
+encode -> decode back to bf16, all layers batched into one call per stage.
+Default (headline) workload: the Llama-3-8B-shaped long-context cache (32
+layers x 8 KV heads x 131072 tokens x 128, bf16, theta 5e5, K3V2, no
+eviction: 17.2 GB in, larger than L2), the largest single-GPU workload.  The
+other four workloads (tiny, Mistral-7B-shaped with 60 % eviction, Qwen2.5-7B-
+shaped with protected layers, decode-append) are timed after it and reported
+under "configs", each with the oracle timed beside it.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
 
@@ -38,13 +42,23 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mistral7b_32k")
+    ap.add_argument("--workload", default="llama3_8b_128k")
+    ap.add_argument("--configs", default="all",
+                    help="other workloads timed after the headline and reported under 'configs' "
+                         "(comma list, 'all' or 'none')")
+    ap.add_argument("--config-steps", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--e2e-chunk", type=int, default=1, help="layers per pipelined chunk (e2e)")
-    ap.add_argument("--cpu-layers", type=int, default=2)
+    ap.add_argument("--cpu-tokens", type=int, default=65536,
+                    help="tokens per layer in the timed oracle sample (at most the layer)")
+    ap.add_argument("--cpu-workers", type=int, default=0,
+                    help="worker processes of the all-cores oracle figure (0: every core)")
+    ap.add_argument("--parity-layers", default="0,-1",
+                    help="layers of the headline cache checked against the oracle in the "
+                         "CPU-baseline leg (comma list, negative from the end)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-attend", action="store_true", help="skip the decode-attention timing")
@@ -247,12 +261,12 @@ def max_over_ranks(ms: float, world: int, device=None) -> float:
     return float(t.item())
 
 
-def build_workload(args):
-    wl = synth.WORKLOADS[args.workload]
+def build_workload(args, name=None):
+    wl = synth.WORKLOADS[name or args.workload]
     kw = {}
-    if args.layers:
+    if args.layers and name is None:
         kw["layers"] = args.layers
-    if args.tokens:
+    if args.tokens and name is None:
         kw["tokens"] = args.tokens
     if kw:
         from dataclasses import replace
@@ -273,10 +287,16 @@ def gen_cache(wl, device, layers=None):
     return K, V
 
 
+def vector_bytes(bits):
+    return 4 * 4 * bits + 4  # packed codes + the meta word
+
+
 def algorithmic_bytes(wl, n_kept, units):
+    """DRAM bytes each stage must move per call over `units` layers: the
+    kernels' algorithmic bytes (the bf16 rows read or written, the packed
+    vectors, the kept lists and scores)."""
     H, T = wl.heads, wl.tokens
-    bk = 4 * 4 * wl.bits_k + 4
-    bv = 4 * 4 * wl.bits_v + 4
+    bk, bv = vector_bytes(wl.bits_k), vector_bytes(wl.bits_v)
     evict = wl.evict_pct > 0 and T > 1 + wl.window
     out = {
         "encode": units * (n_kept * H * (256 + 256 + bk + bv) + (n_kept * 4 if evict else 0)),
@@ -288,62 +308,325 @@ def algorithmic_bytes(wl, n_kept, units):
     return out
 
 
-# --------------------------------------------------------------- oracle arm
-def oracle_pass(oq, Kl, Vl, wl):
-    """One layer through the CPU oracle: score, select, encode, decode."""
-    T = Kl.shape[1]
-    evict = wl.evict_pct > 0 and T > 1 + wl.window
-    kept = None
-    n = T
-    if evict:
-        s = oq.score_unit(Kl, wl.window)
-        kept = oq.select(s, wl.window, wl.evict_pct)
-        n = kept.size
-    r = oq.encode_unit(Kl, Vl, n, kept=kept, theta=wl.theta, bits_k=wl.bits_k, bits_v=wl.bits_v)
-    oq.decode_unit(r["k_codes"], r["k_meta"], r["v_codes"], r["v_meta"], positions=kept,
-                   theta=wl.theta, bits_k=wl.bits_k, bits_v=wl.bits_v)
+KERNEL_OF = {"score": "score_kernel", "select": "select_kernel", "encode": "encode_kernel",
+             "decode": "decode_kernel"}
 
 
-def host_layer(wl, layer, device):
-    k, v = synth.gen_layer(wl, layer, device)
-    u16 = lambda t: t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-    return u16(k), u16(v)
+def timed_region(fn, steps, stream, device, world, n_events):
+    """Run fn(events_of_step) for `steps` steps between a barrier and a
+    synchronize on both sides, clocks sampled meanwhile; returns total ms,
+    the per-step event lists and the clock summary."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(steps):
+            fn(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    return start.elapsed_time(end), evs, clk.summary()
 
 
-def cpu_baseline(wl, layers, device, hl=None):
-    import oracle as oq
+def with_remeasure(measure, world, device):
+    """measure() once more if its clock record shows a hardware or thermal
+    slowdown (every rank takes the same decision)."""
+    res = measure()
+    clocks = res[-1]
+    bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+    redo = int(bool(clocks and bad & set(clocks["reasons"])))
+    if world > 1:
+        t = torch.tensor([redo], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        redo = int(t.item())
+    if redo:
+        res = measure()
+        if res[-1] is not None:
+            res[-1]["remeasured"] = True
+    return res
 
-    oq.build()
-    t = 0.0
-    nbytes = 0
-    for l in range(layers):
-        Kl, Vl = hl if hl is not None else host_layer(wl, l, device)
-        t0 = time.perf_counter()
-        oracle_pass(oq, Kl, Vl, wl)
-        t += time.perf_counter() - t0
-        nbytes += Kl.nbytes + Vl.nbytes
-    return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{layers} of {wl.layers} layers ({wl.heads} heads x {wl.tokens} tokens), "
-                      f"score+select+encode+decode, single-threaded C oracle"}
+
+def time_cache(nq, wl, device, steps, warmup, world):
+    """The whole cache through score -> select -> encode -> decode, every
+    layer in one call per stage, timed with CUDA events on the launching
+    stream.  Protected layers (kept in bf16) are not part of the step."""
+    q_layers = wl.quantised_layers
+    units = len(q_layers)
+    K, V = gen_cache(wl, device)
+    Kq, Vq = (K, V) if units == wl.layers else (K[q_layers[0]:q_layers[-1] + 1],
+                                                   V[q_layers[0]:q_layers[-1] + 1])
+    codec = nq.Codec(units, wl.heads, wl.tokens, wl.theta, wl.bits_k, wl.bits_v,
+                     window=wl.window, evict_pct=wl.evict_pct, device=device)
+    n = codec.n
+    Kd = torch.empty(units, wl.heads, n, 128, dtype=torch.bfloat16, device=device)
+    Vd = torch.empty_like(Kd)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        if codec.evict:
+            if ev: ev[0].record(stream)
+            nq.nq_score(Kq, codec.W, codec.scores, codec.ws)
+            if ev: ev[1].record(stream)
+            nq.nq_select(codec.scores, codec.W, codec.pct, codec.kept)
+            if ev: ev[2].record(stream)
+        elif ev:
+            ev[2].record(stream)
+        nq.nq_encode(Kq, Vq, codec.k_store, codec.v_store, n, codec.rope, codec.max_pos,
+                     kept=codec.kept)
+        if ev: ev[3].record(stream)
+        nq.nq_decode(codec.k_store, codec.v_store, n, Kd, Vd, codec.rope, codec.max_pos,
+                     positions=codec.kept)
+        if ev: ev[4].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+
+    def measure():
+        ms, evs, clocks = timed_region(step, steps, stream, device, world, 5)
+        per = {}
+        if codec.evict:
+            per["score"] = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+            per["select"] = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+        per["encode"] = sum(e[2].elapsed_time(e[3]) for e in evs) / steps
+        per["decode"] = sum(e[3].elapsed_time(e[4]) for e in evs) / steps
+        return ms, per, clocks
+
+    ms, per, clocks = with_remeasure(measure, world, device)
+    ms = max_over_ranks(ms, world, device)
+    per = {k: max_over_ranks(v, world, device) for k, v in per.items()}
+    assert nq.device_error() == 0, "a kernel reported an in-kernel failure"
+    return {"K": K, "V": V, "Kq": Kq, "Vq": Vq, "Kd": Kd, "Vd": Vd, "codec": codec,
+            "ms_step": ms / steps, "per_stage": per, "clocks": clocks, "stream": stream,
+            "launches_per_step": (3 if codec.evict else 0) + 4}
+
+
+def figures(wl, t, world, peak, peak_kind, traffic_for=None):
+    """Throughput, stage bandwidths and rooflines of a timed cache."""
+    codec, per, ms_step = t["codec"], t["per_stage"], t["ms_step"]
+    n, units = codec.n, codec.units
+    in_bytes = t["K"].numel() * 2 + t["V"].numel() * 2  # the whole bf16 cache
+    q_in = t["Kq"].numel() * 2 + t["Vq"].numel() * 2
+    alg = algorithmic_bytes(wl, n, units)
+    roof = {}
+    for stage, ms in per.items():
+        ach = alg[stage] / (ms * 1e-3) / 1e9
+        r = {"kernel": KERNEL_OF[stage], "bound": "hbm", "achieved": ach, "peak": peak,
+             "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
+             "frac_of_8tbs_spec": ach / 8000.0, "algorithmic_bytes": alg[stage], "ms": ms}
+        if stage == "select":
+            r["bound"] = "latency"  # a few MB per call: radix passes on cluster barriers
+        roof[stage] = r
+    enc_ms = sum(v for k, v in per.items() if k != "decode")
+    out_bytes = t["Kd"].numel() * 2 + t["Vd"].numel() * 2
+    bits = codec.packed_bytes * 8
+    if units != wl.layers:  # protected layers stay bf16
+        bits += 16 * (in_bytes - q_in) // 2
+    return {
+        "value": world * in_bytes / (ms_step * 1e-3) / 1e9,
+        "ms_per_step": ms_step,
+        "stages_ms": {k: round(v, 4) for k, v in per.items()},
+        "encode_gbs": q_in / (enc_ms * 1e-3) / 1e9,
+        "decode_gbs": out_bytes / (per["decode"] * 1e-3) / 1e9,
+        "tokens_layers_per_s": world * wl.tokens * wl.layers / (ms_step * 1e-3),
+        "bits_per_elem": bits / (in_bytes / 2),
+        "hbm_frac_of_step": (sum(alg.values()) / (ms_step * 1e-3) / 1e9) / peak,
+        "rooflines": roof,
+    }
+
+
+def time_append(nq, wl, device, world, warmup=3):
+    """The decode-append regime: a store of `sequences` x `layers` units of
+    `tokens` encoded tokens (set-up, not timed), then `append_steps` steps,
+    each appending one bf16 token per unit (encode) and reconstructing every
+    token of layer step mod layers for every sequence (decode)."""
+    S, L, H, T0, steps = wl.sequences, wl.layers, wl.heads, wl.tokens, wl.append_steps
+    cap = T0 + steps
+    store = nq.AppendStore(S, L, H, cap, wl.theta, wl.bits_k, wl.bits_v, device=device)
+    for s in range(S):
+        Ks = torch.empty(L, H, T0, 128, dtype=torch.bfloat16, device=device)
+        Vs = torch.empty_like(Ks)
+        for l in range(L):
+            k, v = synth.gen_layer(wl, l, device, seed_offset=1000 * s)
+            Ks[l].copy_(k)
+            Vs[l].copy_(v)
+        store.fill(s, Ks, Vs)
+        del Ks, Vs
+    g = torch.Generator(device=device)
+    g.manual_seed(wl.seed * 1000003)
+    Kn = (torch.randn(steps, S * L, H, 1, 128, generator=g, device=device) * 2).to(torch.bfloat16)
+    Vn = torch.randn(steps, S * L, H, 1, 128, generator=g, device=device).to(torch.bfloat16)
+    Ko = torch.empty(S, H, cap, 128, dtype=torch.bfloat16, device=device)
+    Vo = torch.empty_like(Ko)
+    stream = torch.cuda.current_stream(device)
+
+    def step_at(i, ev=None):
+        pos = T0 + i
+        if ev: ev[0].record(stream)
+        store.append(Kn[i], Vn[i], pos)
+        if ev: ev[1].record(stream)
+        store.decode_layer(i % L, pos + 1, Ko[:, :, :pos + 1], Vo[:, :, :pos + 1])
+        if ev: ev[2].record(stream)
+
+    for _ in range(warmup):  # rewritten by the timed steps
+        step_at(0)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    counter = {"i": 0}
+
+    def one(ev):
+        step_at(counter["i"], ev)
+        counter["i"] += 1
+
+    def measure():
+        counter["i"] = 0
+        ms, evs, clocks = timed_region(one, steps, stream, device, world, 3)
+        enc = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+        dec = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+        return ms, enc, dec, clocks
+
+    ms, enc, dec, clocks = with_remeasure(measure, world, device)
+    ms, enc, dec = (max_over_ranks(x, world, device) for x in (ms, enc, dec))
+    assert nq.device_error() == 0, "a kernel reported an in-kernel failure"
+    ms_step = ms / steps
+    bk, bv = vector_bytes(wl.bits_k), vector_bytes(wl.bits_v)
+    app_units = S * L * H  # vectors appended per step (keys and values each)
+    in_b = app_units * 256 * 2
+    # decoded per step: every token of one layer for every sequence (mean n over the steps)
+    n_mean = T0 + (steps + 1) / 2
+    out_b = S * H * n_mean * 256 * 2
+    enc_alg = app_units * (512 + bk + bv)
+    dec_alg = S * H * n_mean * (bk + bv + 512)
+    peak, peak_kind = measured_peaks()
+    roof = {}
+    for stage, alg, sms in (("encode", enc_alg, enc), ("decode", dec_alg, dec)):
+        ach = alg / (sms * 1e-3) / 1e9
+        roof[stage] = {"kernel": KERNEL_OF[stage], "bound": "hbm", "achieved": ach, "peak": peak,
+                       "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
+                       "frac_of_8tbs_spec": ach / 8000.0, "algorithmic_bytes": alg, "ms": sms}
+    roof["encode"]["bound"] = "latency"  # 16 384 vectors per append: one short launch pair
+    packed = store.k.nbytes + store.v.nbytes
+    return {"value": world * (in_b + out_b) / (ms_step * 1e-3) / 1e9, "ms_per_step": ms_step,
+            "steps": steps, "total_ms": ms,
+            "stages_ms": {"append_encode": round(enc, 4), "layer_decode": round(dec, 4)},
+            "tokens_layers_per_s": world * (S * L + S * n_mean) / (ms_step * 1e-3),
+            "bits_per_elem": packed * 8 / (S * L * H * cap * 128 * 2),
+            "rooflines": roof, "clocks": clocks,
+            "metric_note": "bf16 bytes appended (in) + decoded (out) per step"}
+
+
+# --------------------------------------------------------------- oracle legs
+def oracle_workers(args) -> int:
+    """Worker processes of the all-cores oracle figure: every host core, at
+    most 32 (each holds about a GB at the largest sample)."""
+    from oracle import parity
+
+    return args.cpu_workers or min(parity.host_cores(), 32)
+
+
+def cpu_baseline(args, wl, pool, workers):
+    """The oracle as it stands, timed on the host cores: single-threaded on one
+    layer sample, and `workers` such samples (distinct layers) in parallel
+    processes (wall clock from the first pass's start to the last one's end).
+    The sample is one layer cut to at most --cpu-tokens tokens."""
+    from oracle import baseline, parity
+
+    fields = baseline.workload_fields(wl)
+    tokens = min(wl.tokens, args.cpu_tokens)
+    job = lambda l: {"workload": fields, "layer": l % wl.layers, "tokens": tokens}  # noqa: E731
+    if wl.name == "decode_append":
+        job = lambda l: {"workload": fields, "units": 64, "seed": l}  # noqa: E731
+        fn = baseline.timed_append_step
+    else:
+        fn = baseline.timed_unit
+    single = pool.submit(fn, job(0)).result()
+    if workers > 1:
+        res = list(pool.map(fn, [job(l) for l in range(workers)]))
+        wall = max(r["t1"] for r in res) - min(r["t0"] for r in res)
+        tot = sum(r["bytes"] for r in res)
+    else:
+        wall, tot = single["seconds"], single["bytes"]
+    what = ("one append of 64 units + one unit's decode" if wl.name == "decode_append" else
+            f"one layer ({wl.heads} heads x {tokens} of {wl.tokens} tokens)")
+    return {"value": tot / wall / 1e9, "unit": "GB/s", "cores": workers, "kind": "oracle",
+            "sample": f"{workers} worker process(es), each {what} through the single-threaded "
+                      f"C oracle (score/select/encode/decode), wall clock of the parallel run",
+            "host_cores": parity.host_cores(),
+            "single_thread": {"value": single["bytes"] / single["seconds"] / 1e9,
+                              "unit": "GB/s", "cores": 1, "sample": what}}
+
+
+def headline_parity(args, wl, t, pool):
+    """The headline cache's GPU outputs on a few layers against the oracle
+    (oracle/parity.py: excused and unexcused mismatches, decoded bf16)."""
+    from oracle import parity
+
+    codec, units = t["codec"], t["codec"].units
+    layers = sorted({(int(x) % units) for x in args.parity_layers.split(",") if x.strip()})
+    u16 = lambda x: x.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    u32 = lambda x: x.cpu().contiguous().numpy().view(np.uint32)  # noqa: E731
+    futs = []
+    for u in layers:
+        job = {"K": u16(t["Kq"][u]), "V": u16(t["Vq"][u]), "theta": wl.theta,
+               "bits_k": wl.bits_k, "bits_v": wl.bits_v, "window": wl.window,
+               "pct": wl.evict_pct if codec.evict else 0,
+               "gpu_scores": codec.scores[u].cpu().numpy() if codec.evict else None,
+               "gpu_kept": codec.kept[u].cpu().numpy() if codec.evict else None,
+               "gk_codes": u32(codec.k_store.codes[u]), "gk_meta": u32(codec.k_store.meta[u]),
+               "gv_codes": u32(codec.v_store.codes[u]), "gv_meta": u32(codec.v_store.meta[u]),
+               "gK": u16(t["Kd"][u]), "gV": u16(t["Vd"][u])}
+        futs.append(pool.submit(parity.check_layer, job))
+    tot = parity.merge(f.result() for f in futs)
+    return {"layers_checked": layers, "elements": tot.get("elements", 0),
+            "excused": tot.get("excused_codes", 0) + tot.get("kept_excused", 0),
+            "unexcused": tot.get("unexcused_codes", 0) + tot.get("kept_unexcused", 0),
+            "kept_set_differences": tot.get("kept_diff", 0),
+            "bf16_elements_differing": tot.get("bf16_diff", 0),
+            "recon_max_rel": tot.get("recon_max_rel", 0.0),
+            "failures": parity.verdict(tot),
+            "rule": "bit-exact codes and kept sets; a mismatch is excused only within 1e-5 "
+                    "relative of a decision boundary (must stay below 1e-6 of elements)"}
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the oracle (the CPU restatement of the method) as it
+    stands, on the host cores, each step a bounded sample of the workload: one
+    layer sample per worker process, all workers in parallel."""
     if rank != 0:
         return
     wl = build_workload(args)
-    device = "cuda" if torch.cuda.is_available() else "cpu"
-    import oracle as oq
+    from oracle import baseline, parity
 
-    oq.build()
-    Kl, Vl = host_layer(wl, 0, device)
-    per = Kl.nbytes + Vl.nbytes
-    for _ in range(args.warmup):
-        oracle_pass(oq, Kl, Vl, wl)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_pass(oq, Kl, Vl, wl)
-    dt = time.perf_counter() - t0
-    val = per * args.steps / dt / 1e9
+    workers = oracle_workers(args)
+    fields = baseline.workload_fields(wl)
+    tokens = min(wl.tokens, args.cpu_tokens // 8 if args.cpu_tokens >= 8 else 1)
+    if wl.name == "decode_append":
+        fn, job = baseline.timed_append_step, lambda l: {"workload": fields, "units": 16, "seed": l}
+    else:
+        fn, job = baseline.timed_unit, lambda l: {"workload": fields, "layer": l % wl.layers,
+                                                  "tokens": tokens}
+    pool = parity.make_pool(workers)
+    try:
+        for _ in range(args.warmup):
+            list(pool.map(fn, [job(l) for l in range(workers)]))
+        nbytes, dt = 0, 0.0
+        for _ in range(args.steps):
+            res = list(pool.map(fn, [job(l) for l in range(workers)]))
+            nbytes += sum(r["bytes"] for r in res)
+            # the step's oracle work: first pass start to last pass end
+            dt += max(r["t1"] for r in res) - min(r["t0"] for r in res)
+    finally:
+        pool.shutdown()
+    val = nbytes / dt / 1e9
+    what = ("one append of 16 units + one unit's decode" if wl.name == "decode_append" else
+            f"one layer ({wl.heads} heads x {tokens} tokens)")
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
@@ -352,15 +635,23 @@ def run_reference(args, world, rank):
         "config": {"workload": wl.name, "layers": wl.layers, "heads": wl.heads, "tokens": wl.tokens,
                    "bits": f"K{wl.bits_k}V{wl.bits_v}", "evict_pct": wl.evict_pct,
                    "window": wl.window, "theta": wl.theta,
-                   "step": "one layer of the cache per step (bounded sample)"},
-        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"1 of {wl.layers} layers per step"},
+                   "step": f"{workers} worker processes x {what} (bounded sample)"},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": workers, "kind": "oracle",
+                         "sample": f"{workers} workers x {what} per step"},
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ our arm
+def config_names(args):
+    if args.configs == "none":
+        return []
+    names = [n for n in synth.WORKLOADS if n != args.workload] if args.configs == "all" else \
+        [n.strip() for n in args.configs.split(",") if n.strip() and n.strip() != args.workload]
+    return names
+
+
 def run_ours(args, world, rank, local):
     from e8_lattice_vector_nq_b200 import nq
 
@@ -369,130 +660,101 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     wl = build_workload(args)
-    units = wl.layers
-    K, V = gen_cache(wl, device)
-    codec = nq.Codec(units, wl.heads, wl.tokens, wl.theta, wl.bits_k, wl.bits_v, window=wl.window,
-                     evict_pct=wl.evict_pct, device=device)
-    n = codec.n
-    Kd = torch.empty(units, wl.heads, n, 128, dtype=torch.bfloat16, device=device)
-    Vd = torch.empty_like(Kd)
-    stream = torch.cuda.current_stream(device)
-    stages = ["score", "select", "encode", "decode"] if codec.evict else ["encode", "decode"]
-
-    def step(ev=None):
-        if codec.evict:
-            if ev: ev[0].record(stream)
-            nq.nq_score(K, codec.W, codec.scores, codec.ws)
-            if ev: ev[1].record(stream)
-            nq.nq_select(codec.scores, codec.W, codec.pct, codec.kept)
-            if ev: ev[2].record(stream)
-        elif ev:
-            ev[2].record(stream)
-        nq.nq_encode(K, V, codec.k_store, codec.v_store, n, codec.rope, codec.max_pos, kept=codec.kept)
-        if ev: ev[3].record(stream)
-        nq.nq_decode(codec.k_store, codec.v_store, n, Kd, Vd, codec.rope, codec.max_pos,
-                     positions=codec.kept)
-        if ev: ev[4].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-
-    def timed():
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler(device.index if device.index is not None else local) as clk:
-            if world > 1:
-                torch.distributed.barrier()
-            torch.cuda.synchronize()
-            start.record(stream)
-            for i in range(args.steps):
-                step(evs[i])
-            end.record(stream)
-            torch.cuda.synchronize()
-            if world > 1:
-                torch.distributed.barrier()
-        per = {}
-        if codec.evict:
-            per["score"] = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-            per["select"] = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-        per["encode"] = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-        per["decode"] = sum(e[3].elapsed_time(e[4]) for e in evs) / args.steps
-        return start.elapsed_time(end), per, clk.summary()
-
-    ms, per_stage, clocks = timed()
-    # a slowdown other than the power cap during the timed region: measure once more
-    bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
-    redo = int(bool(clocks and bad & set(clocks["reasons"])))
-    if world > 1:
-        t = torch.tensor([redo], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        redo = int(t.item())
-    if redo:
-        ms, per_stage, clocks = timed()
-        if clocks is not None:
-            clocks["remeasured"] = True
-    ms = max_over_ranks(ms, world, device)
-    assert nq.device_error() == 0, "a kernel reported an in-kernel failure"
-
-    in_bytes = K.numel() * 2 + V.numel() * 2
-    ms_step = ms / args.steps
-    value = world * in_bytes / (ms_step * 1e-3) / 1e9
     peak, peak_kind = measured_peaks()
-    alg = algorithmic_bytes(wl, n, units)
-    dom = max(per_stage, key=per_stage.get)
-    achieved = alg[dom] / (per_stage[dom] * 1e-3) / 1e9
-    kernel_name = {"score": "score_kernel", "select": "select_kernel", "encode": "encode_kernel",
-                   "decode": "decode_kernel"}[dom]
-    # the recorded figure belongs to the named workload at its full size only
-    full_size = wl == synth.WORKLOADS[args.workload]
-    traffic = recorded_traffic(kernel_name, wl.name) if full_size else None
+    # oracle worker processes (spawn) for the CPU legs, rank 0 only
+    pool, workers = None, 0
+    if not args.no_cpu_baseline and rank == 0:
+        from oracle import parity
 
-    enc_ms = sum(per_stage[s] for s in stages if s != "decode")
-    out_bytes = Kd.numel() * 2 + Vd.numel() * 2
-    packed_bits = codec.packed_bytes * 8
+        workers = oracle_workers(args)
+        pool = parity.make_pool(workers)
+    try:
+        line = _run_ours(args, world, rank, device, wl, peak, peak_kind, pool, workers, nq)
+    finally:
+        if pool is not None:
+            pool.shutdown()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _run_ours(args, world, rank, device, wl, peak, peak_kind, pool, workers, nq):
+    if wl.name == "decode_append":
+        f = time_append(nq, wl, device, world, args.warmup)
+        line = {"metric": METRIC, "value": f["value"], "unit": "GB/s", "n_gpus": world,
+                "steps": f["steps"], "warmup": args.warmup, "ms_per_step": f["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic",
+                "config": {"workload": wl.name, "sequences": wl.sequences, "layers": wl.layers,
+                           "heads": wl.heads, "tokens": wl.tokens, "append_steps": wl.append_steps,
+                           "bits": f"K{wl.bits_k}V{wl.bits_v}", "theta": wl.theta,
+                           "parallelism": f"replicas x{world}"},
+                **{k: v for k, v in f.items() if k not in ("value", "ms_per_step", "steps")}}
+        line["roofline"] = f["rooflines"]["decode"]
+        line["gpu_launches"] = f["steps"] * 4
+        if pool is not None:
+            line["cpu_baseline"] = cpu_baseline(args, wl, pool, workers)
+        return line
+
+    t = time_cache(nq, wl, device, args.steps, args.warmup, world)
+    f = figures(wl, t, world, peak, peak_kind)
+    dom = max(t["per_stage"], key=t["per_stage"].get)
+    roof = dict(f["rooflines"][dom])
+    full_size = wl == synth.WORKLOADS[args.workload]
+    roof["traffic"] = recorded_traffic(roof["kernel"], wl.name) if full_size else None
+    for stage, r in f["rooflines"].items():
+        r["traffic"] = recorded_traffic(r["kernel"], wl.name) if full_size else None
+    codec = t["codec"]
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "metric": METRIC, "value": f["value"], "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": f["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
         "config": {"workload": wl.name, "layers": wl.layers, "heads": wl.heads, "tokens": wl.tokens,
                    "head_dim": 128, "bits": f"K{wl.bits_k}V{wl.bits_v}",
                    "evict_pct": wl.evict_pct, "window": wl.window, "theta": wl.theta,
-                   "kept_per_layer": n, "l2": "inputs larger than L2 (no flush)",
+                   "kept_per_layer": codec.n, "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas x{world}"},
-        "stages_ms": {k: round(v, 4) for k, v in per_stage.items()},
-        "encode_gbs": in_bytes / (enc_ms * 1e-3) / 1e9,
-        "decode_gbs": out_bytes / (per_stage["decode"] * 1e-3) / 1e9,
-        "tokens_layers_per_s": world * wl.tokens * wl.layers / (ms_step * 1e-3),
-        "bits_per_elem": packed_bits / (K.numel() + V.numel()),
-        "hbm_frac_of_step": (sum(alg.values()) / (ms_step * 1e-3) / 1e9) / peak,
-        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "algorithmic_bytes": alg[dom]},
-        "gpu_launches": args.steps * ((3 if codec.evict else 0) + 4),
+        **{k: v for k, v in f.items() if k not in ("value", "ms_per_step")},
+        "roofline": roof,
+        "gpu_launches": args.steps * t["launches_per_step"],
     }
-    if clocks:
-        line["clocks"] = clocks
-
+    if t["clocks"]:
+        line["clocks"] = t["clocks"]
+    K, V, Kd, Vd, stream = t["K"], t["V"], t["Kd"], t["Vd"], t["stream"]
     if not args.no_attend:
         line["decode_attention"] = attend_timing(args, codec, Kd, Vd, stream, world)
-    line["reconstruction"] = reconstruction_quality(K, V, Kd, Vd, codec)
+    line["reconstruction"] = reconstruction_quality(t["Kq"], t["Vq"], Kd, Vd, codec)
     if args.layerwise:
-        line["layerwise_encode"] = layerwise_timing(codec, K, V, stream, world)
+        line["layerwise_encode"] = layerwise_timing(codec, t["Kq"], t["Vq"], stream, world)
     if not args.no_entropy:
-        line["entropy_stage"] = entropy_timing(args, codec, stream, world,
-                                               K.numel() + V.numel())
+        line["entropy_stage"] = entropy_timing(args, codec, stream, world, K.numel() + V.numel())
     if not args.no_e2e:
-        line["e2e"] = e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes)
-    if not args.no_cpu_baseline and rank == 0:
-        del Kd, Vd
-        hl = (K[0].cpu().view(torch.int16).numpy().view(np.uint16),
-              V[0].cpu().view(torch.int16).numpy().view(np.uint16))
-        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_layers, device, hl=hl)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+        in_bytes = K.numel() * 2 + V.numel() * 2
+        line["e2e"] = e2e(args, t["Kq"], t["Vq"], Kd, Vd, codec, stream, world, in_bytes)
+    if pool is not None:
+        line["parity"] = headline_parity(args, wl, t, pool)
+        line["cpu_baseline"] = cpu_baseline(args, wl, pool, workers)
+    del t, K, V, Kd, Vd, codec
+    torch.cuda.empty_cache()
+
+    configs = {}
+    for name in config_names(args):
+        cw = synth.WORKLOADS[name]
+        if cw.name == "decode_append":
+            cf = time_append(nq, cw, device, world, args.warmup)
+        else:
+            ct = time_cache(nq, cw, device, args.config_steps, args.warmup, world)
+            cf = figures(cw, ct, world, peak, peak_kind)
+            cf["clocks"] = ct["clocks"]
+            del ct
+        cf.pop("metric_note", None)
+        if pool is not None:
+            cf["cpu_baseline"] = cpu_baseline(args, cw, pool, 1)
+        configs[name] = cf
+        torch.cuda.empty_cache()
+    if configs:
+        line["configs"] = configs
+    return line
 
 
 def attend_timing(args, codec, Kd, Vd, stream, world, G: int = 4):

@@ -144,6 +144,8 @@ nq_status nq_score(const void* K, nq_kv_strides ks, int units, int heads, int64_
                 nq_score_workspace_bytes(units, heads));
   if (static_cast<int64_t>(units) * ((T + 127) / 128) > 0x7FFFFFFF)
     return fail(NQ_ERR_UNSUPPORTED, "units * T too large for one launch");
+  if (static_cast<int64_t>(units) * heads > 0x7FFFFFFF)
+    return fail(NQ_ERR_UNSUPPORTED, "units * heads too large for one launch");
   return cuda_status(nq::launch_score(K, ks, units, heads, T, W, scores, static_cast<float*>(ws),
                                       reinterpret_cast<cudaStream_t>(stream)),
                      "nq_score launch");

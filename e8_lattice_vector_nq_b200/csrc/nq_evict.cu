@@ -20,6 +20,8 @@
 //                       ordered compaction with warp ballots.
 #include <cooperative_groups.h>
 
+#include <cuda.h>
+
 #include <mutex>
 
 #include "nq_internal.h"
@@ -447,22 +449,46 @@ namespace {
 constexpr int kMaxDevices = 256;
 std::mutex g_scratch_mu;
 float* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 }  // namespace
 
 // Device address of g_score_scratch on the current device.  Host code only
 // sees a host-side stand-in under the array's name, so the address is looked
-// up once per device, with that device current, and cached.
+// up with the device current and cached per device, together with the
+// context it belongs to: after a device reset (a new primary context, the
+// module loaded again) the next call looks the address up again.
 static cudaError_t score_scratch_address(float** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (!get_ctx) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!ctx || !g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
+    // the lookup also makes the device's primary context current if none is
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_score_scratch);
     if (err != cudaSuccess) return err;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
     g_scratch_addr[dev] = static_cast<float*>(p);
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;

@@ -143,9 +143,11 @@ nq_status nq_score(const void *K, nq_kv_strides ks, int units, int heads, int64_
  * cudaMalloc, cudaFree or other allocating routine.
  *   - units * heads above the maximum, or heads above 128: NQ_ERR_UNSUPPORTED,
  *     nothing launched.
- *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before
- *     any stream capture.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it with the device's context; the
+ *     first call after a device reset (a new context) looks it up again.
+ *     Make the first call on a device, and after a reset, before any stream
+ *     capture.
  *   - All calls share the array and it keeps the last call's contents (each
  *     call overwrites every entry it reads, so nothing needs clearing).
  *     Calls whose kernels overlap on the same GPU (different streams, or

@@ -82,6 +82,8 @@ def _load():
             "oq_encode_box_batch": (i64, [P, i64, i32, P, P, i32, P, P]),
             "oq_fold_exact_batch": (None, [P, P, i64, i32, P, P]),
             "oq_unfold_exact_batch": (None, [P, P, i64, i32, P, P]),
+            "oq_encode_margin_batch": (None, [P, i64, i32, P, P, i32, P]),
+            "oq_e8_margin_batch": (None, [P, i64, P]),
             "oq_exact_pack_group": (ctypes.c_uint32, [P, i32, i32]),
             "oq_exact_unpack_group": (None, [ctypes.c_uint32, i32, P, P]),
             "oq_ans_table": (None, [P, i32, P]),
@@ -202,6 +204,32 @@ def encode_vectors(x_bf16, bits: int, rope: bool = False, c=None, s=None):
     m = np.empty(n, np.uint32)
     cl = _load().oq_encode_batch(_p(x), n, int(rope), _p(c), _p(s), bits, _p(w), _p(m))
     return w, m, int(cl)
+
+
+def encode_margins(x_bf16, bits: int, rope: bool = False, c=None, s=None) -> np.ndarray:
+    """Per vector, the smallest relative distance of any encode decision to
+    its boundary (0 on a boundary, at most 1): the scale's fp16 rounding, each
+    coordinate's rounding, the parity move and the coset choice.  Used to tell
+    excusable GPU/oracle mismatches (near a boundary) from real ones."""
+    x = _u16(x_bf16).reshape(-1, D)
+    n = x.shape[0]
+    if c is None:
+        c = np.zeros((n, D // 2), np.float32)
+        s = np.zeros((n, D // 2), np.float32)
+    c = np.ascontiguousarray(c, dtype=np.float32).reshape(n, D // 2)
+    s = np.ascontiguousarray(s, dtype=np.float32).reshape(n, D // 2)
+    out = np.empty(n, np.float64)
+    _load().oq_encode_margin_batch(_p(x), n, int(rope), _p(c), _p(s), bits, _p(out))
+    return out
+
+
+def e8_margins(y) -> np.ndarray:
+    """Per group of 8 fp32 coordinates, the smallest relative distance of an
+    E8 decision (rounding, parity move, coset choice) to its boundary."""
+    y = np.ascontiguousarray(y, dtype=np.float32).reshape(-1, 8)
+    out = np.empty(y.shape[0], np.float64)
+    _load().oq_e8_margin_batch(_p(y), y.shape[0], _p(out))
+    return out
 
 
 def decode_vectors(words, meta, bits: int, rope: bool = False, c=None, s=None):

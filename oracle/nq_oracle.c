@@ -811,6 +811,97 @@ void oq_unfold_exact_batch(const uint32_t *in, const uint16_t *sig16, int64_t n,
         oq_unfold_exact(in + 4 * bits * i, sig16[i], bits, words + 4 * bits * i, meta + i);
 }
 
+/* -------------------------------------- decision margins (parity accounting)
+ * How near each decision of the encoder lies to its boundary.  The parity rule
+ * for the GPU path excuses a mismatch with the oracle only where the oracle's
+ * value sits within a small relative distance (1e-5) of the boundary of a
+ * decision; these functions give that distance (0 = on the boundary, capped
+ * at 1).  They take the decisions exactly as oq_d8_decode, oq_e8_nearest and
+ * oq_encode_vector_mode take them.  Per group of 8 scaled coordinates y, for
+ * the integer coset (shift 0) and the half coset (shift 1/2), with
+ * u = fl32(y - shift), f = rint(u), e = u - f:
+ *   rounding      | |e_i| - 1/2 | / (1/2)       (u_i at a rounding tie)
+ *   parity move   (m1 - m2) / m1, when sum f is odd, m1 >= m2 the two
+ *                 largest |e_i| (which coordinate moves)
+ * and between the cosets |d1 - d0| / max(d0, d1) with the fp32 distances of
+ * oq_d8_decode.  Per vector, also the scale's fp16 rounding: |P - mid| / P,
+ * P = fp32(M * G_b), mid = the midpoint of the two fp16 values around P. */
+static double oq_min(double a, double b) { return a < b ? a : b; }
+
+static double oq_coset_margin(const float *y, float shift)
+{
+    double mg = 1.0, m1 = 0.0, m2 = 0.0;
+    int32_t sum = 0;
+    for (int i = 0; i < 8; i++) {
+        float u = y[i] - shift;
+        float f = rintf(u);
+        double a = fabs((double)(u - f));
+        mg = oq_min(mg, fabs(a - 0.5) / 0.5);
+        sum += (int32_t)f;
+        if (a > m1) { m2 = m1; m1 = a; }
+        else if (a > m2) { m2 = a; }
+    }
+    if ((sum & 1) && m1 > 0.0) mg = oq_min(mg, (m1 - m2) / m1);
+    return mg;
+}
+
+double oq_e8_margin(const float *y)
+{
+    int32_t g[8];
+    double d0 = oq_d8_decode(y, 0.0f, g), d1 = oq_d8_decode(y, 0.5f, g);
+    double mg = oq_min(oq_coset_margin(y, 0.0f), oq_coset_margin(y, 0.5f));
+    double big = d0 > d1 ? d0 : d1;
+    if (big > 0.0) mg = oq_min(mg, fabs(d1 - d0) / big);
+    return mg;
+}
+
+/* Smallest decision margin of the encode of one 128-vector (steps as in
+ * oq_encode_vector_mode: RoPE undo for keys, FWHT, scale, then the E8 step
+ * per group).  A zero vector (sigma 0) takes no decision: margin 1. */
+double oq_encode_margin(const uint16_t *x, int rope, const float *c, const float *s, int bits)
+{
+    float v[OQ_D];
+    for (int i = 0; i < OQ_D; i++) v[i] = oq_bf16_to_f32(x[i]);
+    if (rope) oq_rope_undo(v, c, s);
+    oq_fwht128(v);
+    float M = 0.0f;
+    for (int i = 0; i < OQ_D; i++) M = fmaxf(M, fabsf(v[i]));
+    float P = M * oq_u2f(bits == 3 ? OQ_G3_BITS : OQ_G2_BITS);
+    double mg = 1.0;
+    if (P > 65504.0f) P = 65504.0f; /* saturated: the clamp decides, not a rounding */
+    else if (P > 0.0f) {
+        uint16_t h = oq_f32_to_f16(P);
+        double near = oq_f16_to_f32(h);
+        double other = (double)P >= near ? oq_f16_to_f32((uint16_t)(h + 1))
+                                         : oq_f16_to_f32((uint16_t)(h - 1));
+        mg = oq_min(mg, fabs((double)P - 0.5 * (near + other)) / (double)P);
+    }
+    float sig = oq_f16_to_f32(oq_f32_to_f16(P));
+    if (sig == 0.0f) return mg;
+    float r = oq_u2f(OQ_C_BITS) / sig;
+    for (int g = 0; g < 16; g++) {
+        float y[8];
+        for (int i = 0; i < 8; i++) {
+            float p = v[8 * g + i] * r;
+            y[i] = (p == 0.0f) ? 0.0f : p;
+        }
+        mg = oq_min(mg, oq_e8_margin(y));
+    }
+    return mg;
+}
+
+void oq_encode_margin_batch(const uint16_t *x, int64_t n, int rope, const float *c,
+                            const float *s, int bits, double *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oq_encode_margin(x + OQ_D * i, rope, c + OQ_HALF * i, s + OQ_HALF * i, bits);
+}
+
+void oq_e8_margin_batch(const float *y, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = oq_e8_margin(y + 8 * i);
+}
+
 /* ------------------------------------------------- delta + entropy stage */
 
 /* The lattice indices (the b-bit codes) of a packed store, coded the way the

@@ -1,7 +1,8 @@
 """bench.py's JSON line on a small cache (2 layers of the Mistral-shaped
 workload): every key the benchmark contract asks for is present and
 consistent, and the optional blocks (attention, entropy, layer-by-layer
-encode) run."""
+encode, parity against the oracle) run; a second run checks the per-workload
+summaries (tiny and decode-append at full size)."""
 import json
 import os
 import subprocess
@@ -19,8 +20,9 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def line():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    res = subprocess.run([sys.executable, "bench.py", "--layers", "2", "--steps", "3", "--warmup",
-                          "3", "--e2e-steps", "1", "--cpu-layers", "1", "--layerwise"],
+    res = subprocess.run([sys.executable, "bench.py", "--workload", "mistral7b_32k", "--layers",
+                          "2", "--steps", "3", "--warmup", "3", "--e2e-steps", "1", "--cpu-tokens",
+                          "4096", "--layerwise", "--configs", "none", "--parity-layers", "0,1"],
                          cwd=ROOT, capture_output=True, text=True, timeout=900)
     assert res.returncode == 0, res.stderr[-2000:]
     lines = [x for x in res.stdout.splitlines() if x.startswith("{")]
@@ -48,6 +50,9 @@ def test_roofline_and_baselines(line):
     assert r["traffic"] is None  # recorded for the full 32-layer launch only
     c = line["cpu_baseline"]
     assert c["kind"] == "oracle" and c["cores"] >= 1 and c["value"] > 0 and c["sample"]
+    assert c["host_cores"] >= c["cores"] and c["single_thread"]["value"] > 0
+    for stage in ("score", "select", "encode", "decode"):
+        assert line["rooflines"][stage]["ms"] > 0
     e = line["e2e"]
     assert e["value"] > 0 and e["unit"] == line["unit"]
     assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
@@ -74,3 +79,30 @@ def test_optional_blocks(line):
         assert 0 < s["codes_bits_per_elem_coded"] < 4
     w = line["layerwise_encode"]
     assert w["all_layers_ms"] > 0 and w["layer_by_layer_ms"] > 0
+
+
+def test_parity_block(line):
+    p = line["parity"]
+    assert p["layers_checked"] == [0, 1]
+    assert p["unexcused"] == 0 and p["failures"] == [] and p["bf16_elements_differing"] == 0
+    assert p["elements"] == 2 * 2 * 8 * line["config"]["kept_per_layer"] * 128
+
+
+def test_config_summaries():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    res = subprocess.run([sys.executable, "bench.py", "--workload", "mistral7b_32k", "--layers",
+                          "1", "--steps", "3", "--warmup", "3", "--no-e2e", "--no-attend",
+                          "--no-entropy", "--cpu-tokens", "2048", "--configs",
+                          "tiny,decode_append", "--config-steps", "3"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads([x for x in res.stdout.splitlines() if x.startswith("{")][0])
+    c = line["configs"]
+    assert set(c) == {"tiny", "decode_append"}
+    t = c["tiny"]
+    assert t["value"] > 0 and abs(t["bits_per_elem"] - 2.75) < 1e-9
+    assert t["rooflines"]["encode"]["frac"] > 0 and t["cpu_baseline"]["value"] > 0
+    a = c["decode_append"]
+    assert a["steps"] == 256 and a["stages_ms"]["append_encode"] > 0
+    assert a["stages_ms"]["layer_decode"] > 0 and a["cpu_baseline"]["value"] > 0
