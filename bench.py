@@ -855,32 +855,42 @@ def layerwise_timing(codec, K, V, stream, world, reps: int = 10):
 
 def entropy_timing(args, codec, stream, world, total_elems):
     """The delta + rANS stage over the lattice indices of the whole packed
-    cache (keys and values, every layer in one call each): coded size and
-    encode / decode time, with and without the token difference.  Code bits
-    are per kept element; the cache figure (coded codes + raw meta) is per
-    element of the bf16 input cache, like bits_per_elem.  CUDA events, max
-    over ranks."""
+    cache (keys and values): coded size and encode / decode time, with and
+    without the token difference.  One call per store covers as many layers
+    as its 32-bit stream offsets allow (all of them up to 32K tokens; chunks of
+    layers beyond).  Code bits are per kept element; the cache figure (coded
+    codes + raw meta) is per element of the bf16 input cache, like
+    bits_per_elem.  CUDA events, max over ranks."""
     from e8_lattice_vector_nq_b200 import nq
 
-    res = {}
+    L = nq.lib()
+    units, heads, n = codec.units, codec.heads, codec.n
+    per = units
+    while per > 1 and L.nq_entropy_max_words(per, heads, n) > 0xFFFFFFFF:
+        per = (per + 1) // 2
+    chunks = [slice(u, min(u + per, units)) for u in range(0, units, per)]
+    res = {"layers_per_call": per, "calls_per_store": len(chunks)}
     elems = 0
     for name, st in (("k", codec.k_store), ("v", codec.v_store)):
         elems += st.meta.numel() * 128
     dev = codec.k_store.codes.device
-    out = {"k": nq.PackedStore.empty(codec.units, codec.heads, codec.n, codec.k_store.bits, dev),
-           "v": nq.PackedStore.empty(codec.units, codec.heads, codec.n, codec.v_store.bits, dev)}
-    ws = nq.entropy_workspace(codec.units, codec.heads, codec.n, dev)
+    out = {"k": nq.PackedStore.empty(units, heads, n, codec.k_store.bits, dev),
+           "v": nq.PackedStore.empty(units, heads, n, codec.v_store.bits, dev)}
+    ws = nq.entropy_workspace(per, heads, n, dev)
+    stores = {"k": codec.k_store, "v": codec.v_store}
     coded = {}
     for delta in (True, False):
 
         def enc():
-            for name, st in (("k", codec.k_store), ("v", codec.v_store)):
-                coded[name] = nq.nq_entropy_encode(st, codec.n, delta=delta, ws=ws,
-                                                   coded=coded.get(name))
+            for name, st in stores.items():
+                for c, sl in enumerate(chunks):
+                    coded[(name, c)] = nq.nq_entropy_encode(st.select_units(sl), n, delta=delta,
+                                                            ws=ws, coded=coded.get((name, c)))
 
         def dec():
-            for name in ("k", "v"):
-                nq.nq_entropy_decode(coded[name], out[name])
+            for name in stores:
+                for c, sl in enumerate(chunks):
+                    nq.nq_entropy_decode(coded[(name, c)], out[name].select_units(sl))
 
         def t(fn, reps=5):
             fn()
@@ -895,8 +905,7 @@ def entropy_timing(args, codec, stream, world, total_elems):
 
         enc_ms = t(enc)
         dec_ms = t(dec)
-        exact = all(torch.equal(out[nm].codes, st.codes)
-                    for nm, st in (("k", codec.k_store), ("v", codec.v_store)))
+        exact = all(torch.equal(out[nm].codes, st.codes) for nm, st in stores.items())
         coded_bytes = sum(c.coded_bytes() for c in coded.values())
         code_bytes = codec.k_store.codes.numel() * 4 + codec.v_store.codes.numel() * 4
         meta_bytes = codec.k_store.meta.numel() * 4 + codec.v_store.meta.numel() * 4
