@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-attend", action="store_true", help="skip the decode-attention timing")
+    ap.add_argument("--no-exact", action="store_true",
+                    help="skip the exact (24/16-bit) layout timing")
     ap.add_argument("--no-entropy", action="store_true",
                     help="skip the delta + entropy stage timing")
     ap.add_argument("--layerwise", action="store_true",
@@ -724,6 +726,8 @@ def _run_ours(args, world, rank, device, wl, peak, peak_kind, pool, workers, nq)
     if not args.no_attend:
         line["decode_attention"] = attend_timing(args, codec, Kd, Vd, stream, world)
     line["reconstruction"] = reconstruction_quality(t["Kq"], t["Vq"], Kd, Vd, codec)
+    if not args.no_exact:
+        line["exact_layout"] = exact_timing(args, wl, t, world, peak, peak_kind)
     if args.layerwise:
         line["layerwise_encode"] = layerwise_timing(codec, t["Kq"], t["Vq"], stream, world)
     if not args.no_entropy:
@@ -755,6 +759,59 @@ def _run_ours(args, world, rank, device, wl, peak, peak_kind, pool, workers, nq)
     if configs:
         line["configs"] = configs
     return line
+
+
+def exact_timing(args, wl, t, world, peak, peak_kind):
+    """The exact (24/16-bit) layout on the same cache: nq_encode_exact and
+    nq_decode_exact over every layer in one call each (the box-constrained E8
+    step, the coset bit folded into the codes, a uint16 scale per vector),
+    timed like the main stages; bits per element of the stored cache."""
+    from e8_lattice_vector_nq_b200 import nq
+
+    codec, stream, dev = t["codec"], t["stream"], t["Kd"].device
+    units, heads, n = codec.units, codec.heads, codec.n
+    ks = nq.ExactStore.empty(units, heads, n, wl.bits_k, dev)
+    vs = nq.ExactStore.empty(units, heads, n, wl.bits_v, dev)
+    Kq, Vq, Kd, Vd = t["Kq"], t["Vq"], t["Kd"], t["Vd"]
+
+    def enc():
+        nq.nq_encode_exact(Kq, Vq, ks, vs, n, codec.rope, codec.max_pos, kept=codec.kept)
+
+    def dec():
+        nq.nq_decode_exact(ks, vs, n, Kd, Vd, codec.rope, codec.max_pos, positions=codec.kept)
+
+    def tm(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) / reps, world, dev)
+
+    reps = max(3, min(args.steps, 10))
+    enc_ms, dec_ms = tm(enc, reps), tm(dec, reps)
+    assert nq.device_error() == 0
+    per_vec_bytes = 16 * wl.bits_k + 2 + 16 * wl.bits_v + 2
+    kept_bytes = (n * 4 * units) if codec.kept is not None else 0
+    alg = units * n * heads * (512 + per_vec_bytes) + kept_bytes
+    elems = (t["K"].numel() + t["V"].numel())
+    stored = ks.nbytes + vs.nbytes + kept_bytes
+    roof = {}
+    for stage, ms in (("encode", enc_ms), ("decode", dec_ms)):
+        ach = alg / (ms * 1e-3) / 1e9
+        roof[stage] = {"kernel": f"{stage}_kernel (exact layout)", "bound": "hbm",
+                       "achieved": ach, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                       "frac": ach / peak, "algorithmic_bytes": alg, "ms": ms}
+    return {"encode_ms": enc_ms, "decode_ms": dec_ms,
+            "bits_per_coordinate": {"k": (16 * wl.bits_k + 2) * 8 / 128,
+                                    "v": (16 * wl.bits_v + 2) * 8 / 128},
+            "bits_per_elem": stored * 8 / elems, "rooflines": roof,
+            "encode_vs_regular": enc_ms / t["per_stage"]["encode"],
+            "decode_vs_regular": dec_ms / t["per_stage"]["decode"]}
 
 
 def attend_timing(args, codec, Kd, Vd, stream, world, G: int = 4):

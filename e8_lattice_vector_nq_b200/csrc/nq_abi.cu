@@ -200,11 +200,38 @@ nq_status nq_select(const double* scores, int units, int64_t T, int W, int evict
                      "nq_select launch");
 }
 
-nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_strides vs, int units,
-                    int heads, int64_t T_in, int64_t n, const int32_t* kept, int64_t kept_stride,
-                    int64_t pos_base, const float* rope_tab, int64_t rope_max_pos,
-                    const nq_packed* k_out, const nq_packed* v_out, int64_t slot0,
-                    nq_stream_t stream) {
+// The exact layout travels as an nq_packed whose meta points to the uint16
+// scales (checked here for 2-byte alignment).
+static nq_packed from_exact(const nq_packed_exact* p) {
+  nq_packed q{};
+  if (p) {
+    q.codes = p->codes;
+    q.meta = reinterpret_cast<uint32_t*>(p->sigma);
+    q.unit_stride = p->unit_stride;
+    q.head_stride = p->head_stride;
+    q.bits = p->bits;
+  }
+  return q;
+}
+
+static nq_status check_store(const nq_packed* p, bool exact, const char* name) {
+  if (!p) return fail(NQ_ERR_INVALID, "%s descriptor is NULL", name);
+  if (!exact) return check_packed(p, name);
+  if (p->bits != 2 && p->bits != 3)
+    return fail(NQ_ERR_INVALID, "%s.bits must be 2 or 3 (got %d)", name, p->bits);
+  if (!p->codes || !p->meta) return fail(NQ_ERR_INVALID, "%s codes/sigma is NULL", name);
+  if (!aligned(p->codes, 16)) return fail(NQ_ERR_INVALID, "%s.codes must be 16-byte aligned", name);
+  if (!aligned(p->meta, 2)) return fail(NQ_ERR_INVALID, "%s.sigma must be 2-byte aligned", name);
+  if (p->unit_stride < 0 || p->head_stride < 0)
+    return fail(NQ_ERR_INVALID, "%s strides must be non-negative", name);
+  return NQ_OK;
+}
+
+static nq_status encode_impl(const void* K, nq_kv_strides ks, const void* V, nq_kv_strides vs, int units,
+                      int heads, int64_t T_in, int64_t n, const int32_t* kept,
+                      int64_t kept_stride, int64_t pos_base, const float* rope_tab,
+                      int64_t rope_max_pos, const nq_packed* k_out, const nq_packed* v_out,
+                      int64_t slot0, bool exact, nq_stream_t stream) {
   if (!K && !V) return fail(NQ_ERR_INVALID, "K and V are both NULL");
   if (units < 0 || heads < 1 || heads > 1024 || n < 0 || slot0 < 0 || pos_base < 0)
     return fail(NQ_ERR_INVALID, "need units >= 0, 1 <= heads <= 1024, n >= 0, slot0 >= 0, pos_base >= 0");
@@ -220,7 +247,7 @@ nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_stride
   }
   if (K) {
     if (nq_status st = check_kv(K, ks, "K")) return st;
-    if (nq_status st = check_packed(k_out, "k_out")) return st;
+    if (nq_status st = check_store(k_out, exact, "k_out")) return st;
     if (nq_status st = check_rope(rope_tab, rope_max_pos)) return st;
     if (!kept && pos_base + n > rope_max_pos)
       return fail(NQ_ERR_INVALID, "positions up to %lld exceed rope_max_pos %lld",
@@ -228,7 +255,7 @@ nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_stride
   }
   if (V) {
     if (nq_status st = check_kv(V, vs, "V")) return st;
-    if (nq_status st = check_packed(v_out, "v_out")) return st;
+    if (nq_status st = check_store(v_out, exact, "v_out")) return st;
   }
   // K and V may live in pinned host memory: the kernels then read only the
   // rows they encode across the bus
@@ -255,14 +282,36 @@ nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_stride
   if (K) L.k_out = *k_out;
   if (V) L.v_out = *v_out;
   L.slot0 = slot0;
+  L.exact = exact;
   return cuda_status(nq::launch_encode(L, reinterpret_cast<cudaStream_t>(stream)),
-                     "nq_encode launch");
+                     exact ? "nq_encode_exact launch" : "nq_encode launch");
 }
 
-nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int heads,
-                    int64_t n, int64_t slot0, const int32_t* positions, int64_t pos_stride,
-                    int64_t pos_base, const float* rope_tab, int64_t rope_max_pos, void* K_out,
-                    nq_kv_strides kos, void* V_out, nq_kv_strides vos, nq_stream_t stream) {
+nq_status nq_encode(const void* K, nq_kv_strides ks, const void* V, nq_kv_strides vs, int units,
+                    int heads, int64_t T_in, int64_t n, const int32_t* kept, int64_t kept_stride,
+                    int64_t pos_base, const float* rope_tab, int64_t rope_max_pos,
+                    const nq_packed* k_out, const nq_packed* v_out, int64_t slot0,
+                    nq_stream_t stream) {
+  return encode_impl(K, ks, V, vs, units, heads, T_in, n, kept, kept_stride, pos_base, rope_tab,
+                     rope_max_pos, k_out, v_out, slot0, false, stream);
+}
+
+nq_status nq_encode_exact(const void* K, nq_kv_strides ks, const void* V, nq_kv_strides vs,
+                          int units, int heads, int64_t T_in, int64_t n, const int32_t* kept,
+                          int64_t kept_stride, int64_t pos_base, const float* rope_tab,
+                          int64_t rope_max_pos, const nq_packed_exact* k_out,
+                          const nq_packed_exact* v_out, int64_t slot0, nq_stream_t stream) {
+  const nq_packed k = from_exact(k_out), v = from_exact(v_out);
+  return encode_impl(K, ks, V, vs, units, heads, T_in, n, kept, kept_stride, pos_base, rope_tab,
+                     rope_max_pos, k_out ? &k : nullptr, v_out ? &v : nullptr, slot0, true,
+                     stream);
+}
+
+static nq_status decode_impl(const nq_packed* k_in, const nq_packed* v_in, int units, int heads,
+                             int64_t n, int64_t slot0, const int32_t* positions,
+                             int64_t pos_stride, int64_t pos_base, const float* rope_tab,
+                             int64_t rope_max_pos, void* K_out, nq_kv_strides kos, void* V_out,
+                             nq_kv_strides vos, bool exact, nq_stream_t stream) {
   if (!K_out && !V_out) return fail(NQ_ERR_INVALID, "K_out and V_out are both NULL");
   if (units < 0 || heads < 1 || heads > 1024 || n < 0 || slot0 < 0 || pos_base < 0)
     return fail(NQ_ERR_INVALID, "need units >= 0, 1 <= heads <= 1024, n >= 0, slot0 >= 0, pos_base >= 0");
@@ -273,7 +322,7 @@ nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int
   }
   if (K_out) {
     if (nq_status st = check_kv(K_out, kos, "K_out")) return st;
-    if (nq_status st = check_packed(k_in, "k_in")) return st;
+    if (nq_status st = check_store(k_in, exact, "k_in")) return st;
     if (nq_status st = check_rope(rope_tab, rope_max_pos)) return st;
     if (!positions && pos_base + n > rope_max_pos)
       return fail(NQ_ERR_INVALID, "positions up to %lld exceed rope_max_pos %lld",
@@ -281,9 +330,10 @@ nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int
   }
   if (V_out) {
     if (nq_status st = check_kv(V_out, vos, "V_out")) return st;
-    if (nq_status st = check_packed(v_in, "v_in")) return st;
+    if (nq_status st = check_store(v_in, exact, "v_in")) return st;
   }
   nq::DecodeLaunch L{};
+  L.exact = exact;
   if (K_out) L.k_in = *k_in;
   if (V_out) L.v_in = *v_in;
   L.units = units;
@@ -300,7 +350,31 @@ nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int
   L.V_out = V_out;
   L.vos = vos;
   return cuda_status(nq::launch_decode(L, reinterpret_cast<cudaStream_t>(stream)),
-                     "nq_decode launch");
+                     exact ? "nq_decode_exact launch" : "nq_decode launch");
+}
+
+nq_status nq_decode(const nq_packed* k_in, const nq_packed* v_in, int units, int heads,
+                    int64_t n, int64_t slot0, const int32_t* positions, int64_t pos_stride,
+                    int64_t pos_base, const float* rope_tab, int64_t rope_max_pos, void* K_out,
+                    nq_kv_strides kos, void* V_out, nq_kv_strides vos, nq_stream_t stream) {
+  return decode_impl(k_in, v_in, units, heads, n, slot0, positions, pos_stride, pos_base,
+                     rope_tab, rope_max_pos, K_out, kos, V_out, vos, false, stream);
+}
+
+nq_status nq_decode_exact(const nq_packed_exact* k_in, const nq_packed_exact* v_in, int units,
+                          int heads, int64_t n, int64_t slot0, const int32_t* positions,
+                          int64_t pos_stride, int64_t pos_base, const float* rope_tab,
+                          int64_t rope_max_pos, void* K_out, nq_kv_strides kos, void* V_out,
+                          nq_kv_strides vos, nq_stream_t stream) {
+  const nq_packed k = from_exact(k_in), v = from_exact(v_in);
+  return decode_impl(k_in ? &k : nullptr, v_in ? &v : nullptr, units, heads, n, slot0, positions,
+                     pos_stride, pos_base, rope_tab, rope_max_pos, K_out, kos, V_out, vos, true,
+                     stream);
+}
+
+int64_t nq_packed_exact_bytes_per_vector(int bits) {
+  if (bits != 2 && bits != 3) return -1;
+  return 4 * (4 * bits) + 2;
 }
 
 size_t nq_attend_workspace_bytes(int units, int heads, int G, int64_t n) {
@@ -372,6 +446,19 @@ nq_status nq_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* cod
   return cuda_status(nq::launch_e8_quantise(y, groups, bits, codes, coset,
                                             reinterpret_cast<cudaStream_t>(stream)),
                      "nq_e8_quantise launch");
+}
+
+nq_status nq_e8_box_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
+                             uint8_t* coset, nq_stream_t stream) {
+  if (bits != 2 && bits != 3) return fail(NQ_ERR_INVALID, "bits must be 2 or 3 (got %d)", bits);
+  if (groups < 0) return fail(NQ_ERR_INVALID, "groups must be >= 0");
+  if (groups == 0) return NQ_OK;
+  if (!y || !codes || !coset) return fail(NQ_ERR_INVALID, "y, codes and coset must be non-NULL");
+  if (!aligned(y, 4) || !aligned(codes, 4))
+    return fail(NQ_ERR_INVALID, "y and codes must be 4-byte aligned");
+  return cuda_status(nq::launch_e8_box_quantise(y, groups, bits, codes, coset,
+                                                reinterpret_cast<cudaStream_t>(stream)),
+                     "nq_e8_box_quantise launch");
 }
 
 int64_t nq_entropy_streams(int units, int heads, int64_t n) {

@@ -354,6 +354,89 @@ __device__ __forceinline__ void e8_codes(const float2 (&y)[8], bool halfx, bool 
   gy = ay & kMask;
 }
 
+// ------------------------------------------- E8 inside the code box (fp32x2)
+// The exact (24/16-bit) packing stores each group's coset bit in place of the
+// low bit of its last code, which needs every coded point in E8: the nearest
+// E8 point inside the b-bit code box, per coset the Conway-Sloane D8 step with
+// the box.  For two groups at once (lanes x, y) and one coset (shift 0, f in
+// [-(2^(b-1)-1), 2^(b-1)-1]; shift 1/2, f in [-2^(b-1), 2^(b-1)-1]):
+// u = y - shift, f = clamp(rint(u), lo, hi) (ties to even), e = u - f (exact),
+// d = e0^2 then an fma chain; when the sum of f is odd, the one coordinate
+// whose move by dir = (e >= 0 ? +1 : -1), reversed when that leaves the box,
+// costs least moves, cost fmaf(-2 dir, e, 1), the first index on ties, and d
+// gains that cost.  The half coset wins only when strictly closer.
+__device__ __forceinline__ void box_fix_lane(float (&f)[8], const float (&e)[8], float lo,
+                                             float hi, float& d) {
+  float best = 0.0f, kdir = 0.0f;
+  int k = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float dir = e[i] >= 0.0f ? 1.0f : -1.0f;
+    if (f[i] + dir > hi || f[i] + dir < lo) dir = -dir;
+    const float cost = __fmaf_rn(-2.0f * dir, e[i], 1.0f);
+    if (i == 0 || cost < best) {
+      best = cost;
+      k = i;
+      kdir = dir;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (i == k) f[i] = __fadd_rn(f[i], kdir);
+  d = __fadd_rn(d, best);
+}
+
+__device__ __forceinline__ void d8_box2(const float2 (&y)[8], float shift, float lo, float hi,
+                                        float (&fx)[8], float (&fy)[8], float& dx, float& dy) {
+  const float2 M2 = make_float2(kMagicRound, kMagicRound);
+  const float2 S2 = make_float2(-shift, -shift);
+  float ex[8], ey[8];
+  float2 d = make_float2(0.f, 0.f), sum = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 u = add2(y[i], S2);  // y + (-shift): the rounding of y - shift
+    const float2 r = sub2(add2(u, M2), M2);
+    const float2 f = make_float2(fminf(fmaxf(r.x, lo), hi), fminf(fmaxf(r.y, lo), hi));
+    const float2 e = sub2(u, f);
+    d = i == 0 ? mul2(e, e) : fma2(e, e, d);
+    sum = add2(sum, f);
+    fx[i] = f.x;
+    fy[i] = f.y;
+    ex[i] = e.x;
+    ey[i] = e.y;
+  }
+  const float2 b = add2(sum, M2);  // parity of the integer sum: LSB of the biased value
+  dx = d.x;
+  dy = d.y;
+  if (__float_as_uint(b.x) & 1u) box_fix_lane(fx, ex, lo, hi, dx);
+  if (__float_as_uint(b.y) & 1u) box_fix_lane(fy, ey, lo, hi, dy);
+}
+
+// Folded codes of two groups (lanes x, y) at their nearest E8 point inside the
+// box: code j = f - lo of the chosen coset at bits [b i, b i + b), then the low
+// bit of code 7 replaced by the coset bit (1 = half coset).
+template <int BITS>
+__device__ __forceinline__ void e8_box_codes(const float2 (&y)[8], uint32_t& gx, uint32_t& gy) {
+  constexpr float kH = static_cast<float>(1 << (BITS - 1));
+  float f0x[8], f0y[8], f1x[8], f1y[8], d0x, d0y, d1x, d1y;
+  d8_box2(y, 0.0f, 1.0f - kH, kH - 1.0f, f0x, f0y, d0x, d0y);
+  d8_box2(y, 0.5f, -kH, kH - 1.0f, f1x, f1y, d1x, d1y);
+  const bool hx = d1x < d0x, hy = d1y < d0y;
+  uint32_t ax = 0u, ay = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    // 2^23 + j, exact: the code sits in the low mantissa bits
+    const float jx = hx ? __fadd_rn(f1x[i], kH + kTwo23) : __fadd_rn(f0x[i], kH - 1.0f + kTwo23);
+    const float jy = hy ? __fadd_rn(f1y[i], kH + kTwo23) : __fadd_rn(f0y[i], kH - 1.0f + kTwo23);
+    ax += __float_as_uint(jx) << (BITS * i);
+    ay += __float_as_uint(jy) << (BITS * i);
+  }
+  constexpr uint32_t kMask = (1u << (8 * BITS)) - 1u;
+  constexpr uint32_t kCos = 1u << (7 * BITS);
+  gx = ((ax & kMask) & ~kCos) | (hx ? kCos : 0u);
+  gy = ((ay & kMask) & ~kCos) | (hy ? kCos : 0u);
+}
+
 // --------------------------------------------------------------- encode
 // Staged bf16 row -> this half's 64 coordinates; keys: RoPE removed.
 template <bool ROPE>
@@ -385,9 +468,11 @@ __device__ __forceinline__ void load_half(float2 (&v)[32], uint32_t row, uint32_
   }
 }
 
-template <int BITS>
+// Rotation, scale, E8 step and packing of this thread's half vector; the meta
+// word (regular layout) or the fp16 scale (exact layout) is written by half 0.
+template <int BITS, bool EXACT>
 __device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool valid,
-                                              uint32_t* codes, uint32_t* meta) {
+                                              uint32_t* codes, void* meta) {
   fwht_half(v, half);
   float m4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four chains for latency
 #pragma unroll
@@ -412,13 +497,17 @@ __device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool va
     float2 y[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[i] = mul2(v[8 * q + i], r2);
-    bool hx, hy, ox, oy;
-    e8_choose(y, big, hx, hy, ox, oy);
-    e8_codes<BITS>(y, hx, hy, ox, oy, gx[q], gy[q]);
-    cm |= (static_cast<uint32_t>(hx) << (4 * half + q)) |
-          (static_cast<uint32_t>(hy) << (8 + 4 * half + q));
+    if (EXACT) {
+      e8_box_codes<BITS>(y, gx[q], gy[q]);
+    } else {
+      bool hx, hy, ox, oy;
+      e8_choose(y, big, hx, hy, ox, oy);
+      e8_codes<BITS>(y, hx, hy, ox, oy, gx[q], gy[q]);
+      cm |= (static_cast<uint32_t>(hx) << (4 * half + q)) |
+            (static_cast<uint32_t>(hy) << (8 + 4 * half + q));
+    }
   }
-  cm |= __shfl_xor_sync(0xffffffffu, cm, 16);
+  if (!EXACT) cm |= __shfl_xor_sync(0xffffffffu, cm, 16);
   if (!valid) return;
   if (BITS == 3) {
     // groups 4h..4h+3 -> words 3h..3h+2; groups 8+4h.. -> words 6+3h..
@@ -444,10 +533,15 @@ __device__ __forceinline__ void quantise_half(float2 (&v)[32], int half, bool va
     *reinterpret_cast<uint2*>(codes + 4 + 2 * half) =
         make_uint2(gy[0] | (gy[1] << 16), gy[2] | (gy[3] << 16));
   }
-  if (half == 0) *meta = cm | (static_cast<uint32_t>(__half_as_ushort(sh)) << 16);
+  if (half == 0) {
+    if (EXACT)
+      *static_cast<uint16_t*>(meta) = __half_as_ushort(sh);
+    else
+      *static_cast<uint32_t*>(meta) = cm | (static_cast<uint32_t>(__half_as_ushort(sh)) << 16);
+  }
 }
 
-template <int BITS, bool ROPE>
+template <int BITS, bool ROPE, bool EXACT>
 __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int nthreads = blockDim.x;
@@ -552,7 +646,9 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const CodecArgs a) {
       cp_async_commit();
     }
     const int64_t vec = ep.unit * a.pu + h * a.ph + a.slot0 + ep.slot;
-    quantise_half<BITS>(v, half, ep.valid, a.codes + vec * (4 * BITS), a.meta + vec);
+    void* meta = EXACT ? static_cast<void*>(reinterpret_cast<uint16_t*>(a.meta) + vec)
+                       : static_cast<void*>(a.meta + vec);
+    quantise_half<BITS, EXACT>(v, half, ep.valid, a.codes + vec * (4 * BITS), meta);
   }
   cp_async_wait<0>();
 }
@@ -581,8 +677,34 @@ __device__ __forceinline__ void decode_half(const uint32_t (&w)[4 * BITS], uint3
   }
 }
 
-// Codes and meta of this thread's vector in tile t (registers, one tile ahead).
+// Exact layout -> regular layout in registers: each group's coset bit sits in
+// place of the low bit of its code 7, whose true value is the parity of codes
+// 0..6 (the codes of a point of E8 have an even sum).  Restores that bit in
+// the words and returns the regular meta word (coset mask | sigma << 16).
 template <int BITS>
+__device__ __forceinline__ uint32_t unfold_exact(uint32_t (&w)[4 * BITS], uint32_t sig16) {
+  uint32_t mask = 0u;
+#pragma unroll
+  for (int g = 0; g < 16; ++g) {
+    constexpr int kGB = 8 * BITS;  // bits per group
+    const int p = kGB * g;
+    const int wi = p >> 5, off = p & 31;
+    const int wn = wi + 1 < 4 * BITS ? wi + 1 : wi;
+    const uint32_t G = (off + kGB <= 32 ? (w[wi] >> off) : __funnelshift_r(w[wi], w[wn], off)) &
+                       ((1u << kGB) - 1u);
+    // low bits of codes 0..6: 0x49249 (3-bit fields), 0x1555 (2-bit fields)
+    constexpr uint32_t kLsb = BITS == 3 ? 0x49249u : 0x1555u;
+    const uint32_t h = (G >> (7 * BITS)) & 1u;
+    const uint32_t par = __popc(G & kLsb) & 1u;
+    const int q = p + 7 * BITS;
+    w[q >> 5] ^= (h ^ par) << (q & 31);
+    mask |= h << g;
+  }
+  return mask | (sig16 << 16);
+}
+
+// Codes and meta of this thread's vector in tile t (registers, one tile ahead).
+template <int BITS, bool EXACT>
 __device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int warp, int slot_l,
                                            uint32_t (&w)[4 * BITS], uint32_t& meta) {
   const Tile tl = tile_of(a, t);
@@ -599,7 +721,10 @@ __device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int wa
       w[4 * c + 2] = q.z;
       w[4 * c + 3] = q.w;
     }
-    meta = __ldg(a.meta + vec);
+    if (EXACT)
+      meta = unfold_exact<BITS>(w, __ldg(reinterpret_cast<const unsigned short*>(a.meta) + vec));
+    else
+      meta = __ldg(a.meta + vec);
   }
 }
 
@@ -608,7 +733,7 @@ __device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int wa
 // store: 16-byte chunk c of row r sits at chunk (c ^ (r % 8)) of its box row.
 constexpr int kOutTileBytes = 2 * kSlots * 128;
 
-template <int BITS, bool ROPE>
+template <int BITS, bool ROPE, bool EXACT>
 __global__ void __launch_bounds__(256, 2)
     decode_kernel(const CodecArgs a, const __grid_constant__ CUtensorMap out_map) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -646,7 +771,7 @@ __global__ void __launch_bounds__(256, 2)
     __syncthreads();
     if (my_tiles > 0) combine_rope_rows(raw_of(0), cs_of(0), tid, nthreads);
   }
-  if (my_tiles > 0) load_codes<BITS>(a, first, warp, slot_l, w, meta);
+  if (my_tiles > 0) load_codes<BITS, EXACT>(a, first, warp, slot_l, w, meta);
 
   for (int64_t k = 0; k < my_tiles; ++k) {
     if (ROPE) {
@@ -664,7 +789,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
     for (int i = 0; i < 4 * BITS; ++i) wc[i] = w[i];
     const uint32_t mc = meta;
-    if (k + 1 < my_tiles) load_codes<BITS>(a, first + (k + 1) * step, warp, slot_l, w, meta);
+    if (k + 1 < my_tiles) load_codes<BITS, EXACT>(a, first + (k + 1) * step, warp, slot_l, w, meta);
     // the warp's previous tensor store has finished reading the tile
     if (lane == 0) bulk_wait_read_all();
     __syncwarp();
@@ -726,7 +851,7 @@ static cudaError_t make_out_map(CUtensorMap* m, const CodecArgs& a, int units) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BITS, bool ROPE>
+template <int BITS, bool ROPE, bool EXACT>
 static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t stream) {
   a.hg = pick_head_group(a.heads);
   a.ngroups = a.heads / a.hg;
@@ -754,10 +879,10 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
     if (e != cudaSuccess) return e;
     smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes +
            (ROPE ? 2 * kCsBytes + 2 * kRawBytes : 0);
-    fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE>);
+    fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE, EXACT>);
   } else {
     smem = 2 * (static_cast<size_t>(rows_bytes) + (ROPE ? kCsBytes : 0)) + (ROPE ? kRawBytes : 0);
-    fn = reinterpret_cast<const void*>(encode_kernel<BITS, ROPE>);
+    fn = reinterpret_cast<const void*>(encode_kernel<BITS, ROPE, EXACT>);
   }
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -772,19 +897,26 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   if (per_sm < 1) per_sm = 1;
   const int64_t grid = min64(a.num_tiles, static_cast<int64_t>(sms) * per_sm);
   if (decode)
-    decode_kernel<BITS, ROPE><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a, map);
+    decode_kernel<BITS, ROPE, EXACT><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a, map);
   else
-    encode_kernel<BITS, ROPE><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
+    encode_kernel<BITS, ROPE, EXACT><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-static cudaError_t launch_kind(bool decode, const CodecArgs& a, int bits, bool rope, int units,
-                               cudaStream_t stream) {
+static cudaError_t launch_kind(bool decode, const CodecArgs& a, int bits, bool rope, bool exact,
+                               int units, cudaStream_t stream) {
+  if (exact) {
+    if (bits == 3)
+      return rope ? launch_one<3, true, true>(decode, a, units, stream)
+                  : launch_one<3, false, true>(decode, a, units, stream);
+    return rope ? launch_one<2, true, true>(decode, a, units, stream)
+                : launch_one<2, false, true>(decode, a, units, stream);
+  }
   if (bits == 3)
-    return rope ? launch_one<3, true>(decode, a, units, stream)
-                : launch_one<3, false>(decode, a, units, stream);
-  return rope ? launch_one<2, true>(decode, a, units, stream)
-              : launch_one<2, false>(decode, a, units, stream);
+    return rope ? launch_one<3, true, false>(decode, a, units, stream)
+                : launch_one<3, false, false>(decode, a, units, stream);
+  return rope ? launch_one<2, true, false>(decode, a, units, stream)
+              : launch_one<2, false, false>(decode, a, units, stream);
 }
 
 cudaError_t codec_read_clear_error(uint32_t* flags) {
@@ -826,7 +958,7 @@ cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream) {
     k.meta = L.k_out.meta;
     k.pu = L.k_out.unit_stride;
     k.ph = L.k_out.head_stride;
-    cudaError_t err = launch_kind(false, k, L.k_out.bits, true, L.units, stream);
+    cudaError_t err = launch_kind(false, k, L.k_out.bits, true, L.exact, L.units, stream);
     if (err != cudaSuccess) return err;
   }
   if (L.V) {
@@ -839,7 +971,7 @@ cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream) {
     v.meta = L.v_out.meta;
     v.pu = L.v_out.unit_stride;
     v.ph = L.v_out.head_stride;
-    return launch_kind(false, v, L.v_out.bits, false, L.units, stream);
+    return launch_kind(false, v, L.v_out.bits, false, L.exact, L.units, stream);
   }
   return cudaSuccess;
 }
@@ -857,7 +989,7 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
     k.meta = L.k_in.meta;
     k.pu = L.k_in.unit_stride;
     k.ph = L.k_in.head_stride;
-    cudaError_t err = launch_kind(true, k, L.k_in.bits, true, L.units, stream);
+    cudaError_t err = launch_kind(true, k, L.k_in.bits, true, L.exact, L.units, stream);
     if (err != cudaSuccess) return err;
   }
   if (L.V_out) {
@@ -870,17 +1002,19 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
     v.meta = L.v_in.meta;
     v.pu = L.v_in.unit_stride;
     v.ph = L.v_in.head_stride;
-    return launch_kind(true, v, L.v_in.bits, false, L.units, stream);
+    return launch_kind(true, v, L.v_in.bits, false, L.exact, L.units, stream);
   }
   return cudaSuccess;
 }
 
 // ------------------------------------------------------ E8 quantiser alone
 // One thread per pair of groups (2p in lane x, 2p + 1 in lane y) of a
-// [groups][8] fp32 array, with the encode kernel's decision and code
-// functions.  The CTA loop bound is uniform across each warp (threads past
-// the end run on zeros), as the warp vote in e8_choose needs.
-template <int BITS>
+// [groups][8] fp32 array, with the encode kernels' decision and code
+// functions: the regular step (nearest point, then clamp) or, with BOX, the
+// nearest point inside the code box with the coset bit folded into code 7.
+// The CTA loop bound is uniform across each warp (threads past the end run on
+// zeros), as the warp vote in e8_choose needs.
+template <int BITS, bool BOX>
 __global__ void __launch_bounds__(256) e8_quantise_kernel(const float* __restrict__ y,
                                                           int64_t groups, uint32_t* codes,
                                                           uint8_t* coset) {
@@ -902,10 +1036,17 @@ __global__ void __launch_bounds__(256) e8_quantise_kernel(const float* __restric
       yy[i] = make_float2(a[i], b[i]);
       big = fmaxf(big, fmaxf(fabsf(a[i]), fabsf(b[i])));
     }
-    bool hx, hy, ox, oy;
-    e8_choose(yy, !(big < 7.0f), hx, hy, ox, oy);
     uint32_t cx, cy;
-    e8_codes<BITS>(yy, hx, hy, ox, oy, cx, cy);
+    bool hx, hy;
+    if (BOX) {
+      e8_box_codes<BITS>(yy, cx, cy);
+      hx = (cx >> (7 * BITS)) & 1u;
+      hy = (cy >> (7 * BITS)) & 1u;
+    } else {
+      bool ox, oy;
+      e8_choose(yy, !(big < 7.0f), hx, hy, ox, oy);
+      e8_codes<BITS>(yy, hx, hy, ox, oy, cx, cy);
+    }
     if (g0 < groups) {
       codes[g0] = cx;
       coset[g0] = hx ? 1 : 0;
@@ -917,8 +1058,9 @@ __global__ void __launch_bounds__(256) e8_quantise_kernel(const float* __restric
   }
 }
 
-cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
-                               uint8_t* coset, cudaStream_t stream) {
+template <bool BOX>
+static cudaError_t launch_e8(const float* y, int64_t groups, int bits, uint32_t* codes,
+                             uint8_t* coset, cudaStream_t stream) {
   if (groups <= 0) return cudaSuccess;
   int dev = 0, sms = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -928,10 +1070,22 @@ cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_
   const int64_t pairs = (groups + 1) / 2;
   const int64_t grid = min64((pairs + 255) / 256, static_cast<int64_t>(sms) * 8);
   if (bits == 3)
-    e8_quantise_kernel<3><<<static_cast<unsigned>(grid), 256, 0, stream>>>(y, groups, codes, coset);
+    e8_quantise_kernel<3, BOX><<<static_cast<unsigned>(grid), 256, 0, stream>>>(y, groups, codes,
+                                                                                coset);
   else
-    e8_quantise_kernel<2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(y, groups, codes, coset);
+    e8_quantise_kernel<2, BOX><<<static_cast<unsigned>(grid), 256, 0, stream>>>(y, groups, codes,
+                                                                                coset);
   return cudaGetLastError();
+}
+
+cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
+                               uint8_t* coset, cudaStream_t stream) {
+  return launch_e8<false>(y, groups, bits, codes, coset, stream);
+}
+
+cudaError_t launch_e8_box_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
+                                   uint8_t* coset, cudaStream_t stream) {
+  return launch_e8<true>(y, groups, bits, codes, coset, stream);
 }
 
 }  // namespace nq

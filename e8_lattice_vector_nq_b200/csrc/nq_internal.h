@@ -31,12 +31,14 @@ struct EncodeLaunch {
   int64_t pos_base;
   const float* rope_tab;
   int64_t rope_max_pos;
-  nq_packed k_out, v_out;
+  nq_packed k_out, v_out;  // exact layout: meta points to the uint16 scales
   int64_t slot0;
+  bool exact;
 };
 
 struct DecodeLaunch {
-  nq_packed k_in, v_in;
+  nq_packed k_in, v_in;  // exact layout: meta points to the uint16 scales
+  bool exact;
   int units, heads;
   int64_t n, slot0;
   const int32_t* positions;
@@ -74,6 +76,8 @@ int64_t attend_ctas(int units, int heads, int64_t n);  // CTAs of the partial ke
 cudaError_t launch_attend(const AttendLaunch& L, cudaStream_t stream);
 cudaError_t launch_e8_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
                                uint8_t* coset, cudaStream_t stream);
+cudaError_t launch_e8_box_quantise(const float* y, int64_t groups, int bits, uint32_t* codes,
+                                   uint8_t* coset, cudaStream_t stream);
 
 int64_t entropy_streams(int units, int heads, int64_t n);
 int64_t entropy_max_words(int units, int heads, int64_t n);

@@ -36,6 +36,12 @@ class Packed(ctypes.Structure):
                 ("bits", ctypes.c_int32)]
 
 
+class PackedExact(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("sigma", ctypes.c_void_p),
+                ("unit_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64),
+                ("bits", ctypes.c_int32)]
+
+
 _lib = None
 
 EXPORTS = (
@@ -45,6 +51,8 @@ EXPORTS = (
     "nq_select", "nq_encode", "nq_decode", "nq_e8_quantise", "nq_attend_workspace_bytes",
     "nq_attend", "nq_device_error", "nq_entropy_streams", "nq_entropy_max_words",
     "nq_entropy_workspace_bytes", "nq_entropy_encode", "nq_entropy_decode",
+    "nq_packed_exact_bytes_per_vector", "nq_encode_exact", "nq_decode_exact",
+    "nq_e8_box_quantise",
 )
 
 
@@ -58,6 +66,7 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(SO_PATH)
     P, i64, i32, sz, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_double
     PK = ctypes.POINTER(Packed)
+    PX = ctypes.POINTER(PackedExact)
     sig = {
         "nq_last_error": (ctypes.c_char_p, []),
         "nq_version": (i32, []),
@@ -83,6 +92,12 @@ def lib() -> ctypes.CDLL:
         "nq_entropy_workspace_bytes": (sz, [i32, i32, i64]),
         "nq_entropy_encode": (i32, [PK, i32, i32, i64, i64, i32, P, P, P, i64, P, sz, P]),
         "nq_entropy_decode": (i32, [P, P, P, i32, i32, i64, i32, PK, i64, P]),
+        "nq_packed_exact_bytes_per_vector": (i64, [i32]),
+        "nq_encode_exact": (i32, [P, KVStrides, P, KVStrides, i32, i32, i64, i64, P, i64, i64, P,
+                                  i64, PX, PX, i64, P]),
+        "nq_decode_exact": (i32, [PX, PX, i32, i32, i64, i64, P, i64, i64, P, i64, P, KVStrides,
+                                  P, KVStrides, P]),
+        "nq_e8_box_quantise": (i32, [P, i64, i32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -155,6 +170,43 @@ class PackedStore:
     @property
     def nbytes(self) -> int:
         return self.codes.numel() * 4 + self.meta.numel() * 4
+
+
+@dataclass
+class ExactStore:
+    """Device arrays of one exact-layout store (nq.h, nq_packed_exact): codes
+    [units][heads][cap][4*bits] (uint32 words in an int32 tensor; the low bit
+    of code 8g+7 holds group g's coset bit) and sigma [units][heads][cap]
+    (fp16 scale bits in an int16 tensor)."""
+
+    codes: torch.Tensor
+    sigma: torch.Tensor
+    bits: int
+
+    @classmethod
+    def empty(cls, units: int, heads: int, cap: int, bits: int, device="cuda") -> "ExactStore":
+        codes = torch.empty(units, heads, cap, 4 * bits, dtype=torch.int32, device=device)
+        sigma = torch.empty(units, heads, cap, dtype=torch.int16, device=device)
+        return cls(codes, sigma, bits)
+
+    def select_units(self, sl) -> "ExactStore":
+        return ExactStore(self.codes[sl], self.sigma[sl], self.bits)
+
+    def desc(self) -> PackedExact:
+        assert self.codes.stride(1) == self.sigma.stride(1) * 4 * self.bits
+        assert self.codes.stride(0) == self.sigma.stride(0) * 4 * self.bits
+        return PackedExact(self.codes.data_ptr(), self.sigma.data_ptr(), self.sigma.stride(0),
+                           self.sigma.stride(1), self.bits)
+
+    def codes_store(self) -> PackedStore:
+        """The codes as an nq_packed for the entropy stage (which reads codes
+        only; the meta array given is a placeholder that is never read)."""
+        meta = torch.empty(self.sigma.shape, dtype=torch.int32, device=self.codes.device)
+        return PackedStore(self.codes, meta, self.bits)
+
+    @property
+    def nbytes(self) -> int:
+        return self.codes.numel() * 4 + self.sigma.numel() * 2
 
 
 # -------------------------------------------------------------- RoPE tables
@@ -280,6 +332,63 @@ def nq_decode(k_in: PackedStore | None, v_in: PackedStore | None, n: int,
                            vos, _stream(stream)))
 
 
+def nq_encode_exact(K: torch.Tensor | None, V: torch.Tensor | None, k_out: ExactStore | None,
+                    v_out: ExactStore | None, n: int, rope_tab: torch.Tensor | None = None,
+                    rope_max_pos: int = 0, kept: torch.Tensor | None = None, pos_base: int = 0,
+                    slot0: int = 0, stream=None):
+    """nq_encode into exact-layout stores (see nq.h, nq_encode_exact)."""
+    _require_device_readable(K, V)
+    _require_cuda(kept, rope_tab)
+    ref = K if K is not None else V
+    units, heads, T_in, _ = ref.shape
+    kd = k_out.desc() if K is not None else None
+    vd = v_out.desc() if V is not None else None
+    ks = kv_strides(K) if K is not None else KVStrides(0, 0, 0)
+    vs = kv_strides(V) if V is not None else KVStrides(0, 0, 0)
+    if kept is not None:
+        assert kept.dtype == torch.int32 and kept.stride(-1) == 1
+    for st in (k_out if K is not None else None, v_out if V is not None else None):
+        if st is not None and (st.sigma.shape[0] < units or st.sigma.shape[1] < heads
+                               or st.sigma.shape[2] < slot0 + n):
+            raise ValueError("exact store too small for units x heads x (slot0 + n)")
+    _check(lib().nq_encode_exact(_ptr(K), ks, _ptr(V), vs, units, heads, T_in, int(n), _ptr(kept),
+                                 kept.stride(0) if kept is not None else 0, int(pos_base),
+                                 _ptr(rope_tab), int(rope_max_pos),
+                                 ctypes.byref(kd) if kd is not None else None,
+                                 ctypes.byref(vd) if vd is not None else None, int(slot0),
+                                 _stream(stream)))
+
+
+def nq_decode_exact(k_in: ExactStore | None, v_in: ExactStore | None, n: int,
+                    K_out: torch.Tensor | None, V_out: torch.Tensor | None,
+                    rope_tab: torch.Tensor | None = None, rope_max_pos: int = 0,
+                    positions: torch.Tensor | None = None, pos_base: int = 0, slot0: int = 0,
+                    stream=None):
+    """nq_decode from exact-layout stores (see nq.h, nq_decode_exact)."""
+    _require_cuda(K_out, V_out, positions, rope_tab)
+    ref = K_out if K_out is not None else V_out
+    units, heads = ref.shape[0], ref.shape[1]
+    kd = k_in.desc() if K_out is not None else None
+    vd = v_in.desc() if V_out is not None else None
+    kos = kv_strides(K_out) if K_out is not None else KVStrides(0, 0, 0)
+    vos = kv_strides(V_out) if V_out is not None else KVStrides(0, 0, 0)
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.stride(-1) == 1
+    for st in (k_in if K_out is not None else None, v_in if V_out is not None else None):
+        if st is not None and (st.sigma.shape[0] < units or st.sigma.shape[1] < heads
+                               or st.sigma.shape[2] < slot0 + n):
+            raise ValueError("exact store too small for units x heads x (slot0 + n)")
+    for o in (K_out, V_out):
+        if o is not None and o.shape[2] < n:
+            raise ValueError("output has fewer than n tokens")
+    _check(lib().nq_decode_exact(ctypes.byref(kd) if kd is not None else None,
+                                 ctypes.byref(vd) if vd is not None else None, units, heads,
+                                 int(n), int(slot0), _ptr(positions),
+                                 positions.stride(0) if positions is not None else 0,
+                                 int(pos_base), _ptr(rope_tab), int(rope_max_pos), _ptr(K_out),
+                                 kos, _ptr(V_out), vos, _stream(stream)))
+
+
 def nq_attend(q: torch.Tensor, k_in: PackedStore, v_in: PackedStore, n: int, G: int,
               rope_tab: torch.Tensor, rope_max_pos: int, scale: float | None = None,
               positions: torch.Tensor | None = None, pos_base: int = 0, slot0: int = 0,
@@ -322,6 +431,21 @@ def nq_e8_quantise(y: torch.Tensor, bits: int, stream=None):
     codes = torch.empty(g, dtype=torch.int32, device=y.device)
     coset = torch.empty(g, dtype=torch.uint8, device=y.device)
     _check(lib().nq_e8_quantise(_ptr(y), g, int(bits), _ptr(codes), _ptr(coset), _stream(stream)))
+    return codes, coset
+
+
+def nq_e8_box_quantise(y: torch.Tensor, bits: int, stream=None):
+    """The exact layout's lattice step alone on [groups][8] fp32 rows (device):
+    returns (codes int32 [groups] with the coset bit in the low bit of code 7,
+    coset uint8 [groups])."""
+    _require_cuda(y)
+    if y.dtype != torch.float32 or y.dim() != 2 or y.shape[1] != 8 or not y.is_contiguous():
+        raise ValueError("y must be a contiguous float32 [groups, 8] tensor")
+    g = y.shape[0]
+    codes = torch.empty(g, dtype=torch.int32, device=y.device)
+    coset = torch.empty(g, dtype=torch.uint8, device=y.device)
+    _check(lib().nq_e8_box_quantise(_ptr(y), g, int(bits), _ptr(codes), _ptr(coset),
+                                    _stream(stream)))
     return codes, coset
 
 

@@ -219,6 +219,54 @@ nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int
                     int64_t pos_base, const float *rope_tab, int64_t rope_max_pos, void *K_out,
                     nq_kv_strides kos, void *V_out, nq_kv_strides vos, nq_stream_t stream);
 
+/* --------------------------------------- exact (24/16-bit) index packing
+ * The lattice step at exactly b bits per coordinate plus the scale ([NQ-pt]
+ * step 5 stores the E8 indices at "2 bits/dim"): the coset bit of each group
+ * rides in the low bit of the group's last code, which a point of E8 does
+ * not need -- its codes j = q + 2^(b-1) - 1 (integer coset) or
+ * j = (q - 1/2) + 2^(b-1) (half coset) have an even sum, so the low bit of
+ * j_7 is the parity of j_0 .. j_6.  This needs every coded point in E8, so the
+ * lattice step is the nearest E8 point INSIDE the b-bit code box (the
+ * library's parity-preserving reading of the clamp), per coset:
+ *   u = y - shift (shift 0: f in [-(2^(b-1)-1), 2^(b-1)-1];
+ *                  shift 1/2: f in [-2^(b-1), 2^(b-1)-1]),
+ *   f_i = clamp(rint(u_i), lo, hi) (ties to even), e_i = u_i - f_i,
+ *   d = e_0^2 then fmaf chain; when sum f is odd the one coordinate whose move
+ *   by dir = (e >= 0 ? +1 : -1), reversed when that leaves the box, costs
+ *   least -- cost fmaf(-2 dir, e, 1), first index on ties -- moves, d += cost;
+ *   the half coset wins only when d1 < d0.
+ * It equals nq_encode's point whenever that point lies in the box.
+ * Layout (nq_packed_exact): codes as in nq_packed (4*bits uint32 words per
+ * vector, code c at bits [b*c, b*c + b)), except that the low bit of code
+ * 8g+7 holds group g's coset bit (1 = half coset); sigma: one fp16 scale per
+ * vector (uint16, 2-byte aligned).  4*(4*bits) + 2 bytes per vector: 50 for
+ * K3 (3.125 bits per coordinate), 34 for V2 (2.125).
+ * nq_encode_exact / nq_decode_exact take the same arguments, with the same
+ * rules and errors, as nq_encode / nq_decode, with exact-layout stores; the
+ * steps before and after the lattice step are theirs.  Decode restores each
+ * code 7's low bit from the parity of codes 0..6.  The codes of an exact
+ * store can go through nq_entropy_encode / nq_entropy_decode as they are (an
+ * nq_packed with the same codes, strides and bits; its meta is not read). */
+typedef struct {
+    uint32_t *codes;
+    uint16_t *sigma;
+    int64_t unit_stride;
+    int64_t head_stride;
+    int32_t bits; /* 2 or 3 */
+} nq_packed_exact;
+
+int64_t nq_packed_exact_bytes_per_vector(int bits);
+nq_status nq_encode_exact(const void *K, nq_kv_strides ks, const void *V, nq_kv_strides vs,
+                          int units, int heads, int64_t T_in, int64_t n, const int32_t *kept,
+                          int64_t kept_stride, int64_t pos_base, const float *rope_tab,
+                          int64_t rope_max_pos, const nq_packed_exact *k_out,
+                          const nq_packed_exact *v_out, int64_t slot0, nq_stream_t stream);
+nq_status nq_decode_exact(const nq_packed_exact *k_in, const nq_packed_exact *v_in, int units,
+                          int heads, int64_t n, int64_t slot0, const int32_t *positions,
+                          int64_t pos_stride, int64_t pos_base, const float *rope_tab,
+                          int64_t rope_max_pos, void *K_out, nq_kv_strides kos, void *V_out,
+                          nq_kv_strides vos, nq_stream_t stream);
+
 /* ----------------------------------------------------- decode attention
  * Decode-phase attention over the packed cache, reconstructing keys and
  * values inside the attention (the on-demand reconstruction within
@@ -304,6 +352,14 @@ nq_status nq_entropy_decode(const uint16_t *words, const uint32_t *offsets, cons
  * values are out of contract (no fault, unspecified codes). */
 nq_status nq_e8_quantise(const float *y, int64_t groups, int bits, uint32_t *codes,
                          uint8_t *coset, nq_stream_t stream);
+
+/* The lattice step of nq_encode_exact on its own: each row of y is snapped
+ * to the nearest E8 point inside the b-bit code box (see nq_encode_exact),
+ * codes[g] holds its 8 codes (code i at bits [b*i, b*i + b)) with the low
+ * bit of code 7 replaced by the coset bit, coset[g] the coset (1 = half).
+ * Same arguments, alignment rules and errors as nq_e8_quantise. */
+nq_status nq_e8_box_quantise(const float *y, int64_t groups, int bits, uint32_t *codes,
+                             uint8_t *coset, nq_stream_t stream);
 
 /* -------------------------------------------------------------- status
  * Reads and clears the device error word reserved for in-kernel failure

@@ -99,18 +99,25 @@ def kept_set_parity(s_or: np.ndarray, kept_or: np.ndarray, kept_gpu: np.ndarray,
             "kept_unexcused": int((~near).sum())}
 
 
-def _codes_parity(oq, x_rows, gw, gm, ow, om, bits, rope, c, s):
-    """One store (keys or values): compare [N][4b] words and [N] meta words."""
+def _codes_parity(oq, x_rows, gw, gm, ow, om, bits, rope, c, s, exact=False):
+    """One store (keys or values): compare [N][4b] words and [N] meta words
+    (exact layout: [N] fp16 scales, and no mismatch is excused: the margins
+    describe the regular step's decisions, not the box step's)."""
     bad = np.nonzero(np.any(gw != ow, axis=1) | (gm != om))[0]
     res = {"vectors": int(gm.size), "mismatch_vectors": int(bad.size), "mismatch_codes": 0,
            "excused_codes": 0, "unexcused_codes": 0}
     if bad.size:
         gc, oc = code_fields(gw[bad], bits), code_fields(ow[bad], bits)
-        per_vec = (gc != oc).sum(axis=1) + 128 * ((gm[bad] & 0xFFFF0000) != (om[bad] & 0xFFFF0000))
+        hi = 0xFFFF if exact else 0xFFFF0000
+        per_vec = (gc != oc).sum(axis=1) + 128 * ((gm[bad] & hi) != (om[bad] & hi))
         per_vec = np.maximum(per_vec, (gm[bad] != om[bad]).astype(np.int64))
-        mg = oq.encode_margins(x_rows[bad], bits, rope=rope,
-                               c=None if c is None else c[bad], s=None if s is None else s[bad])
-        near = mg <= EXCUSE_REL
+        if exact:
+            near = np.zeros(bad.size, bool)
+        else:
+            mg = oq.encode_margins(x_rows[bad], bits, rope=rope,
+                                   c=None if c is None else c[bad],
+                                   s=None if s is None else s[bad])
+            near = mg <= EXCUSE_REL
         res["mismatch_codes"] = int(per_vec.sum())
         res["excused_codes"] = int(per_vec[near].sum())
         res["unexcused_codes"] = int(per_vec[~near].sum())
@@ -126,6 +133,9 @@ def check_layer(job: dict) -> dict:
     gpu_scores [T] fp64 (evicting units), gpu_kept [n] int32 (or None: slots
                are tokens 0..n-1)
     gk_codes [H][n][4 bk], gk_meta [H][n], gv_codes, gv_meta  (GPU store)
+    exact      True for an exact-layout store (gk_meta / gv_meta then hold
+               the fp16 scales; the oracle side is its box-constrained
+               encoder folded into that layout)
     gK, gV     [H][n][128] uint16 GPU decode output (optional)
     Returns counts (see module doc) and the oracle's seconds."""
     import oracle as oq
@@ -152,19 +162,27 @@ def check_layer(job: dict) -> dict:
     Vx = V[:, src].reshape(-1, 128)
     c, s = oq.rope_cs(theta, pos_base + src)
     c, s = np.tile(c, (H, 1)), np.tile(s, (H, 1))
-    kw, km, _ = oq.encode_vectors(Kx, bk, rope=True, c=c, s=s)
-    vw, vm, _ = oq.encode_vectors(Vx, bv)
+    exact = bool(job.get("exact", False))
+    if exact:  # box-constrained step, folded into the exact layout
+        kw, km = oq.fold_exact(*oq.encode_vectors_box(Kx, bk, rope=True, c=c, s=s), bk)
+        vw, vm = oq.fold_exact(*oq.encode_vectors_box(Vx, bv), bv)
+    else:
+        kw, km, _ = oq.encode_vectors(Kx, bk, rope=True, c=c, s=s)
+        vw, vm, _ = oq.encode_vectors(Vx, bv)
     t_oracle = time.perf_counter() - t0
     rk, bad_k = _codes_parity(oq, Kx, job["gk_codes"].reshape(-1, 4 * bk),
-                              job["gk_meta"].reshape(-1), kw, km, bk, True, c, s)
+                              job["gk_meta"].reshape(-1), kw, km, bk, True, c, s, exact)
     rv, bad_v = _codes_parity(oq, Vx, job["gv_codes"].reshape(-1, 4 * bv),
-                              job["gv_meta"].reshape(-1), vw, vm, bv, False, None, None)
+                              job["gv_meta"].reshape(-1), vw, vm, bv, False, None, None, exact)
     out["vectors"] = rk["vectors"] + rv["vectors"]
     out["elements"] = 128 * out["vectors"]
     for key in ("mismatch_vectors", "mismatch_codes", "excused_codes", "unexcused_codes"):
         out[key] = rk[key] + rv[key]
     if job.get("gK") is not None:
         t1 = time.perf_counter()
+        if exact:
+            kw, km = oq.unfold_exact(kw, km, bk)
+            vw, vm = oq.unfold_exact(vw, vm, bv)
         Ko = oq.decode_vectors(kw, km, bk, rope=True, c=c, s=s)
         Vo = oq.decode_vectors(vw, vm, bv)
         t_oracle += time.perf_counter() - t1

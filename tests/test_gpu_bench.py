@@ -70,6 +70,14 @@ def test_reconstruction_diagnostic(line):
     assert 0.85 < r["v"]["cosine_mean"] <= 1.0 and 0.0 < r["v"]["rel_l2_mean"] < 0.6
 
 
+def test_exact_layout_block(line):
+    x = line["exact_layout"]
+    assert x["encode_ms"] > 0 and x["decode_ms"] > 0
+    assert x["bits_per_coordinate"] == {"k": 3.125, "v": 2.125}
+    assert x["bits_per_elem"] < line["bits_per_elem"]
+    assert x["rooflines"]["encode"]["frac"] > 0
+
+
 def test_optional_blocks(line):
     a = line["decode_attention"]
     assert a["fused_ms"] > 0 and a["decode_then_sdpa_ms"] > 0

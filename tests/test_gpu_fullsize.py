@@ -18,6 +18,9 @@ full against the CPU oracle on all host cores (oracle/parity.py):
                   of layer s mod 32 at steps 0, 1, 31 and 255 for those
                   sequences (a sample, stated as such)
 
+The exact (24/16-bit) layout is checked the same way on every layer of the
+Mistral- and Llama-shaped caches (no mismatch is excused there).
+
 Parity rule (the benchmark spec): kept sets and codes bit-exact except where the
 oracle's value lies within 1e-5 relative of a decision boundary; those are
 counted, reported and must stay below 1e-6 of the elements; decoded bf16
@@ -233,3 +236,53 @@ def test_decode_append_full(nq, pool):
                            gv_meta=u32(vm[s, l, :, :n]), gK=per_seq[s][0], gV=per_seq[s][1])
 
     assert_parity(wl.name, parity.run_jobs(pool, jobs()))
+
+
+def run_exact(nq, wl, pool):
+    """The exact (24/16-bit) layout over the whole cache in one call per stage
+    (scores, selection, nq_encode_exact, nq_decode_exact), every layer checked
+    against the oracle's box-constrained encoder folded into that layout."""
+    from oracle import parity
+
+    K, V = gen_cache(wl)
+    L, H, T = wl.layers, wl.heads, wl.tokens
+    evict = wl.evict_pct > 0 and T > 1 + wl.window
+    kept, scores, n = None, None, T
+    if evict:
+        scores = nq.nq_score(K, wl.window)
+        kept = nq.nq_select(scores, wl.window, wl.evict_pct)
+        n = kept.shape[1]
+    rope = nq.rope_tables(wl.theta, T)
+    ks = nq.ExactStore.empty(L, H, n, wl.bits_k)
+    vs = nq.ExactStore.empty(L, H, n, wl.bits_v)
+    nq.nq_encode_exact(K, V, ks, vs, n, rope, T, kept=kept)
+    Kd = torch.empty(L, H, n, 128, dtype=torch.bfloat16, device="cuda")
+    Vd = torch.empty_like(Kd)
+    nq.nq_decode_exact(ks, vs, n, Kd, Vd, rope, T, positions=kept)
+    torch.cuda.synchronize()
+    assert nq.device_error() == 0
+
+    def jobs():
+        for l in range(L):
+            yield {"K": u16(K[l]), "V": u16(V[l]), "theta": wl.theta, "bits_k": wl.bits_k,
+                   "bits_v": wl.bits_v, "window": wl.window, "pct": wl.evict_pct if evict else 0,
+                   "exact": True,
+                   "gpu_scores": scores[l].cpu().numpy() if evict else None,
+                   "gpu_kept": kept[l].cpu().numpy() if evict else None,
+                   "gk_codes": u32(ks.codes[l]),
+                   "gk_meta": ks.sigma[l].cpu().numpy().view(np.uint16),
+                   "gv_codes": u32(vs.codes[l]),
+                   "gv_meta": vs.sigma[l].cpu().numpy().view(np.uint16),
+                   "gK": u16(Kd[l]), "gV": u16(Vd[l])}
+
+    return parity.run_jobs(pool, jobs())
+
+
+def test_mistral7b_32k_exact_layout_full(nq, pool):
+    wl = synth.WORKLOADS["mistral7b_32k"]
+    assert_parity(wl.name + ":exact", run_exact(nq, wl, pool))
+
+
+def test_llama3_8b_128k_exact_layout_full(nq, pool):
+    wl = synth.WORKLOADS["llama3_8b_128k"]
+    assert_parity(wl.name + ":exact", run_exact(nq, wl, pool))

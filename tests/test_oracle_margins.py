@@ -160,3 +160,29 @@ def test_parity_jobs_run_in_spawn_workers(oq):
     assert tot["units"] == 3 and tot["vectors"] == 3 * 2 * 8 * 40
     assert tot["mismatch_vectors"] == 1 and tot["unexcused_codes"] == 1
     assert parity.verdict(tot) and "code mismatches" in parity.verdict(tot)[0]
+
+
+def test_parity_counts_exact_layout(oq):
+    """The exact-layout path of the accounting: the oracle's own folded
+    store passes; one flipped coset bit (the low bit of a code 7) fails."""
+    import torch
+
+    from oracle import parity
+
+    wl = synth.WORKLOADS["tiny"]
+    K, V = synth.gen_layer(wl, 0, "cpu", tokens=24)
+    k16 = K.contiguous().view(torch.int16).numpy().view(np.uint16)
+    v16 = V.contiguous().view(torch.int16).numpy().view(np.uint16)
+    H, n = k16.shape[0], 24
+    c, s = oq.rope_cs(wl.theta, np.arange(n))
+    kw, ks = oq.fold_exact(*oq.encode_vectors_box(k16.reshape(-1, 128), 3, rope=True,
+                                                  c=np.tile(c, (H, 1)), s=np.tile(s, (H, 1))), 3)
+    vw, vs = oq.fold_exact(*oq.encode_vectors_box(v16.reshape(-1, 128), 2), 2)
+    job = {"K": k16, "V": v16, "theta": wl.theta, "bits_k": 3, "bits_v": 2, "window": 0, "pct": 0,
+           "exact": True, "gk_codes": kw.reshape(H, n, 12), "gk_meta": ks.reshape(H, n),
+           "gv_codes": vw.reshape(H, n, 8), "gv_meta": vs.reshape(H, n)}
+    assert parity.verdict(parity.check_layer(job)) == []
+    bad = dict(job, gk_codes=job["gk_codes"].copy())
+    bad["gk_codes"][0, 3, 0] ^= 1 << 21  # group 0's coset bit
+    r = parity.check_layer(bad)
+    assert r["unexcused_codes"] >= 1 and parity.verdict(r)
