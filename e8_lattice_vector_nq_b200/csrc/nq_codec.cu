@@ -346,8 +346,8 @@ __device__ __forceinline__ void e8_codes(const float2 (&y)[8], bool halfx, bool 
     if (hity) f.y = __fadd_rn(f.y, copysignf(1.0f, E[i].y));
     const float2 a2 = make_float2(fma_sat(f.x, ix, cx), fma_sat(f.y, iy, cy));
     const float2 J = fma2(a2, R2, B2);  // 2^23 + code: the code sits in the low mantissa bits
-    ax += __float_as_uint(J.x) << (BITS * i);
-    ay += __float_as_uint(J.y) << (BITS * i);
+    ax = mad_u32(__float_as_uint(J.x), 1u << (BITS * i), ax);
+    ay = mad_u32(__float_as_uint(J.y), 1u << (BITS * i), ay);
   }
   constexpr uint32_t kMask = (1u << (8 * BITS)) - 1u;
   gx = ax & kMask;
@@ -428,8 +428,8 @@ __device__ __forceinline__ void e8_box_codes(const float2 (&y)[8], uint32_t& gx,
     // 2^23 + j, exact: the code sits in the low mantissa bits
     const float jx = hx ? __fadd_rn(f1x[i], kH + kTwo23) : __fadd_rn(f0x[i], kH - 1.0f + kTwo23);
     const float jy = hy ? __fadd_rn(f1y[i], kH + kTwo23) : __fadd_rn(f0y[i], kH - 1.0f + kTwo23);
-    ax += __float_as_uint(jx) << (BITS * i);
-    ay += __float_as_uint(jy) << (BITS * i);
+    ax = mad_u32(__float_as_uint(jx), 1u << (BITS * i), ax);
+    ay = mad_u32(__float_as_uint(jy), 1u << (BITS * i), ay);
   }
   constexpr uint32_t kMask = (1u << (8 * BITS)) - 1u;
   constexpr uint32_t kCos = 1u << (7 * BITS);

@@ -104,6 +104,14 @@ __device__ __forceinline__ float4 lds128f(uint32_t addr) {
   return v;
 }
 
+// a * b + c (low 32 bits) in one instruction; packing a code at a bit offset
+// k is mad_u32(code, 1 << k, word) (a shift-and-add for a power-of-two b).
+__device__ __forceinline__ uint32_t mad_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // ----------------------------------------------------- packed fp32 pairs
 // IEEE round-to-nearest per lane (sm_100 f32x2 instructions).
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }

@@ -151,27 +151,33 @@ def test_exact_strided_offsets(nq, oq):
 
 
 def test_exact_degenerate_vectors(nq, oq):
-    wl = synth.WORKLOADS["tiny"]
-    K = torch.zeros(1, 2, 48, 128, dtype=torch.bfloat16, device="cuda")
-    V = torch.zeros_like(K)
-    g = torch.Generator(device="cuda")
-    g.manual_seed(5)
-    K[0, :, 16:32] = (torch.randn(2, 16, 128, device="cuda", generator=g) * 1e30).to(torch.bfloat16)
-    K[0, :, 32:48] = (torch.randn(2, 16, 128, device="cuda", generator=g) * 1e-30).to(torch.bfloat16)
-    V[0, :, 16:] = K[0, :, 16:]
-    rope = nq.rope_tables(wl.theta, 48)
-    ks = nq.ExactStore.empty(1, 2, 48, 3)
-    vs = nq.ExactStore.empty(1, 2, 48, 2)
-    nq.nq_encode_exact(K, V, ks, vs, 48, rope, 48)
+    """Zero rows (sigma 0), a saturated scale (coordinates far outside the
+    box), tiny values, exact lattice-like inputs; inputs within the library's
+    contract (|x| <= 2^30)."""
+    H, T = 2, 40
+    x = torch.randn(1, H, T, 128, device="cuda")
+    x[0, 0, 0] = 0
+    x[0, 0, 1] = 1e9
+    x[0, 0, 5] = -1e9 * (torch.arange(128, device="cuda") % 2)
+    x[0, 1, 2] = -1e-30
+    x[0, 1, 3] = torch.arange(128, device="cuda") % 3 - 1.0
+    x[0, 1, 4] = 0.5
+    K = x.to(torch.bfloat16)
+    V = (x * 3).to(torch.bfloat16)
+    rope = nq.rope_tables(1e4, T)
+    ks = nq.ExactStore.empty(1, H, T, 3)
+    vs = nq.ExactStore.empty(1, H, T, 2)
+    nq.nq_encode_exact(K, V, ks, vs, T, rope, T)
     torch.cuda.synchronize()
-    c, s = oq.rope_cs(wl.theta, np.arange(48))
-    kw, ksig = oracle_exact(oq, u16(K[0]).reshape(-1, 128), 3, rope=True, c=np.tile(c, (2, 1)),
-                            s=np.tile(s, (2, 1)))
+    c, s = oq.rope_cs(1e4, np.arange(T))
+    kw, ksig = oracle_exact(oq, u16(K[0]).reshape(-1, 128), 3, rope=True, c=np.tile(c, (H, 1)),
+                            s=np.tile(s, (H, 1)))
     vw, vsig = oracle_exact(oq, u16(V[0]).reshape(-1, 128), 2)
     assert np.array_equal(u32(ks.codes[0]).reshape(-1, 12), kw)
     assert np.array_equal(u16(ks.sigma[0]).reshape(-1), ksig)
     assert np.array_equal(u32(vs.codes[0]).reshape(-1, 8), vw)
     assert np.array_equal(u16(vs.sigma[0]).reshape(-1), vsig)
+    assert u16(ks.sigma[0])[0, 1] == 0x7BFF  # the saturated scale, 65504
 
 
 def test_exact_store_size(nq):
