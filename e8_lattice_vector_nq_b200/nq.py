@@ -584,14 +584,17 @@ class HostRoundTrip:
     current stream, which afterwards waits for the last copy."""
 
     def __init__(self, codec: Codec, K: torch.Tensor, V: torch.Tensor, K_out: torch.Tensor,
-                 V_out: torch.Tensor, chunk_units: int = 1, values_in_place: bool | None = None):
+                 V_out: torch.Tensor, chunk_units: int = 1, values_in_place: bool | None = None,
+                 units: int | None = None):
         self.codec, self.K, self.V, self.K_out, self.V_out = codec, K, V, K_out, V_out
         # With eviction only the kept value rows are needed: the encode kernel
         # reads them straight from the pinned host cache, so the rows it drops
         # never cross the bus (keys are copied whole: every key is scored).
         self.values_in_place = codec.evict if values_in_place is None else values_in_place
-        self.chunks = [slice(u, min(u + chunk_units, codec.units))
-                       for u in range(0, codec.units, chunk_units)]
+        # the leading `units` units of the codec (all by default)
+        self.units = codec.units if units is None else min(int(units), codec.units)
+        self.chunks = [slice(u, min(u + chunk_units, self.units))
+                       for u in range(0, self.units, chunk_units)]
         self.h2d, self.comp, self.d2h = (torch.cuda.Stream(K.device) for _ in range(3))
         ev = lambda: [torch.cuda.Event() for _ in self.chunks]  # noqa: E731
         self.in_ready, self.comp_done, self.out_done = ev(), ev(), ev()
@@ -602,7 +605,7 @@ class HostRoundTrip:
         if not self.values_in_place:
             return Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size()
         c = self.codec
-        return Kh.numel() * Kh.element_size() + c.units * c.heads * c.n * 128 * Vh.element_size()
+        return Kh.numel() * Kh.element_size() + self.units * c.heads * c.n * 128 * Vh.element_size()
 
     def run(self, Kh: torch.Tensor, Vh: torch.Tensor, K_out_h: torch.Tensor,
             V_out_h: torch.Tensor):
