@@ -723,6 +723,8 @@ def _run_ours(args, world, rank, device, wl, peak, peak_kind, pool, workers, nq)
     if t["clocks"]:
         line["clocks"] = t["clocks"]
     K, V, Kd, Vd, stream = t["K"], t["V"], t["Kd"], t["Vd"], t["stream"]
+    if pool is not None:  # the timed step's outputs, before any other leg reuses the buffers
+        line["parity"] = headline_parity(args, wl, t, pool)
     if not args.no_attend:
         line["decode_attention"] = attend_timing(args, codec, Kd, Vd, stream, world)
     line["reconstruction"] = reconstruction_quality(t["Kq"], t["Vq"], Kd, Vd, codec)
@@ -736,7 +738,6 @@ def _run_ours(args, world, rank, device, wl, peak, peak_kind, pool, workers, nq)
         in_bytes = K.numel() * 2 + V.numel() * 2
         line["e2e"] = e2e(args, t["Kq"], t["Vq"], Kd, Vd, codec, stream, world, in_bytes)
     if pool is not None:
-        line["parity"] = headline_parity(args, wl, t, pool)
         line["cpu_baseline"] = cpu_baseline(args, wl, pool, workers)
     del t, K, V, Kd, Vd, codec
     torch.cuda.empty_cache()
@@ -758,6 +759,8 @@ def _run_ours(args, world, rank, device, wl, peak, peak_kind, pool, workers, nq)
         torch.cuda.empty_cache()
     if configs:
         line["configs"] = configs
+    if not args.no_entropy:
+        line["entropy_correlated"] = entropy_correlated(args, device, world)
     return line
 
 
@@ -794,6 +797,10 @@ def exact_timing(args, wl, t, world, peak, peak_kind):
 
     reps = max(3, min(args.steps, 10))
     enc_ms, dec_ms = tm(enc, reps), tm(dec, reps)
+    # the outputs hold the exact layout's reconstruction now: put the regular one back
+    nq.nq_decode(codec.k_store, codec.v_store, n, Kd, Vd, codec.rope, codec.max_pos,
+                 positions=codec.kept)
+    torch.cuda.synchronize()
     assert nq.device_error() == 0
     per_vec_bytes = 16 * wl.bits_k + 2 + 16 * wl.bits_v + 2
     kept_bytes = (n * 4 * units) if codec.kept is not None else 0
@@ -857,10 +864,18 @@ def attend_timing(args, codec, Kd, Vd, stream, world, G: int = 4):
 
     f_ms, u_ms, s_ms = t(fused), t(unfused), t(sdpa)
     packed = codec.k_store.nbytes + codec.v_store.nbytes
+    # eight query heads per KV head (the variant that runs one CTA per SM)
+    q8 = torch.randn(units, heads * 8, 128, device=Kd.device, generator=g)
+    ws8 = torch.empty(max(nq.lib().nq_attend_workspace_bytes(units, heads, 8, n), 16) // 4,
+                      dtype=torch.float32, device=Kd.device)
+    f8_ms = t(lambda: nq.nq_attend(q8, codec.k_store, codec.v_store, n, 8, codec.rope,
+                                   codec.max_pos, scale=scale, positions=codec.kept, ws=ws8))
     return {"query_heads_per_kv_head": G, "tokens": n, "units": units, "kv_heads": heads,
             "fused_ms": f_ms, "decode_then_sdpa_ms": u_ms, "sdpa_on_bf16_ms": s_ms,
             "speedup_vs_decode_then_sdpa": u_ms / f_ms,
-            "fused_packed_read_gbs": packed / (f_ms * 1e-3) / 1e9}
+            "fused_packed_read_gbs": packed / (f_ms * 1e-3) / 1e9,
+            "fused_ms_8_query_heads_per_kv_head": f8_ms,
+            "fused_packed_read_gbs_8_query_heads": packed / (f8_ms * 1e-3) / 1e9}
 
 
 def reconstruction_quality(K, V, Kd, Vd, codec, layers=(0, 15, 31)):
@@ -996,6 +1011,47 @@ def pinned_buffers(K, V, Kd, Vd):
             torch.cuda.synchronize()
             use //= 2
     return 0, None
+
+
+def entropy_correlated(args, device, world, rho: float = 0.95, layers: int = 4):
+    """The delta + rANS stage on a cache whose tokens are correlated (an AR(1)
+    process along the tokens, rho between neighbours; synth.gen_layer_correlated),
+    the situation the pages' "consecutive tokens give similar lattice indices"
+    describes: Mistral-shaped layers, no eviction (consecutive tokens stay
+    neighbours), K3V2.  Coded size with and without the token difference, and
+    the lossless round trip."""
+    from e8_lattice_vector_nq_b200 import nq
+
+    wl = synth.WORKLOADS["mistral7b_32k"]
+    K = torch.empty(layers, wl.heads, wl.tokens, 128, dtype=torch.bfloat16, device=device)
+    V = torch.empty_like(K)
+    for l in range(layers):
+        k, v = synth.gen_layer_correlated(wl, l, device, rho=rho)
+        K[l].copy_(k)
+        V[l].copy_(v)
+    codec = nq.Codec(layers, wl.heads, wl.tokens, wl.theta, wl.bits_k, wl.bits_v, device=device)
+    codec.encode(K, V)
+    elems = (codec.k_store.meta.numel() + codec.v_store.meta.numel()) * 128
+    code_bytes = codec.k_store.codes.numel() * 4 + codec.v_store.codes.numel() * 4
+    meta_bytes = codec.k_store.meta.numel() * 4 + codec.v_store.meta.numel() * 4
+    res = {"rho": rho, "layers": layers, "tokens": wl.tokens, "heads": wl.heads, "bits": "K3V2",
+           "codes_bits_per_elem_raw": code_bytes * 8 / elems}
+    for delta in (True, False):
+        coded = {nm: nq.nq_entropy_encode(st, codec.n, delta=delta)
+                 for nm, st in (("k", codec.k_store), ("v", codec.v_store))}
+        exact = True
+        for nm, st in (("k", codec.k_store), ("v", codec.v_store)):
+            back = nq.PackedStore.empty(layers, wl.heads, codec.n, st.bits, device)
+            nq.nq_entropy_decode(coded[nm], back)
+            exact = exact and torch.equal(back.codes, st.codes)
+        cb = sum(c.coded_bytes() for c in coded.values())
+        res["delta" if delta else "plain"] = {
+            "codes_bits_per_elem_coded": cb * 8 / elems, "codes_ratio": code_bytes / cb,
+            "cache_bits_per_elem_with_meta": (cb + meta_bytes) * 8 / elems,
+            "round_trip_exact": bool(exact)}
+    del K, V, codec
+    torch.cuda.empty_cache()
+    return res
 
 
 def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):

@@ -77,7 +77,7 @@ struct AttSmem {
 };
 
 template <int BK, int BV, int GT>
-__global__ void __launch_bounds__(256, 2) attend_partial_kernel(const AttendArgs a) {
+__global__ void __launch_bounds__(256, GT == 8 ? 1 : 2) attend_partial_kernel(const AttendArgs a) {
   extern __shared__ __align__(16) unsigned char att_smem[];
   using S = AttSmem<BV, GT>;
   constexpr int GP = (GT + 1) / 2;  // query heads in fp32x2 pairs (GT = 1: one lane unused)
@@ -198,15 +198,16 @@ __global__ void __launch_bounds__(256, 2) attend_partial_kernel(const AttendArgs
     // ---- keys and scores (a token past the chunk has kappa 0 and score -inf)
     float sc[GT];
     {
+      // only this half's code words are read (the other half's stay zero and
+      // are not used by the reconstruction)
       uint32_t wc[4 * BK];
       const uint32_t kt = kcb + (k & 1) * (kSlots * kKStride) + slot_l * kKStride;
 #pragma unroll
+      for (int c = 0; c < 4 * BK; ++c) wc[c] = 0u;
+#pragma unroll
       for (int c = 0; c < BK; ++c) {
-        const uint4 x = lds128(kt + c * 16);
-        wc[4 * c] = x.x;
-        wc[4 * c + 1] = x.y;
-        wc[4 * c + 2] = x.z;
-        wc[4 * c + 3] = x.w;
+        wc[BK * half + c] = lds32(kt + 4 * (BK * half + c));
+        wc[2 * BK + BK * half + c] = lds32(kt + 4 * (2 * BK + BK * half + c));
       }
       float2 v[32];
       reconstruct_half<BK>(wc, kmc, half, v);

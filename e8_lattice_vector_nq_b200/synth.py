@@ -128,6 +128,52 @@ def gen_layer(wl: Workload, layer: int, device="cpu", tokens: int | None = None,
     return K, V
 
 
+def ar1_noise(shape, rho: float, g: torch.Generator, device, block: int = 64) -> torch.Tensor:
+    """Unit-variance Gaussian noise [..., T, D] correlated along the token axis:
+    z_t = rho z_{t-1} + sqrt(1 - rho^2) e_t (an AR(1) process per channel),
+    computed block by block (a scaled cumulative sum inside each block of 64
+    tokens, the carry between blocks)."""
+    *lead, T, Dd = shape
+    e = torch.randn(*lead, T, Dd, generator=g, device=device, dtype=torch.float64)
+    out = torch.empty_like(e)
+    c = (1.0 - rho * rho) ** 0.5
+    t = torch.arange(block, dtype=torch.float64, device=device)
+    up = (rho ** t)[:, None]           # rho^k
+    down = (rho ** (-t))[:, None]      # rho^-k
+    carry = e[..., 0, :]               # z_0 ~ N(0, 1)
+    for b0 in range(0, T, block):
+        b1 = min(T, b0 + block)
+        k = b1 - b0
+        x = c * e[..., b0:b1, :]
+        if b0 == 0:
+            x = x.clone()
+            x[..., 0, :] = carry
+            z = up[:k] * torch.cumsum(x * down[:k], dim=-2)
+        else:
+            z = up[:k] * (rho * carry[..., None, :] + torch.cumsum(x * down[:k], dim=-2))
+        out[..., b0:b1, :] = z
+        carry = z[..., -1, :]
+    return out.to(torch.float32)
+
+
+def gen_layer_correlated(wl: Workload, layer: int, device="cpu", rho: float = 0.95,
+                         tokens: int | None = None):
+    """gen_layer with token-to-token correlation: the same per-channel scales,
+    outliers and rotary embedding, but z drawn as an AR(1) process along the
+    tokens (rho between neighbours) instead of independently, the way
+    consecutive tokens of a real cache resemble each other."""
+    T = wl.tokens if tokens is None else int(tokens)
+    g = layer_generator(wl.seed + 7919, layer, device)
+    lam_k, lam_v = _scales(wl, g, device)
+    pos = torch.arange(T, dtype=torch.int64, device=device)
+    zk = ar1_noise((wl.heads, T, D), rho, g, device)
+    kpre = (zk * lam_k[:, None, :]).to(torch.float64)
+    K = rope_forward_fp64(kpre, pos, wl.theta).to(torch.bfloat16)
+    zv = ar1_noise((wl.heads, T, D), rho, g, device)
+    V = (zv * lam_v[:, None, :]).to(torch.bfloat16)
+    return K, V
+
+
 def gen_prerope_keys(wl: Workload, layer: int, device="cpu", tokens: int | None = None):
     """The keys of ``gen_layer`` before rotation (fp64), for RoPE pins."""
     T = wl.tokens if tokens is None else int(tokens)

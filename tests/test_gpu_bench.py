@@ -85,6 +85,10 @@ def test_optional_blocks(line):
         s = line["entropy_stage"][mode]
         assert s["round_trip_exact"] is True
         assert 0 < s["codes_bits_per_elem_coded"] < 4
+    c = line["entropy_correlated"]
+    assert c["delta"]["round_trip_exact"] and c["plain"]["round_trip_exact"]
+    # correlated tokens: the difference makes the codes cheaper to code
+    assert c["delta"]["codes_ratio"] > c["plain"]["codes_ratio"]
     w = line["layerwise_encode"]
     assert w["all_layers_ms"] > 0 and w["layer_by_layer_ms"] > 0
 
