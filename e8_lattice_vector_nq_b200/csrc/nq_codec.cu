@@ -39,6 +39,8 @@
 
 #include "nq_codec_math.cuh"
 #include "nq_internal.h"
+#include "nq_tc_slots.cuh"
+#include "nq_tcgen05.cuh"
 
 namespace nq {
 
@@ -808,6 +810,364 @@ __global__ void __launch_bounds__(256, 2)
   if (lane == 0) bulk_wait_all();
 }
 
+// ------------------------------------------------ decode on the tensor cores
+// The transform inside decode is an exact integer matrix product: per vector
+// w = H t with H the 128 x 128 Sylvester matrix, t_k = 2 j_k - 2^b + 2 - h_g(k)
+// and |w| <= 896.  decode_tc_kernel runs it on the tensor cores
+// (tcgen05.mma kind::f16, fp32 accumulators in TMEM) for tiles of 128 vectors
+// (8 heads x 16 slots): D = A B^T with
+//  * A (128 x 160, f16): per vector, its 128 codes as 1024 + j 2^d in the slot
+//    order of tc_unpack, 16 slots 2 h_g (the group coset bits) and 16 slots 1;
+//  * B (128 x 160, f16, the same for every tile): row n is output coordinate
+//    c(n) = n/2 + 64 (n % 2), so that a thread's TMEM columns 2i, 2i+1 are the
+//    RoPE pair (i, i+64); code slot p holds 2^(1-d_p) H[c(n)][code_p], coset
+//    slot g holds -(1/2) sum over group g of H[c(n)][k] (0 or +-4), and the
+//    16 constant slots split beta_n = (2 - 2^b) 128 [c(n) = 0]
+//    - sum_p 2^(11-d_p) H[c(n)][code_p] (which cancels the 1024 offsets) into
+//    parts of at most 2^14, each exact in f16.
+// Every product and partial sum is an integer of magnitude below 2^18, so
+// D = w exactly whatever the summation order.  The epilogue (one thread per
+// vector) then forms x = fp32(w kappa), applies the RoPE rotation and the bf16
+// rounding with the same operations as decode_half, and writes the 128-byte
+// swizzled boxes of the same TMA stores.
+//
+// One CTA per SM holds NWG = 4 warpgroups of 128 threads.  Each owns 128 TMEM
+// columns, an A tile whose rows double as the output staging of the same
+// rows (so a warp waits only for its own earlier stores before it writes its
+// rows of the next tile), its coset slots and a RoPE table, and walks its own
+// tiles: write A -> one thread issues the ten MMAs and commits them to the
+// warpgroup's mbarrier -> combine the tile's RoPE table and prefetch the next
+// tile's codes and table rows -> wait for the mbarrier (bounded: past
+// kTcWaitLimit polls the device error word gets kErrMmaTimeout and the
+// warpgroup stops) -> epilogue -> TMA stores.  The output bytes a SM can
+// have in flight are its staging tiles, so the layout gives them as much of
+// the 227 KB as it can: four warpgroups of 32 KB.
+constexpr int kTcA = 32768;    // A: 128 rows x 128 f16 in two 128-byte swizzled K blocks; then
+                               // the output staging: per block of 16 rows two 2 KB boxes
+constexpr int kTcAx = 4096;    // coset slots: 128 rows x 16 f16 as two 2 KB chunk columns
+constexpr int kTcB = 32768;    // B: 128 rows x 128 f16, the layout of A
+constexpr int kTcBx = 8192;    // B extra: coset and constant slots, four 2 KB chunk columns
+constexpr int kTcOnes = 4096;  // A constant slots (1.0), shared by the warpgroups
+constexpr int kTcTab = 1024;   // setup: slot table (code, shift) and per-row constants
+constexpr int kTcShared = kTcB + kTcBx + kTcOnes + kTcTab;
+constexpr uint32_t kTcIdesc = idesc_f16_f32(128, 128);
+constexpr uint32_t kTcWaitLimit = 1u << 20;
+constexpr uint32_t kErrMmaTimeout = 2u;
+
+template <bool ROPE>
+__host__ __device__ constexpr int tc_wg_bytes() {
+  return kTcA + kTcAx + (ROPE ? kCsBytes : 0);
+}
+template <int NWG, bool ROPE>
+__host__ __device__ constexpr int tc_smem_bytes() {
+  return 1024 + kTcShared + NWG * tc_wg_bytes<ROPE>() + 64;
+}
+
+// AND of pred over the `count` threads of named barrier `id`.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0u;
+}
+
+// The constant operands (see above), built once per CTA: B main in the
+// 128-byte swizzled K-major layout; B extra as four 2 KB chunk columns
+// (chunk c of row n at c * 2048 + n * 16: coset slots 0..15, constant slots
+// 16..31); the A constant slots (1.0) as two chunk columns.  tab: generic
+// pointer to kTcTab bytes of scratch (slot codes, shifts, per-row beta).
+template <int BITS>
+__device__ void tc_build_constants(uint32_t b_main, uint32_t b_x, uint32_t ones,
+                                   unsigned char* tab, int tid, int nthreads) {
+  unsigned char* s_code = tab;
+  unsigned char* s_shift = tab + 128;
+  int* s_beta = reinterpret_cast<int*>(tab + 256);
+  for (int i = tid; i < 128; i += nthreads) {
+    int code, d;
+    tc_slot<BITS>(i, code, d);
+    s_code[i] = static_cast<unsigned char>(code);
+    s_shift[i] = static_cast<unsigned char>(d);
+    const int cn = (i >> 1) + 64 * (i & 1);  // row i's coordinate
+    s_beta[i] = cn == 0 ? (2 - (1 << BITS)) * 128 : 0;
+  }
+  for (int i = tid; i < kTcOnes / 16; i += nthreads)
+    sts128(ones + i * 16, make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u));
+  __syncthreads();
+  for (int e = tid; e < 128 * 16; e += nthreads) {
+    const int n = e >> 4, c = e & 15;
+    const int cn = (n >> 1) + 64 * (n & 1);
+    uint32_t v[4];
+    int part = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t pair = 0u;
+#pragma unroll
+      for (int l = 0; l < 2; ++l) {
+        const int p = 8 * c + 2 * u + l;
+        const int code = s_code[p], d = s_shift[p];
+        const uint32_t neg = static_cast<uint32_t>(__popc(cn & code) & 1);
+        pair |= ((neg << 15) | (static_cast<uint32_t>(16 - d) << 10)) << (16 * l);  // +-2^(1-d)
+        part += neg ? (1 << (11 - d)) : -(1 << (11 - d));  // -2^(11-d) H
+      }
+      v[u] = pair;
+    }
+    sts128(b_main + (c >> 3) * 16384 + (n >> 3) * 1024 + (n & 7) * 128 + (((c & 7) ^ (n & 7)) << 4),
+           make_uint4(v[0], v[1], v[2], v[3]));
+    atomicAdd(s_beta + n, part);
+  }
+  __syncthreads();
+  for (int n = tid; n < 128; n += nthreads) {
+    const int cn = (n >> 1) + 64 * (n & 1);
+    uint32_t cw[8], bw[8];
+    int beta = s_beta[n];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      uint32_t pc = 0u, pb = 0u;
+#pragma unroll
+      for (int l = 0; l < 2; ++l) {
+        const int g = 2 * u + l;  // -4 (-1)^popc(c & 8g) where c % 8 == 0, else 0
+        pc |= ((cn & 7) ? 0u : ((__popc(cn & (8 * g)) & 1) ? 0x4400u : 0xC400u)) << (16 * l);
+        const int part = beta > 16384 ? 16384 : (beta < -16384 ? -16384 : beta);
+        beta -= part;
+        pb |= static_cast<uint32_t>(__half_as_ushort(__int2half_rn(part))) << (16 * l);
+      }
+      cw[u] = pc;
+      bw[u] = pb;
+    }
+    sts128(b_x + n * 16, make_uint4(cw[0], cw[1], cw[2], cw[3]));
+    sts128(b_x + 2048 + n * 16, make_uint4(cw[4], cw[5], cw[6], cw[7]));
+    sts128(b_x + 4096 + n * 16, make_uint4(bw[0], bw[1], bw[2], bw[3]));
+    sts128(b_x + 6144 + n * 16, make_uint4(bw[4], bw[5], bw[6], bw[7]));
+  }
+}
+
+// Row r of A: the 128 codes (16 chunks of 8 slots) and the 16 coset slots
+// (2.0 for a set bit g of meta, else 0).
+template <int BITS>
+__device__ __forceinline__ void tc_write_a(const uint32_t (&w)[4 * BITS], uint32_t meta,
+                                           uint32_t a_main, uint32_t a_x, int r) {
+  uint32_t h[64];
+  tc_unpack<BITS>(w, h);
+  const uint32_t rowb = a_main + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    sts128(rowb + (c >> 3) * 16384 + (((c & 7) ^ (r & 7)) << 4),
+           make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]));
+  // y = mask | mask << 15: bit 2u of mask at bit 2u, bit 2u+1 at bit 16 + 2u
+  const uint32_t mask = meta & 0xFFFFu, y = mask | (mask << 15);
+  uint32_t cw[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) cw[u] = (y << (14 - 2 * u)) & 0x40004000u;
+  sts128(a_x + r * 16, make_uint4(cw[0], cw[1], cw[2], cw[3]));
+  sts128(a_x + 2048 + r * 16, make_uint4(cw[4], cw[5], cw[6], cw[7]));
+}
+
+// Columns 32q .. 32q+31 of this thread's row of D (d: their bits) -> bf16
+// coordinates 16q .. 16q+15 and 64+16q .. 79+16q in the swizzled boxes at
+// rowb (box 1 at +16384).
+template <bool ROPE>
+__device__ __forceinline__ void tc_chunk(const uint32_t (&d)[32], int q, float2 k2, uint32_t csa,
+                                         uint32_t rowb, int rsw) {
+  float2 v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    v[e] = mul2(make_float2(__uint_as_float(d[2 * e]), __uint_as_float(d[2 * e + 1])), k2);
+  if (ROPE) {
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const float4 t = lds128f(csa + (8 * q + jj) * (kSlots * 16));
+#pragma unroll
+      for (int ww = 0; ww < 2; ++ww) {
+        const float c = ww ? t.z : t.x, s = ww ? t.w : t.y;
+        const float2 P = v[2 * jj + ww];
+        const float2 Q = mul2(P, make_float2(s, s));
+        v[2 * jj + ww] = make_float2(__fmaf_rn(P.x, c, -Q.y), __fmaf_rn(P.y, c, Q.x));
+      }
+    }
+  }
+#pragma unroll
+  for (int h8 = 0; h8 < 2; ++h8) {
+    uint32_t A[4], B[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int e = 8 * h8 + 2 * t;
+      const __nv_bfloat162 pa = __floats2bfloat162_rn(v[e].x, v[e + 1].x);
+      const __nv_bfloat162 pb = __floats2bfloat162_rn(v[e].y, v[e + 1].y);
+      A[t] = *reinterpret_cast<const uint32_t*>(&pa);
+      B[t] = *reinterpret_cast<const uint32_t*>(&pb);
+    }
+    const uint32_t cc = static_cast<uint32_t>(((2 * q + h8) ^ rsw) << 4);
+    sts128(rowb + cc, make_uint4(A[0], A[1], A[2], A[3]));
+    sts128(rowb + 16384 + cc, make_uint4(B[0], B[1], B[2], B[3]));
+  }
+}
+
+// This thread's row of D (taddr: its TMEM lane, the warpgroup's columns) ->
+// bf16 in the output staging at out.
+template <bool ROPE>
+__device__ __forceinline__ void tc_epilogue(uint32_t taddr, uint32_t meta, uint32_t out,
+                                            uint32_t csa, int r) {
+  const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(meta >> 16)));
+  const float kappa = __fmul_rn(__fmul_rn(sig, 0.5f), __uint_as_float(kCBits));
+  const float2 k2 = make_float2(kappa, kappa);
+  const uint32_t rowb = out + (r >> 3) * 1024 + (r & 7) * 128;
+  const int rsw = r & 7;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t d[32];
+    tmem_ld32(taddr + 32 * q, d);
+    tmem_ld_wait(d);
+    tc_chunk<ROPE>(d, q, k2, csa, rowb, rsw);
+  }
+}
+
+template <int BITS, bool ROPE, bool EXACT, int NWG>
+__global__ void __launch_bounds__(128 * NWG, 1)
+    decode_tc_kernel(const CodecArgs a, const __grid_constant__ CUtensorMap out_map) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const int tid = threadIdx.x, wg = tid >> 7, t = tid & 127, wl = (tid >> 5) & 3, lane = tid & 31;
+  constexpr uint32_t kWg = static_cast<uint32_t>(tc_wg_bytes<ROPE>());
+  constexpr uint32_t kCols = NWG <= 2 ? 256u : 512u;
+  static_assert(128 * NWG <= 512, "one accumulator of 128 columns per warpgroup");
+  const uint32_t b_main = base, b_x = base + kTcB, ones = b_x + kTcBx, tab = ones + kTcOnes;
+  const uint32_t a_main = base + kTcShared + wg * kWg, a_x = a_main + kTcA, cs = a_x + kTcAx;
+  const uint32_t bars = base + kTcShared + NWG * kWg;
+  const uint32_t mbar = bars + 8 * wg, tslot = bars + 8 * NWG;
+
+  if (tid < 32) {
+    tmem_alloc(tslot, kCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int g = 0; g < NWG; ++g) mbar_init(bars + 8 * g, 1);
+    fence_mbar_init();
+  }
+  tc_build_constants<BITS>(b_main, b_x, ones, smem_raw + (tab - raw), tid, blockDim.x);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = lds32(tslot) + static_cast<uint32_t>(128 * wg);
+  const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * wl) << 16);
+
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * NWG + wg;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * NWG;
+  const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
+  const int rb = t >> 4, slot = t & 15;
+  uint32_t w[4 * BITS];
+  uint32_t meta = 0u;
+#pragma unroll
+  for (int i = 0; i < 4 * BITS; ++i) w[i] = 0u;
+  // RoPE table rows of this thread's four cs entries (slot, j = t/16 + 8u) of
+  // the next tile, fetched a tile ahead.
+  float4 ra[4], rbw[4];
+  bool rvalid = false;
+  auto fetch_rope = [&](int64_t tile) {
+    const int32_t src = slot_src(a, tile_of(a, tile), slot);
+    rvalid = src >= 0;
+    if (rvalid) {
+      const int64_t pos = a.pos_base + src;
+      int64_t hi = pos >> 8;
+      hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
+      const float4* ta = reinterpret_cast<const float4*>(a.tab + hi * kHalf);
+      const float4* tb = reinterpret_cast<const float4*>(a.tab + (a.n_a + (pos & 255)) * kHalf);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        ra[u] = __ldg(ta + (t >> 4) + 8 * u);
+        rbw[u] = __ldg(tb + (t >> 4) + 8 * u);
+      }
+    }
+  };
+  if (my_tiles > 0) {
+    load_codes<BITS, EXACT>(a, first, rb, slot, w, meta);
+    if (ROPE) fetch_rope(first);
+  }
+
+  for (int64_t k = 0; k < my_tiles; ++k) {
+    // this warp's rows of A are its output staging: its last stores must have read them
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+    tc_write_a<BITS>(w, meta, a_main, a_x, t);
+    const uint32_t mk = meta;
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar_sync(1 + wg, 128);  // also: every epilogue of tile k-1 has read the RoPE table
+    if (t == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+        umma_f16(tmem, desc_sw128(a_main + off), desc_sw128(b_main + off), kTcIdesc, s > 0);
+      }
+      umma_f16(tmem, desc_plain(a_x, 2048, 128), desc_plain(b_x, 2048, 128), kTcIdesc, 1u);
+      umma_f16(tmem, desc_plain(ones, 2048, 128), desc_plain(b_x + 4096, 2048, 128), kTcIdesc, 1u);
+      umma_commit(mbar);
+    }
+    if (ROPE) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (rvalid) {
+          const float4 A = ra[u], B = rbw[u];
+          v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
+          v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
+          v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
+          v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
+        }
+        sts128(cs + (((t >> 4) + 8 * u) * kSlots + slot) * 16,
+               make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+                          __float_as_uint(v.w)));
+      }
+    }
+    if (k + 1 < my_tiles) {
+      load_codes<BITS, EXACT>(a, first + (k + 1) * step, rb, slot, w, meta);
+      if (ROPE) fetch_rope(first + (k + 1) * step);
+    }
+    // the MMAs are done (A has been read: its rows become the staging) and, by
+    // the same barrier, every thread's part of the RoPE table is written
+    bool done = false;
+    for (uint32_t spin = 0; spin < kTcWaitLimit && !done; ++spin)
+      done = mbar_try_wait(mbar, static_cast<uint32_t>(k & 1));
+    if (!bar_and(1 + wg, 128, done)) {
+      if (t == 0) atomicOr(&g_nq_error, kErrMmaTimeout);
+      break;
+    }
+    tc_fence_after();
+    tc_epilogue<ROPE>(t_row, mk, a_main, cs + slot * 16, t);
+    tc_fence_before();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      // rows past n are clipped by the tensor map (its token extent is n)
+      const Tile tl = tile_of(a, first + k * step);
+      const int y = static_cast<int>(tl.stile * kSlots);
+#pragma unroll
+      for (int b2 = 0; b2 < 2; ++b2) {
+        const int rbi = 2 * wl + b2;
+        const uint32_t src = a_main + rbi * 2048;
+        tma_store_4d(&out_map, src, 0, y, tl.group * a.hg + rbi, tl.unit);
+        tma_store_4d(&out_map, src + 16384, 64, y, tl.group * a.hg + rbi, tl.unit);
+      }
+      bulk_commit();
+    }
+  }
+  if (lane == 0) bulk_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  if (tid < 32) {
+    tc_fence_after();
+    tmem_dealloc(lds32(tslot), kCols);
+  }
+}
+
 // ---------------------------------------------------------------- launch
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against the driver library).
@@ -851,6 +1211,28 @@ static cudaError_t make_out_map(CUtensorMap* m, const CodecArgs& a, int units) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// One CTA of kTcWarpgroups warpgroups per SM (190 KB of shared memory for
+// values, 222 KB for keys), persistent over the tiles.
+constexpr int kTcWarpgroups = 4;
+
+template <int BITS, bool ROPE, bool EXACT>
+static cudaError_t launch_decode_tc(const CodecArgs& a, const CUtensorMap& map,
+                                   cudaStream_t stream) {
+  constexpr int NWG = kTcWarpgroups;
+  const void* fn = reinterpret_cast<const void*>(decode_tc_kernel<BITS, ROPE, EXACT, NWG>);
+  constexpr int smem = tc_smem_bytes<NWG, ROPE>();
+  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  int dev = 0, sms = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  const int64_t grid = min64((a.num_tiles + NWG - 1) / NWG, static_cast<int64_t>(sms));
+  decode_tc_kernel<BITS, ROPE, EXACT, NWG>
+      <<<static_cast<unsigned>(grid), 128 * NWG, smem, stream>>>(a, map);
+  return cudaGetLastError();
+}
+
 template <int BITS, bool ROPE, bool EXACT>
 static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t stream) {
   a.hg = pick_head_group(a.heads);
@@ -877,6 +1259,8 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   if (decode) {
     cudaError_t e = make_out_map(&map, a, units);
     if (e != cudaSuccess) return e;
+    // tiles of 8 heads fill the 128 rows of the tensor-core kernel
+    if (a.hg == 8) return launch_decode_tc<BITS, ROPE, EXACT>(a, map, stream);
     smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes +
            (ROPE ? 2 * kCsBytes + 2 * kRawBytes : 0);
     fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE, EXACT>);

@@ -36,10 +36,13 @@
  * - Inputs must be finite with |x| <= 2^30; other values are out of
  *   contract (no fault: the kernels stay within their buffers, the codes of
  *   such a vector are unspecified).
- * - No kernel spin-waits: staging uses cp.async groups and bulk-copy groups,
- *   whose waits complete in hardware.  nq_device_error() reads the device
- *   error word reserved for in-kernel failure reports (no current kernel
- *   sets it, so it reads 0 after any sequence of valid calls).
+ * - Staging uses cp.async groups and bulk-copy groups, whose waits complete
+ *   in hardware.  The one polled wait is decode's wait for its own
+ *   tensor-core products (an mbarrier that the MMA unit signals on
+ *   completion); it is bounded (2^20 polls), and when it expires the kernel
+ *   sets bit 1 of the device error word and its warpgroup stops (that call's
+ *   output is then incomplete).  nq_device_error() reads the device error
+ *   word; it reads 0 after any sequence of valid calls.
  */
 #ifndef NQ_H
 #define NQ_H
@@ -213,7 +216,10 @@ nq_status nq_encode(const void *K, nq_kv_strides ks, const void *V, nq_kv_stride
  *         details": RoPE restored after quantisation):
  *           o_i = fmaf(x_i, c, -(x_{i+64}*s)),  o_i+64 = fmaf(x_i+64, c, x_i*s)
  *   bf16 round-to-nearest-even into K_out/V_out[u][h][i] (strides kos/vos).
- * k_in/v_in may be NULL (that output is skipped). */
+ * k_in/v_in may be NULL (that output is skipped).  When heads is a multiple
+ * of 8 the transform runs on the tensor cores as an exact f16 product with
+ * fp32 accumulation (every partial sum an integer below 2^18), otherwise on
+ * the CUDA cores; both give the bits above. */
 nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int heads,
                     int64_t n, int64_t slot0, const int32_t *positions, int64_t pos_stride,
                     int64_t pos_base, const float *rope_tab, int64_t rope_max_pos, void *K_out,
@@ -362,9 +368,10 @@ nq_status nq_e8_box_quantise(const float *y, int64_t groups, int bits, uint32_t 
                              uint8_t *coset, nq_stream_t stream);
 
 /* -------------------------------------------------------------- status
- * Reads and clears the device error word reserved for in-kernel failure
- * reports (bit 0: an asynchronous copy did not complete).  Synchronises the
- * current device, so a pending launch error surfaces here as NQ_ERR_CUDA. */
+ * Reads and clears the device error word of in-kernel failure reports
+ * (bit 1: a tensor-core product of nq_decode / nq_decode_exact did not
+ * complete within its bounded wait).  Synchronises the current device, so a
+ * pending launch error surfaces here as NQ_ERR_CUDA. */
 nq_status nq_device_error(uint32_t *flags_out);
 
 #ifdef __cplusplus
