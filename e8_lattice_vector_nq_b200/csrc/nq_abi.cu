@@ -525,6 +525,15 @@ nq_status nq_entropy_decode(const uint16_t* words, const uint32_t* offsets, cons
                      "nq_entropy_decode launch");
 }
 
+nq_status nq_set_decode_engine(int engine) {
+  if (engine != NQ_DECODE_AUTO && engine != NQ_DECODE_TENSOR_CORES && engine != NQ_DECODE_CUDA_CORES)
+    return fail(NQ_ERR_INVALID, "decode engine must be 0, 1 or 2 (got %d)", engine);
+  nq::set_decode_engine(engine);
+  return NQ_OK;
+}
+
+int nq_get_decode_engine(void) { return nq::decode_engine(); }
+
 nq_status nq_device_error(uint32_t* flags_out) {
   if (!flags_out) return fail(NQ_ERR_INVALID, "flags_out is NULL");
   return cuda_status(nq::codec_read_clear_error(flags_out), "nq_device_error");

@@ -35,6 +35,7 @@
 // two launches.
 #include <cuda.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "nq_codec_math.cuh"
@@ -1066,8 +1067,6 @@ __global__ void __launch_bounds__(128 * NWG, 1)
   uint32_t meta = 0u;
 #pragma unroll
   for (int i = 0; i < 4 * BITS; ++i) w[i] = 0u;
-  // RoPE table rows of this thread's four cs entries (slot, j = t/16 + 8u) of
-  // the next tile, fetched a tile ahead.
   float4 ra[4], rbw[4];
   bool rvalid = false;
   auto fetch_rope = [&](int64_t tile) {
@@ -1211,6 +1210,10 @@ static cudaError_t make_out_map(CUtensorMap* m, const CodecArgs& a, int units) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+static std::atomic<int> g_decode_engine{NQ_DECODE_AUTO};
+void set_decode_engine(int engine) { g_decode_engine.store(engine); }
+int decode_engine() { return g_decode_engine.load(); }
+
 // One CTA of kTcWarpgroups warpgroups per SM (190 KB of shared memory for
 // values, 222 KB for keys), persistent over the tiles.
 constexpr int kTcWarpgroups = 4;
@@ -1259,8 +1262,18 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   if (decode) {
     cudaError_t e = make_out_map(&map, a, units);
     if (e != cudaSuccess) return e;
-    // tiles of 8 heads fill the 128 rows of the tensor-core kernel
-    if (a.hg == 8) return launch_decode_tc<BITS, ROPE, EXACT>(a, map, stream);
+    // tiles of 8 heads fill the 128 rows of the tensor-core kernel; it pays for
+    // its per-CTA setup from about two tiles per warpgroup on
+    const int engine = decode_engine();
+    if (a.hg == 8 && engine != NQ_DECODE_CUDA_CORES) {
+      int dev = 0, sms = 0;
+      if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+      if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+      if (engine == NQ_DECODE_TENSOR_CORES ||
+          a.num_tiles >= static_cast<int64_t>(2) * kTcWarpgroups * sms)
+        return launch_decode_tc<BITS, ROPE, EXACT>(a, map, stream);
+    }
     smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes +
            (ROPE ? 2 * kCsBytes + 2 * kRawBytes : 0);
     fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE, EXACT>);

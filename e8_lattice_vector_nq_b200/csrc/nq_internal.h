@@ -71,6 +71,9 @@ cudaError_t launch_encode(const EncodeLaunch& L, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 
 cudaError_t codec_read_clear_error(uint32_t* flags);
+// Decode engine (nq_decode_engine values), read at each decode launch.
+void set_decode_engine(int engine);
+int decode_engine();
 size_t attend_workspace_floats(int units, int heads, int G, int64_t n);
 int64_t attend_ctas(int units, int heads, int64_t n);  // CTAs of the partial kernel
 cudaError_t launch_attend(const AttendLaunch& L, cudaStream_t stream);

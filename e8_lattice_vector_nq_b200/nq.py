@@ -52,7 +52,7 @@ EXPORTS = (
     "nq_attend", "nq_device_error", "nq_entropy_streams", "nq_entropy_max_words",
     "nq_entropy_workspace_bytes", "nq_entropy_encode", "nq_entropy_decode",
     "nq_packed_exact_bytes_per_vector", "nq_encode_exact", "nq_decode_exact",
-    "nq_e8_box_quantise",
+    "nq_e8_box_quantise", "nq_set_decode_engine", "nq_get_decode_engine",
 )
 
 
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         "nq_attend": (i32, [P, i32, i32, i32, PK, PK, i64, i64, P, i64, i64, P, i64,
                             ctypes.c_float, P, P, P, sz, P]),
         "nq_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32)]),
+        "nq_set_decode_engine": (i32, [i32]),
+        "nq_get_decode_engine": (i32, []),
         "nq_entropy_streams": (i64, [i32, i32, i64]),
         "nq_entropy_max_words": (i64, [i32, i32, i64]),
         "nq_entropy_workspace_bytes": (sz, [i32, i32, i64]),
@@ -512,6 +514,18 @@ def nq_entropy_decode(coded: EntropyCoded, out: PackedStore, slot0: int = 0, str
     _check(lib().nq_entropy_decode(_ptr(coded.words), _ptr(coded.offsets), _ptr(coded.freq),
                                    coded.units, coded.heads, coded.n, int(coded.delta),
                                    ctypes.byref(d), int(slot0), _stream(stream)))
+
+
+DECODE_AUTO, DECODE_TENSOR_CORES, DECODE_CUDA_CORES = 0, 1, 2
+
+
+def set_decode_engine(engine: int) -> None:
+    """Select the decode kernel (nq.h, nq_set_decode_engine); process-wide."""
+    _check(lib().nq_set_decode_engine(int(engine)))
+
+
+def get_decode_engine() -> int:
+    return int(lib().nq_get_decode_engine())
 
 
 def device_error() -> int:

@@ -367,6 +367,26 @@ nq_status nq_e8_quantise(const float *y, int64_t groups, int bits, uint32_t *cod
 nq_status nq_e8_box_quantise(const float *y, int64_t groups, int bits, uint32_t *codes,
                              uint8_t *coset, nq_stream_t stream);
 
+/* ------------------------------------------------------- decode engine
+ * Which kernel nq_decode / nq_decode_exact run (process-wide, default
+ * NQ_DECODE_AUTO):
+ *   NQ_DECODE_AUTO          the tensor cores when heads is a multiple of 8 and
+ *                           the call has at least 2 * 4 * (SM count) tiles of
+ *                           8 heads x 16 slots (below that the per-CTA setup of
+ *                           the tensor-core kernel outweighs it), else the CUDA
+ *                           cores;
+ *   NQ_DECODE_TENSOR_CORES  the tensor cores whenever heads is a multiple of 8;
+ *   NQ_DECODE_CUDA_CORES    always the CUDA-core kernel.
+ * Both give the same bits.  Returns NQ_ERR_INVALID for another value.  Not
+ * synchronised with launches in flight: set it between calls. */
+typedef enum {
+  NQ_DECODE_AUTO = 0,
+  NQ_DECODE_TENSOR_CORES = 1,
+  NQ_DECODE_CUDA_CORES = 2
+} nq_decode_engine;
+nq_status nq_set_decode_engine(int engine);
+int nq_get_decode_engine(void);
+
 /* -------------------------------------------------------------- status
  * Reads and clears the device error word of in-kernel failure reports
  * (bit 1: a tensor-core product of nq_decode / nq_decode_exact did not

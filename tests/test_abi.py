@@ -158,3 +158,20 @@ def test_empty_work_is_ok_without_device(nq):
     assert L.nq_entropy_encode(ctypes.byref(pk), 0, 8, 64, 0, 1, None, None, None, 0, None, 0,
                                None) == 0
     assert L.nq_entropy_decode(None, None, None, 0, 8, 64, 0, ctypes.byref(pk), 0, None) == 0
+
+
+def test_decode_engine_switch(nq):
+    """The decode engine is a process-wide setting: auto by default, each
+    documented value accepted and read back, anything else refused."""
+    assert nq.get_decode_engine() == nq.DECODE_AUTO
+    try:
+        for e in (nq.DECODE_TENSOR_CORES, nq.DECODE_CUDA_CORES, nq.DECODE_AUTO):
+            nq.set_decode_engine(e)
+            assert nq.get_decode_engine() == e
+        L = nq.lib()
+        assert L.nq_set_decode_engine(3) == nq.NQ_ERR_INVALID
+        assert "decode engine" in L.nq_last_error().decode()
+        assert nq.get_decode_engine() == nq.DECODE_AUTO
+    finally:
+        nq.set_decode_engine(nq.DECODE_AUTO)
+

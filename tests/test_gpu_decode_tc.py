@@ -1,14 +1,16 @@
 """GPU decode on the tensor cores against the oracle, bit for bit.
 
 nq_decode runs its 128-point transform as an f16 matrix product on the tensor
-cores whenever the head count is a multiple of 8 (tiles of 8 heads x 16
-slots); other head counts take the CUDA-core kernel, which the other parity
-files cover.  The cases here drive the tensor-core path with stores that span
-the whole code space (random code words, every coset mask, scales from zero
-and subnormal to the largest fp16), ragged slot counts on both sides of the
-16-slot tile, head groups (16 and 24 heads), kept-list positions, output
-views with padding, slot and position offsets, and the exact layout.  Every
-decoded bf16 element must equal the oracle's decode of the same store.
+cores for head counts that are multiples of 8 (tiles of 8 heads x 16 slots);
+by default only for calls large enough to pay for its per-CTA setup, so this
+file selects that engine for every size (nq_set_decode_engine) and checks it
+against the CUDA-core engine as well.  The cases here drive the tensor-core
+path with stores that span the whole code space (random code words, every
+coset mask, scales from zero and subnormal to the largest fp16), ragged slot
+counts on both sides of the 16-slot tile, head groups (16 and 24 heads),
+kept-list positions, output views with padding, slot and position offsets,
+and the exact layout.  Every decoded bf16 element must equal the oracle's
+decode of the same store.
 """
 import numpy as np
 import pytest
@@ -26,7 +28,9 @@ def nq():
     from e8_lattice_vector_nq_b200 import build, nq as nqmod
 
     build.build()
-    return nqmod
+    nqmod.set_decode_engine(nqmod.DECODE_TENSOR_CORES)
+    yield nqmod
+    nqmod.set_decode_engine(nqmod.DECODE_AUTO)
 
 
 def u16(t):
@@ -164,3 +168,36 @@ def test_exact_layout_random_stores(nq, oq):
             ref = oq.decode_vectors(w, m, bits, rope=rope_on, c=c if rope_on else None,
                                     s=s if rope_on else None).reshape(heads, n, 128)
             assert np.array_equal(u16(out[u]), ref)
+
+
+@pytest.mark.parametrize("heads,n,exact", [(8, 37, False), (16, 700, False), (8, 129, True)])
+def test_engines_give_the_same_bits(nq, heads, n, exact):
+    """The tensor-core and CUDA-core engines decode the same store to the same bits."""
+    units, theta = 2, 1e6
+    if exact:
+        ks, vs = nq.ExactStore.empty(units, heads, n, 3), nq.ExactStore.empty(units, heads, n, 2)
+        for st, seed in ((ks, 1), (vs, 2)):
+            g = np.random.default_rng(seed)
+            st.codes.copy_(torch.from_numpy(g.integers(0, 2**32, size=st.codes.shape,
+                                                       dtype=np.uint64).astype(np.uint32).view(np.int32)))
+            st.sigma.copy_(torch.from_numpy(g.integers(0, 0x7C00, size=st.sigma.shape)
+                                            .astype(np.uint16).view(np.int16)))
+        dec = nq.nq_decode_exact
+    else:
+        ks, vs = random_store(nq, units, heads, n, 3, 31), random_store(nq, units, heads, n, 2, 32)
+        dec = nq.nq_decode
+    rope = nq.rope_tables(theta, n)
+    outs = []
+    try:
+        for engine in (nq.DECODE_TENSOR_CORES, nq.DECODE_CUDA_CORES):
+            nq.set_decode_engine(engine)
+            Kd = torch.empty(units, heads, n, 128, dtype=torch.bfloat16, device="cuda")
+            Vd = torch.empty_like(Kd)
+            dec(ks, vs, n, Kd, Vd, rope, n)
+            torch.cuda.synchronize()
+            outs.append((u16(Kd), u16(Vd)))
+    finally:
+        nq.set_decode_engine(nq.DECODE_TENSOR_CORES)
+    assert nq.device_error() == 0
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
