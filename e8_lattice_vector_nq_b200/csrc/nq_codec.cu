@@ -84,6 +84,10 @@ struct CodecArgs {
   FastDiv div_groups, div_stiles;
   int64_t pairs;  // encode: units * n (unit, slot) pairs, below 2^31
   FastDiv div_n;  // encode: division by n
+  // tensor-core decode: a tile holds tc_m slot tiles of one head group
+  int tc_m;
+  int64_t tc_sgroups;  // ceil(slot_tiles / tc_m)
+  FastDiv div_sgroups;
 };
 
 struct Tile {
@@ -103,13 +107,18 @@ __device__ __forceinline__ Tile tile_of(const CodecArgs& a, int64_t t64) {
   return r;
 }
 
-// Source token of this lane's slot (lanes l and l+16 share slot l % 16) in
-// tile tl: the kept-list entry, or the slot itself; -1 past the last slot.
-__device__ __forceinline__ int32_t slot_src(const CodecArgs& a, const Tile& tl, int slot_l) {
-  const int64_t slot = tl.stile * kSlots + slot_l;
+// Source token of slot stile * 16 + slot_l of a unit: the kept-list entry, or
+// the slot itself; -1 past the last slot.
+__device__ __forceinline__ int32_t slot_src_at(const CodecArgs& a, int unit, int64_t stile,
+                                               int slot_l) {
+  const int64_t slot = stile * kSlots + slot_l;
   if (slot >= a.n) return -1;
-  return a.idx ? __ldg(a.idx + static_cast<int64_t>(tl.unit) * a.idx_stride + slot)
+  return a.idx ? __ldg(a.idx + static_cast<int64_t>(unit) * a.idx_stride + slot)
                : static_cast<int32_t>(slot);
+}
+// The same for this lane's slot (lanes l and l+16 share slot l % 16) in tile tl.
+__device__ __forceinline__ int32_t slot_src(const CodecArgs& a, const Tile& tl, int slot_l) {
+  return slot_src_at(a, tl.unit, tl.stile, slot_l);
 }
 
 // Encode tiles walk the (unit, slot) pairs of all units as one list, 16 pairs
@@ -706,15 +715,15 @@ __device__ __forceinline__ uint32_t unfold_exact(uint32_t (&w)[4 * BITS], uint32
   return mask | (sig16 << 16);
 }
 
-// Codes and meta of this thread's vector in tile t (registers, one tile ahead).
+// Codes and meta of the vector (unit, head h, slot stile * 16 + slot_l), if
+// that slot is below n (registers, loaded one tile ahead).
 template <int BITS, bool EXACT>
-__device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int warp, int slot_l,
-                                           uint32_t (&w)[4 * BITS], uint32_t& meta) {
-  const Tile tl = tile_of(a, t);
-  const int h = tl.group * a.hg + warp;
-  const int64_t slot = tl.stile * kSlots + slot_l;
+__device__ __forceinline__ void load_codes_at(const CodecArgs& a, int unit, int h, int64_t stile,
+                                              int slot_l, uint32_t (&w)[4 * BITS],
+                                              uint32_t& meta) {
+  const int64_t slot = stile * kSlots + slot_l;
   if (slot < a.n) {
-    const int64_t vec = tl.unit * a.pu + h * a.ph + a.slot0 + slot;
+    const int64_t vec = unit * a.pu + h * a.ph + a.slot0 + slot;
     const uint4* src = reinterpret_cast<const uint4*>(a.codes + vec * (4 * BITS));
 #pragma unroll
     for (int c = 0; c < BITS; ++c) {
@@ -729,6 +738,14 @@ __device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int wa
     else
       meta = __ldg(a.meta + vec);
   }
+}
+
+// Codes and meta of this thread's vector in tile t (warp: its head in the group).
+template <int BITS, bool EXACT>
+__device__ __forceinline__ void load_codes(const CodecArgs& a, int64_t t, int warp, int slot_l,
+                                           uint32_t (&w)[4 * BITS], uint32_t& meta) {
+  const Tile tl = tile_of(a, t);
+  load_codes_at<BITS, EXACT>(a, tl.unit, tl.group * a.hg + warp, tl.stile, slot_l, w, meta);
 }
 
 // Output tile of one warp: 16 rows x 256 bytes as two 16 x 128-byte boxes
@@ -816,7 +833,8 @@ __global__ void __launch_bounds__(256, 2)
 // w = H t with H the 128 x 128 Sylvester matrix, t_k = 2 j_k - 2^b + 2 - h_g(k)
 // and |w| <= 896.  decode_tc_kernel runs it on the tensor cores
 // (tcgen05.mma kind::f16, fp32 accumulators in TMEM) for tiles of 128 vectors
-// (8 heads x 16 slots): D = A B^T with
+// (8 / hg slot tiles of 16 slots for a group of hg heads; with hg = 3, 5, 6 or
+// 7 some of the 8 row blocks idle): D = A B^T with
 //  * A (128 x 160, f16): per vector, its 128 codes as 1024 + j 2^d in the slot
 //    order of tc_unpack, 16 slots 2 h_g (the group coset bits) and 16 slots 1;
 //  * B (128 x 160, f16, the same for every tile): row n is output coordinate
@@ -855,13 +873,13 @@ constexpr uint32_t kTcIdesc = idesc_f16_f32(128, 128);
 constexpr uint32_t kTcWaitLimit = 1u << 20;
 constexpr uint32_t kErrMmaTimeout = 2u;
 
-template <bool ROPE>
+template <int TABLES>
 __host__ __device__ constexpr int tc_wg_bytes() {
-  return kTcA + kTcAx + (ROPE ? kCsBytes : 0);
+  return kTcA + kTcAx + TABLES * kCsBytes;
 }
-template <int NWG, bool ROPE>
+template <int NWG, int TABLES>
 __host__ __device__ constexpr int tc_smem_bytes() {
-  return 1024 + kTcShared + NWG * tc_wg_bytes<ROPE>() + 64;
+  return 1024 + kTcShared + NWG * tc_wg_bytes<TABLES>() + 64;
 }
 
 // AND of pred over the `count` threads of named barrier `id`.
@@ -1028,14 +1046,18 @@ __device__ __forceinline__ void tc_epilogue(uint32_t taddr, uint32_t meta, uint3
   }
 }
 
-template <int BITS, bool ROPE, bool EXACT, int NWG>
+// TABLES: RoPE tables per warpgroup (one per slot tile of a tile; 0 for
+// values).  HG8: head groups of 8, one slot tile per tile (the tiling then
+// folds to constants).
+template <int BITS, bool ROPE, bool EXACT, int NWG, int TABLES, bool HG8>
 __global__ void __launch_bounds__(128 * NWG, 1)
     decode_tc_kernel(const CodecArgs a, const __grid_constant__ CUtensorMap out_map) {
+  static_assert(ROPE == (TABLES > 0), "keys carry one table per slot tile, values none");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const int tid = threadIdx.x, wg = tid >> 7, t = tid & 127, wl = (tid >> 5) & 3, lane = tid & 31;
-  constexpr uint32_t kWg = static_cast<uint32_t>(tc_wg_bytes<ROPE>());
+  constexpr uint32_t kWg = static_cast<uint32_t>(tc_wg_bytes<TABLES>());
   constexpr uint32_t kCols = NWG <= 2 ? 256u : 512u;
   static_assert(128 * NWG <= 512, "one accumulator of 128 columns per warpgroup");
   const uint32_t b_main = base, b_x = base + kTcB, ones = b_x + kTcBx, tab = ones + kTcOnes;
@@ -1062,31 +1084,65 @@ __global__ void __launch_bounds__(128 * NWG, 1)
   const int64_t first = static_cast<int64_t>(blockIdx.x) * NWG + wg;
   const int64_t step = static_cast<int64_t>(gridDim.x) * NWG;
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
+  // Row t of a tile: row block rb = t / 16 is slot tile mi of the tile (rb / hg)
+  // for head rb % hg of the head group, slot t % 16; blocks past m * hg idle.
+  const int hg = HG8 ? 8 : a.hg, m = HG8 ? 1 : a.tc_m;
   const int rb = t >> 4, slot = t & 15;
+  const bool rb_used = rb < m * hg;
+  const int mi = rb_used ? rb / hg : 0, hrel = rb_used ? rb % hg : 0;
+  // A tile index -> (head group, unit, first slot tile).
+  auto tile_at = [&](int64_t t64, int& group, int& unit, int64_t& stile0) {
+    const uint32_t tt = static_cast<uint32_t>(t64);
+    const uint32_t q = fdiv(tt, a.div_groups);
+    const uint32_t u = fdiv(q, a.div_sgroups);
+    group = static_cast<int>(tt - q * a.div_groups.d);
+    unit = static_cast<int>(u);
+    stile0 = static_cast<int64_t>(q - u * a.div_sgroups.d) * m;
+  };
+  auto load_row = [&](int64_t t64, uint32_t (&wr)[4 * BITS], uint32_t& mr) {
+    int group, unit;
+    int64_t stile0;
+    tile_at(t64, group, unit, stile0);
+    const int64_t st = stile0 + mi;
+    if (HG8 || (rb_used && st < a.slot_tiles))
+      load_codes_at<BITS, EXACT>(a, unit, group * hg + hrel, st, slot, wr, mr);
+  };
   uint32_t w[4 * BITS];
   uint32_t meta = 0u;
 #pragma unroll
   for (int i = 0; i < 4 * BITS; ++i) w[i] = 0u;
-  float4 ra[4], rbw[4];
-  bool rvalid = false;
-  auto fetch_rope = [&](int64_t tile) {
-    const int32_t src = slot_src(a, tile_of(a, tile), slot);
-    rvalid = src >= 0;
-    if (rvalid) {
-      const int64_t pos = a.pos_base + src;
-      int64_t hi = pos >> 8;
-      hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
-      const float4* ta = reinterpret_cast<const float4*>(a.tab + hi * kHalf);
-      const float4* tb = reinterpret_cast<const float4*>(a.tab + (a.n_a + (pos & 255)) * kHalf);
+  // RoPE table rows of this thread's four cs entries (slot, j = t/16 + 8u) of
+  // each table of the next tile, fetched a tile ahead.
+  constexpr int kT = TABLES > 0 ? TABLES : 1;
+  float4 ra[kT][4], rbw[kT][4];
+  bool rvalid[kT];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        ra[u] = __ldg(ta + (t >> 4) + 8 * u);
-        rbw[u] = __ldg(tb + (t >> 4) + 8 * u);
+  for (int x = 0; x < kT; ++x) rvalid[x] = false;
+  auto fetch_rope = [&](int64_t t64) {
+    int group, unit;
+    int64_t stile0;
+    tile_at(t64, group, unit, stile0);
+#pragma unroll
+    for (int x = 0; x < kT; ++x) {
+      const int32_t src = HG8 || stile0 + x < a.slot_tiles
+                              ? slot_src_at(a, unit, stile0 + x, slot) : -1;
+      rvalid[x] = src >= 0;
+      if (rvalid[x]) {
+        const int64_t pos = a.pos_base + src;
+        int64_t hi = pos >> 8;
+        hi = hi < 0 ? 0 : (hi >= a.n_a ? a.n_a - 1 : hi);  // out-of-contract positions stay in bounds
+        const float4* ta = reinterpret_cast<const float4*>(a.tab + hi * kHalf);
+        const float4* tb = reinterpret_cast<const float4*>(a.tab + (a.n_a + (pos & 255)) * kHalf);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          ra[x][u] = __ldg(ta + (t >> 4) + 8 * u);
+          rbw[x][u] = __ldg(tb + (t >> 4) + 8 * u);
+        }
       }
     }
   };
   if (my_tiles > 0) {
-    load_codes<BITS, EXACT>(a, first, rb, slot, w, meta);
+    load_row(first, w, meta);
     if (ROPE) fetch_rope(first);
   }
 
@@ -1098,7 +1154,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
     const uint32_t mk = meta;
     fence_proxy_async_smem();
     tc_fence_before();
-    named_bar_sync(1 + wg, 128);  // also: every epilogue of tile k-1 has read the RoPE table
+    named_bar_sync(1 + wg, 128);  // also: every epilogue of tile k-1 has read the RoPE tables
     if (t == 0) {
       tc_fence_after();
 #pragma unroll
@@ -1112,26 +1168,29 @@ __global__ void __launch_bounds__(128 * NWG, 1)
     }
     if (ROPE) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (rvalid) {
-          const float4 A = ra[u], B = rbw[u];
-          v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
-          v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
-          v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
-          v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
+      for (int x = 0; x < kT; ++x) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (rvalid[x]) {
+            const float4 A = ra[x][u], B = rbw[x][u];
+            v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
+            v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
+            v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
+            v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
+          }
+          sts128(cs + x * kCsBytes + (((t >> 4) + 8 * u) * kSlots + slot) * 16,
+                 make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+                            __float_as_uint(v.w)));
         }
-        sts128(cs + (((t >> 4) + 8 * u) * kSlots + slot) * 16,
-               make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
-                          __float_as_uint(v.w)));
       }
     }
     if (k + 1 < my_tiles) {
-      load_codes<BITS, EXACT>(a, first + (k + 1) * step, rb, slot, w, meta);
+      load_row(first + (k + 1) * step, w, meta);
       if (ROPE) fetch_rope(first + (k + 1) * step);
     }
     // the MMAs are done (A has been read: its rows become the staging) and, by
-    // the same barrier, every thread's part of the RoPE table is written
+    // the same barrier, every thread's part of the RoPE tables is written
     bool done = false;
     for (uint32_t spin = 0; spin < kTcWaitLimit && !done; ++spin)
       done = mbar_try_wait(mbar, static_cast<uint32_t>(k & 1));
@@ -1140,20 +1199,26 @@ __global__ void __launch_bounds__(128 * NWG, 1)
       break;
     }
     tc_fence_after();
-    tc_epilogue<ROPE>(t_row, mk, a_main, cs + slot * 16, t);
+    tc_epilogue<ROPE>(t_row, mk, a_main, cs + (ROPE ? mi : 0) * kCsBytes + slot * 16, t);
     tc_fence_before();
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
       // rows past n are clipped by the tensor map (its token extent is n)
-      const Tile tl = tile_of(a, first + k * step);
-      const int y = static_cast<int>(tl.stile * kSlots);
+      int group, unit;
+      int64_t stile0;
+      tile_at(first + k * step, group, unit, stile0);
 #pragma unroll
       for (int b2 = 0; b2 < 2; ++b2) {
         const int rbi = 2 * wl + b2;
+        if (rbi >= m * hg) continue;
+        const int64_t st = stile0 + rbi / hg;
+        if (!HG8 && st >= a.slot_tiles) continue;
+        const int y = static_cast<int>(st * kSlots);
+        const int h = group * hg + rbi % hg;
         const uint32_t src = a_main + rbi * 2048;
-        tma_store_4d(&out_map, src, 0, y, tl.group * a.hg + rbi, tl.unit);
-        tma_store_4d(&out_map, src + 16384, 64, y, tl.group * a.hg + rbi, tl.unit);
+        tma_store_4d(&out_map, src, 0, y, h, unit);
+        tma_store_4d(&out_map, src + 16384, 64, y, h, unit);
       }
       bulk_commit();
     }
@@ -1214,26 +1279,61 @@ static std::atomic<int> g_decode_engine{NQ_DECODE_AUTO};
 void set_decode_engine(int engine) { g_decode_engine.store(engine); }
 int decode_engine() { return g_decode_engine.load(); }
 
-// One CTA of kTcWarpgroups warpgroups per SM (190 KB of shared memory for
-// values, 222 KB for keys), persistent over the tiles.
-constexpr int kTcWarpgroups = 4;
+// Tensor-core decode tiles: 128 rows = m slot tiles x hg heads x 16 slots,
+// m = 8 / hg (rows past m * hg * 16 idle).  Keys need one RoPE table per slot
+// tile, so they take hg >= 3 (m <= 2) and, with two tables, three warpgroups
+// (shared memory); values take any hg.
+static int tc_slot_tiles_per_tile(int hg, bool rope) {
+  const int m = 8 / hg;
+  return rope && m > 2 ? 0 : m;
+}
 
-template <int BITS, bool ROPE, bool EXACT>
-static cudaError_t launch_decode_tc(const CodecArgs& a, const CUtensorMap& map,
-                                   cudaStream_t stream) {
-  constexpr int NWG = kTcWarpgroups;
-  const void* fn = reinterpret_cast<const void*>(decode_tc_kernel<BITS, ROPE, EXACT, NWG>);
-  constexpr int smem = tc_smem_bytes<NWG, ROPE>();
+template <int BITS, bool ROPE, bool EXACT, int NWG, int TABLES, bool HG8>
+static cudaError_t launch_decode_tc_on(const CodecArgs& a, const CUtensorMap& map, int sms,
+                                       cudaStream_t stream) {
+  const void* fn =
+      reinterpret_cast<const void*>(decode_tc_kernel<BITS, ROPE, EXACT, NWG, TABLES, HG8>);
+  constexpr int smem = tc_smem_bytes<NWG, TABLES>();
+  static_assert(smem <= 232448, "one CTA per SM within 227 KB");
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
+  const int64_t grid = min64((a.num_tiles + NWG - 1) / NWG, static_cast<int64_t>(sms));
+  decode_tc_kernel<BITS, ROPE, EXACT, NWG, TABLES, HG8>
+      <<<static_cast<unsigned>(grid), 128 * NWG, smem, stream>>>(a, map);
+  return cudaGetLastError();
+}
+
+// Runs the tensor-core decode when the engine setting and the call allow it
+// (*used = true), else leaves the call to the CUDA-core kernel.
+template <int BITS, bool ROPE, bool EXACT>
+static cudaError_t launch_decode_tc(CodecArgs a, const CUtensorMap& map, cudaStream_t stream,
+                                    bool* used) {
+  *used = false;
+  const int engine = decode_engine();
+  const int m = tc_slot_tiles_per_tile(a.hg, ROPE);
+  if (engine == NQ_DECODE_CUDA_CORES || m == 0) return cudaSuccess;
+  const int nwg = ROPE && m == 2 ? 3 : 4;
+  a.tc_m = m;
+  a.tc_sgroups = (a.slot_tiles + m - 1) / m;
+  a.num_tiles = static_cast<int64_t>(a.num_tiles / a.slot_tiles) * a.tc_sgroups;  // units * groups * sgroups
+  a.div_sgroups = make_fastdiv(static_cast<uint32_t>(a.tc_sgroups));
   int dev = 0, sms = 0;
+  cudaError_t err;
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
   if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return err;
-  const int64_t grid = min64((a.num_tiles + NWG - 1) / NWG, static_cast<int64_t>(sms));
-  decode_tc_kernel<BITS, ROPE, EXACT, NWG>
-      <<<static_cast<unsigned>(grid), 128 * NWG, smem, stream>>>(a, map);
-  return cudaGetLastError();
+  // the per-CTA setup (the constant B operand) pays from about two tiles per warpgroup on
+  if (engine == NQ_DECODE_AUTO && a.num_tiles < static_cast<int64_t>(2) * nwg * sms)
+    return cudaSuccess;
+  *used = true;
+  constexpr int T1 = ROPE ? 1 : 0;
+  if (a.hg == 8) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, T1, true>(a, map, sms, stream);
+  if constexpr (!ROPE) {
+    return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, false>(a, map, sms, stream);
+  } else {
+    if (m == 1) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 1, false>(a, map, sms, stream);
+    return launch_decode_tc_on<BITS, ROPE, EXACT, 3, 2, false>(a, map, sms, stream);
+  }
 }
 
 template <int BITS, bool ROPE, bool EXACT>
@@ -1262,18 +1362,9 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
   if (decode) {
     cudaError_t e = make_out_map(&map, a, units);
     if (e != cudaSuccess) return e;
-    // tiles of 8 heads fill the 128 rows of the tensor-core kernel; it pays for
-    // its per-CTA setup from about two tiles per warpgroup on
-    const int engine = decode_engine();
-    if (a.hg == 8 && engine != NQ_DECODE_CUDA_CORES) {
-      int dev = 0, sms = 0;
-      if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-      if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-        return e;
-      if (engine == NQ_DECODE_TENSOR_CORES ||
-          a.num_tiles >= static_cast<int64_t>(2) * kTcWarpgroups * sms)
-        return launch_decode_tc<BITS, ROPE, EXACT>(a, map, stream);
-    }
+    bool used = false;
+    if ((e = launch_decode_tc<BITS, ROPE, EXACT>(a, map, stream, &used)) != cudaSuccess || used)
+      return e;
     smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes +
            (ROPE ? 2 * kCsBytes + 2 * kRawBytes : 0);
     fn = reinterpret_cast<const void*>(decode_kernel<BITS, ROPE, EXACT>);

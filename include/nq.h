@@ -216,10 +216,12 @@ nq_status nq_encode(const void *K, nq_kv_strides ks, const void *V, nq_kv_stride
  *         details": RoPE restored after quantisation):
  *           o_i = fmaf(x_i, c, -(x_{i+64}*s)),  o_i+64 = fmaf(x_i+64, c, x_i*s)
  *   bf16 round-to-nearest-even into K_out/V_out[u][h][i] (strides kos/vos).
- * k_in/v_in may be NULL (that output is skipped).  When heads is a multiple
- * of 8 the transform runs on the tensor cores as an exact f16 product with
- * fp32 accumulation (every partial sum an integer below 2^18), otherwise on
- * the CUDA cores; both give the bits above. */
+ * k_in/v_in may be NULL (that output is skipped).  The transform runs on the
+ * tensor cores as an exact f16 product with fp32 accumulation (every partial
+ * sum an integer below 2^18) in tiles of 128 vectors (8 / hg slot tiles of a
+ * group of hg heads, hg the largest divisor of heads up to 8; keys need
+ * hg >= 3), or on the CUDA cores (see nq_set_decode_engine); both give the
+ * bits above. */
 nq_status nq_decode(const nq_packed *k_in, const nq_packed *v_in, int units, int heads,
                     int64_t n, int64_t slot0, const int32_t *positions, int64_t pos_stride,
                     int64_t pos_base, const float *rope_tab, int64_t rope_max_pos, void *K_out,
@@ -370,12 +372,12 @@ nq_status nq_e8_box_quantise(const float *y, int64_t groups, int bits, uint32_t 
 /* ------------------------------------------------------- decode engine
  * Which kernel nq_decode / nq_decode_exact run (process-wide, default
  * NQ_DECODE_AUTO):
- *   NQ_DECODE_AUTO          the tensor cores when heads is a multiple of 8 and
- *                           the call has at least 2 * 4 * (SM count) tiles of
- *                           8 heads x 16 slots (below that the per-CTA setup of
- *                           the tensor-core kernel outweighs it), else the CUDA
- *                           cores;
- *   NQ_DECODE_TENSOR_CORES  the tensor cores whenever heads is a multiple of 8;
+ *   NQ_DECODE_AUTO          the tensor cores where they apply (see nq_decode)
+ *                           and the call has at least two 128-vector tiles per
+ *                           warpgroup of the SMs (8 or 6 tiles per SM; below
+ *                           that the per-CTA setup of the tensor-core kernel
+ *                           outweighs it), else the CUDA cores;
+ *   NQ_DECODE_TENSOR_CORES  the tensor cores wherever they apply;
  *   NQ_DECODE_CUDA_CORES    always the CUDA-core kernel.
  * Both give the same bits.  Returns NQ_ERR_INVALID for another value.  Not
  * synchronised with launches in flight: set it between calls. */

@@ -1,16 +1,18 @@
 """GPU decode on the tensor cores against the oracle, bit for bit.
 
 nq_decode runs its 128-point transform as an f16 matrix product on the tensor
-cores for head counts that are multiples of 8 (tiles of 8 heads x 16 slots);
-by default only for calls large enough to pay for its per-CTA setup, so this
-file selects that engine for every size (nq_set_decode_engine) and checks it
-against the CUDA-core engine as well.  The cases here drive the tensor-core
-path with stores that span the whole code space (random code words, every
-coset mask, scales from zero and subnormal to the largest fp16), ragged slot
-counts on both sides of the 16-slot tile, head groups (16 and 24 heads),
-kept-list positions, output views with padding, slot and position offsets,
-and the exact layout.  Every decoded bf16 element must equal the oracle's
-decode of the same store.
+cores, in tiles of 128 vectors: 8 / hg slot tiles of a group of hg heads
+(hg = the largest divisor of the head count up to 8; keys need hg >= 3).  By
+default it does so only for calls large enough to pay for its per-CTA setup,
+so this file selects that engine for every size (nq_set_decode_engine) and
+checks it against the CUDA-core engine as well.  The cases here drive the
+tensor-core path with stores that span the whole code space (random code
+words, every coset mask, scales from zero and subnormal to the largest fp16),
+ragged slot counts on both sides of the 16-slot tile, every head-group size
+1..8 (with idle rows for 3, 5, 6 and 7), several head groups (16 and 24
+heads), kept-list positions with one and two RoPE tables per tile, output
+views with padding, slot and position offsets, and the exact layout.  Every
+decoded bf16 element must equal the oracle's decode of the same store.
 """
 import numpy as np
 import pytest
@@ -73,6 +75,8 @@ def oracle_decode(oq, store, u, slot0, n, bits, rope, theta, positions):
 @pytest.mark.parametrize("heads,n,bk,bv", [
     (8, 1, 3, 2), (8, 15, 2, 3), (8, 16, 3, 3), (8, 17, 2, 2), (8, 255, 3, 2),
     (16, 1000, 3, 2), (24, 333, 2, 3), (8, 4100, 3, 2),
+    (4, 1000, 3, 2), (4, 17, 2, 3), (12, 333, 3, 2), (3, 257, 2, 3), (5, 100, 3, 2),
+    (7, 77, 3, 3), (6, 48, 2, 2), (2, 300, 3, 2), (1, 500, 3, 3), (1, 15, 2, 2),
 ])
 def test_random_stores_match_oracle(nq, oq, heads, n, bk, bv):
     units, theta = 3, 5e5
@@ -90,9 +94,11 @@ def test_random_stores_match_oracle(nq, oq, heads, n, bk, bv):
         assert np.array_equal(u16(Vd[u]), oracle_decode(oq, vs, u, 0, n, bv, False, theta, pos))
 
 
-def test_kept_positions_views_and_offsets(nq, oq):
-    """Evicted-cache positions, padded output views, slot0 > 0, pos_base > 0."""
-    units, heads, n, slot0, pos_base, theta = 2, 8, 300, 37, 1000, 1e6
+@pytest.mark.parametrize("heads", [8, 4, 3])
+def test_kept_positions_views_and_offsets(nq, oq, heads):
+    """Evicted-cache positions, padded output views, slot0 > 0, pos_base > 0
+    (one RoPE table per tile for 8 heads, two for 4 and 3)."""
+    units, n, slot0, pos_base, theta = 2, 300, 37, 1000, 1e6
     ks = random_store(nq, units, heads, 400, 3, 5)
     vs = random_store(nq, units, heads, 400, 2, 6)
     g = np.random.default_rng(3)
@@ -118,7 +124,7 @@ def test_kept_positions_views_and_offsets(nq, oq):
     assert torch.count_nonzero(out_k[..., :16]) == 0 and torch.count_nonzero(out_v[..., 128:]) == 0
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode_append"])
+@pytest.mark.parametrize("name", ["tiny", "decode_append", "qwen25_7b_64k", "mistral7b_32k"])
 def test_encoded_caches_match_oracle(nq, oq, name):
     """Real encodes (the codes the method produces) through the tensor-core decode."""
     wl = synth.WORKLOADS[name]
@@ -134,7 +140,8 @@ def test_encoded_caches_match_oracle(nq, oq, name):
     torch.cuda.synchronize()
     assert nq.device_error() == 0
     for u in range(units):
-        pos = np.arange(codec.n)
+        pos = (codec.kept[u].cpu().numpy().astype(np.int64) if codec.evict
+               else np.arange(codec.n))
         assert np.array_equal(u16(Kd[u]), oracle_decode(oq, codec.k_store, u, 0, codec.n, wl.bits_k,
                                                         True, wl.theta, pos))
         assert np.array_equal(u16(Vd[u]), oracle_decode(oq, codec.v_store, u, 0, codec.n,
@@ -170,7 +177,8 @@ def test_exact_layout_random_stores(nq, oq):
             assert np.array_equal(u16(out[u]), ref)
 
 
-@pytest.mark.parametrize("heads,n,exact", [(8, 37, False), (16, 700, False), (8, 129, True)])
+@pytest.mark.parametrize("heads,n,exact", [(8, 37, False), (16, 700, False), (8, 129, True),
+                                            (4, 500, False), (3, 33, True), (1, 100, False)])
 def test_engines_give_the_same_bits(nq, heads, n, exact):
     """The tensor-core and CUDA-core engines decode the same store to the same bits."""
     units, theta = 2, 1e6
