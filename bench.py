@@ -316,12 +316,23 @@ KERNEL_OF = {"score": "score_kernel", "select": "select_kernel", "encode": "enco
              "decode": "decode_kernel"}
 
 
-def kernel_of(stage: str, heads: int) -> str:
-    """The kernel a stage launches: decode runs on the tensor cores for head
-    counts that fill its 8-head tiles."""
-    if stage == "decode" and heads % 8 == 0:
-        return "decode_tc_kernel"
-    return KERNEL_OF[stage]
+def kernel_of(stage: str, heads: int, units: int = 0, n: int = 0) -> str:
+    """The kernel a stage launches.  Decode (the default engine) runs on the
+    tensor cores when the head group hg (largest divisor of heads up to 8) is
+    at least 3 and the call has two 128-vector tiles per warpgroup of the SMs
+    (tiles = units * groups * ceil(slot tiles / (8 // hg)), 4 warpgroups per
+    SM, 3 for keys with two RoPE tables); the key launch decides the name."""
+    if stage != "decode":
+        return KERNEL_OF[stage]
+    hg = max(g for g in range(1, 9) if heads % g == 0)
+    m = 8 // hg
+    if m > 2:
+        return KERNEL_OF[stage]
+    slot_tiles = (n + 15) // 16
+    tiles = units * (heads // hg) * ((slot_tiles + m - 1) // m)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+    nwg = 3 if m == 2 else 4
+    return "decode_tc_kernel" if tiles >= 2 * nwg * sms else KERNEL_OF[stage]
 
 
 def timed_region(fn, steps, stream, device, world, n_events):
@@ -429,7 +440,7 @@ def figures(wl, t, world, peak, peak_kind, traffic_for=None):
     roof = {}
     for stage, ms in per.items():
         ach = alg[stage] / (ms * 1e-3) / 1e9
-        r = {"kernel": kernel_of(stage, wl.heads), "bound": "hbm", "achieved": ach, "peak": peak,
+        r = {"kernel": kernel_of(stage, wl.heads, units, n), "bound": "hbm", "achieved": ach, "peak": peak,
              "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
              "frac_of_8tbs_spec": ach / 8000.0, "algorithmic_bytes": alg[stage], "ms": ms}
         if stage == "select":
@@ -520,7 +531,7 @@ def time_append(nq, wl, device, world, warmup=3):
     roof = {}
     for stage, alg, sms in (("encode", enc_alg, enc), ("decode", dec_alg, dec)):
         ach = alg / (sms * 1e-3) / 1e9
-        roof[stage] = {"kernel": kernel_of(stage, H), "bound": "hbm", "achieved": ach, "peak": peak,
+        roof[stage] = {"kernel": kernel_of(stage, H, S, int(n_mean)), "bound": "hbm", "achieved": ach, "peak": peak,
                        "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
                        "frac_of_8tbs_spec": ach / 8000.0, "algorithmic_bytes": alg, "ms": sms}
     roof["encode"]["bound"] = "latency"  # 16 384 vectors per append: one short launch pair
@@ -820,7 +831,7 @@ def exact_timing(args, wl, t, world, peak, peak_kind):
     roof = {}
     for stage, ms in (("encode", enc_ms), ("decode", dec_ms)):
         ach = alg / (ms * 1e-3) / 1e9
-        roof[stage] = {"kernel": f"{stage}_kernel (exact layout)", "bound": "hbm",
+        roof[stage] = {"kernel": kernel_of(stage, heads, units, n) + " (exact layout)", "bound": "hbm",
                        "achieved": ach, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                        "frac": ach / peak, "algorithmic_bytes": alg, "ms": ms}
     return {"encode_ms": enc_ms, "decode_ms": dec_ms,
