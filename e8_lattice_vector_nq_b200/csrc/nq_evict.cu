@@ -45,6 +45,10 @@ constexpr int kScoreThreads = 256;
 
 // 4 CTAs (32 warps) per SM: more 16-byte loads in flight per SM (a few
 // registers spill to L1).
+// SHARE: fewer heads than warps, so wph = floor(8 / heads) (2, 4 or 8) warps
+// share a head, each taking 1 / wph of the tile's tokens and every warp loads;
+// otherwise one warp per head.
+template <bool SHARE>
 __global__ void __launch_bounds__(kScoreThreads, 4) score_kernel(const uint16_t* __restrict__ K,
                                                               nq_kv_strides ks, int heads,
                                                               int64_t T,
@@ -57,8 +61,12 @@ __global__ void __launch_bounds__(kScoreThreads, 4) score_kernel(const uint16_t*
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = lane >> 4, chunk = lane & 15;
   const int nwarps = kScoreThreads / 32;
+  constexpr int kPairs = kScoreTok / 2;  // iterations of two tokens per warp and head
+  const int wph = SHARE ? nwarps / heads : 1;
+  const int span = SHARE ? kPairs / wph : kPairs;
 
-  for (int h = warp; h < heads; h += nwarps) {
+  for (int hw = warp; hw < heads * wph; hw += nwarps) {
+    const int h = SHARE ? hw % heads : hw, it_begin = SHARE ? (hw / heads) * span : 0;
     const float* mh = mean + (static_cast<int64_t>(u) * heads + h) * kD + chunk * 8;
     double m[8];
 #pragma unroll
@@ -67,7 +75,7 @@ __global__ void __launch_bounds__(kScoreThreads, 4) score_kernel(const uint16_t*
     // 8 independent 16-byte loads per lane are in flight before any math
     constexpr int kBatch = 8;
 #pragma unroll 1
-    for (int it0 = 0; it0 < kScoreTok / 2; it0 += kBatch) {
+    for (int it0 = it_begin; it0 < it_begin + span; it0 += kBatch) {
       uint4 q[kBatch];
 #pragma unroll
       for (int b = 0; b < kBatch; ++b) {
@@ -426,13 +434,20 @@ cudaError_t launch_score(const void* K, nq_kv_strides ks, int units, int heads, 
   if (err != cudaSuccess) return err;
   const int64_t tiles = (T + kScoreTok - 1) / kScoreTok;
   const size_t smem = static_cast<size_t>(heads) * kScoreTok * sizeof(double);
+  const bool share = heads < kScoreThreads / 32;
+  const void* fn = share ? reinterpret_cast<const void*>(score_kernel<true>)
+                         : reinterpret_cast<const void*>(score_kernel<false>);
   if (smem > 48 * 1024) {
-    err = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  score_kernel<<<static_cast<unsigned>(units * tiles), kScoreThreads, smem, stream>>>(
-      static_cast<const uint16_t*>(K), ks, heads, T, mean_ws, scores);
+  if (share)
+    score_kernel<true><<<static_cast<unsigned>(units * tiles), kScoreThreads, smem, stream>>>(
+        static_cast<const uint16_t*>(K), ks, heads, T, mean_ws, scores);
+  else
+    score_kernel<false><<<static_cast<unsigned>(units * tiles), kScoreThreads, smem, stream>>>(
+        static_cast<const uint16_t*>(K), ks, heads, T, mean_ws, scores);
   return cudaGetLastError();
 }
 
