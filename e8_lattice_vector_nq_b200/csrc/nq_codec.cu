@@ -377,25 +377,32 @@ __device__ __forceinline__ void e8_codes(const float2 (&y)[8], bool halfx, bool 
 // whose move by dir = (e >= 0 ? +1 : -1), reversed when that leaves the box,
 // costs least moves, cost fmaf(-2 dir, e, 1), the first index on ties, and d
 // gains that cost.  The half coset wins only when strictly closer.
-__device__ __forceinline__ void box_fix_lane(float (&f)[8], const float (&e)[8], float lo,
-                                             float hi, float& d) {
-  float best = 0.0f, kdir = 0.0f;
-  int k = 0;
+// The move for one lane, without branches (a lane-dependent branch here made
+// warps run both paths): every coordinate's move and cost, then the first
+// coordinate of least cost moves and d gains that cost, only when the sum is
+// odd.  The first index attaining the minimum is the one a scan keeping the
+// first strictly smaller cost finds.
+__device__ __forceinline__ void box_fix_bf(float (&f)[8], const float (&e)[8], float lo, float hi,
+                                           bool odd, float& d) {
+  float c[8], u[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float dir = e[i] >= 0.0f ? 1.0f : -1.0f;
-    if (f[i] + dir > hi || f[i] + dir < lo) dir = -dir;
-    const float cost = __fmaf_rn(-2.0f * dir, e[i], 1.0f);
-    if (i == 0 || cost < best) {
-      best = cost;
-      k = i;
-      kdir = dir;
-    }
+    const bool p = e[i] >= 0.0f;
+    float v = p ? 1.0f : -1.0f;
+    if (f[i] == (p ? hi : lo)) v = -v;  // f is on the grid in [lo, hi]: f + dir leaves it
+    c[i] = __fmaf_rn(-2.0f * v, e[i], 1.0f);
+    u[i] = v;
   }
+  const float m = fminf(fminf(fminf(fminf(c[0], c[1]), c[2]), fminf(fminf(c[3], c[4]), c[5])),
+                        fminf(c[6], c[7]));
+  bool done = !odd;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (i == k) f[i] = __fadd_rn(f[i], kdir);
-  d = __fadd_rn(d, best);
+  for (int i = 0; i < 8; ++i) {
+    const bool hit = !done && c[i] == m;
+    done = done || hit;
+    if (hit) f[i] = __fadd_rn(f[i], u[i]);
+  }
+  if (odd) d = __fadd_rn(d, m);
 }
 
 __device__ __forceinline__ void d8_box2(const float2 (&y)[8], float shift, float lo, float hi,
@@ -420,8 +427,8 @@ __device__ __forceinline__ void d8_box2(const float2 (&y)[8], float shift, float
   const float2 b = add2(sum, M2);  // parity of the integer sum: LSB of the biased value
   dx = d.x;
   dy = d.y;
-  if (__float_as_uint(b.x) & 1u) box_fix_lane(fx, ex, lo, hi, dx);
-  if (__float_as_uint(b.y) & 1u) box_fix_lane(fy, ey, lo, hi, dy);
+  box_fix_bf(fx, ex, lo, hi, __float_as_uint(b.x) & 1u, dx);
+  box_fix_bf(fy, ey, lo, hi, __float_as_uint(b.y) & 1u, dy);
 }
 
 // Folded codes of two groups (lanes x, y) at their nearest E8 point inside the
