@@ -845,8 +845,8 @@ __global__ void __launch_bounds__(256, 2)
 //  * A (128 x 160, f16): per vector, its 128 codes as 1024 + j 2^d in the slot
 //    order of tc_unpack, 16 slots 2 h_g (the group coset bits) and 16 slots 1;
 //  * B (128 x 160, f16, the same for every tile): row n is output coordinate
-//    c(n) = n/2 + 64 (n % 2), so that a thread's TMEM columns 2i, 2i+1 are the
-//    RoPE pair (i, i+64); code slot p holds 2^(1-d_p) H[c(n)][code_p], coset
+//    c(n) = tc_coord(n) (columns 4k .. 4k+3: 2k, 2k+1, 2k+64, 2k+65, two RoPE
+//    pairs as two register pairs); code slot p holds 2^(1-d_p) H[c(n)][code_p], coset
 //    slot g holds -(1/2) sum over group g of H[c(n)][k] (0 or +-4), and the
 //    16 constant slots split beta_n = (2 - 2^b) 128 [c(n) = 0]
 //    - sum_p 2^(11-d_p) H[c(n)][code_p] (which cancels the 1024 offsets) into
@@ -903,6 +903,13 @@ __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool pred) 
   return r != 0u;
 }
 
+// Output coordinate of row n of B (TMEM column n): columns 4k .. 4k+3 hold
+// coordinates 2k, 2k+1, 2k+64, 2k+65, so a thread's register pairs are
+// (x_2k, x_2k+1) and their RoPE partners (x_2k+64, x_2k+65).
+__host__ __device__ constexpr int tc_coord(int n) {
+  return 2 * (n >> 2) + (n & 1) + 64 * ((n >> 1) & 1);
+}
+
 // The constant operands (see above), built once per CTA: B main in the
 // 128-byte swizzled K-major layout; B extra as four 2 KB chunk columns
 // (chunk c of row n at c * 2048 + n * 16: coset slots 0..15, constant slots
@@ -919,7 +926,7 @@ __device__ void tc_build_constants(uint32_t b_main, uint32_t b_x, uint32_t ones,
     tc_slot<BITS>(i, code, d);
     s_code[i] = static_cast<unsigned char>(code);
     s_shift[i] = static_cast<unsigned char>(d);
-    const int cn = (i >> 1) + 64 * (i & 1);  // row i's coordinate
+    const int cn = tc_coord(i);  // row i's coordinate
     s_beta[i] = cn == 0 ? (2 - (1 << BITS)) * 128 : 0;
   }
   for (int i = tid; i < kTcOnes / 16; i += nthreads)
@@ -927,7 +934,7 @@ __device__ void tc_build_constants(uint32_t b_main, uint32_t b_x, uint32_t ones,
   __syncthreads();
   for (int e = tid; e < 128 * 16; e += nthreads) {
     const int n = e >> 4, c = e & 15;
-    const int cn = (n >> 1) + 64 * (n & 1);
+    const int cn = tc_coord(n);
     uint32_t v[4];
     int part = 0;
 #pragma unroll
@@ -949,7 +956,7 @@ __device__ void tc_build_constants(uint32_t b_main, uint32_t b_x, uint32_t ones,
   }
   __syncthreads();
   for (int n = tid; n < 128; n += nthreads) {
-    const int cn = (n >> 1) + 64 * (n & 1);
+    const int cn = tc_coord(n);
     uint32_t cw[8], bw[8];
     int beta = s_beta[n];
 #pragma unroll
@@ -996,25 +1003,27 @@ __device__ __forceinline__ void tc_write_a(const uint32_t (&w)[4 * BITS], uint32
 
 // Columns 32q .. 32q+31 of this thread's row of D (d: their bits) -> bf16
 // coordinates 16q .. 16q+15 and 64+16q .. 79+16q in the swizzled boxes at
-// rowb (box 1 at +16384).
+// rowb (box 1 at +16384).  Columns 32q + 4g .. +3 are X = (x_2k, x_2k+1) and
+// Y = (x_2k+64, x_2k+65), k = 8q + g; the table entry of k is (c_2k, c_2k+1,
+// s_2k, s_2k+1), so one packed multiply and one packed fma per half rotate two
+// pairs with each lane's own roundings fmaf(x, c, -(y s)), fmaf(y, c, x s).
 template <bool ROPE>
 __device__ __forceinline__ void tc_chunk(const uint32_t (&d)[32], int q, float2 k2, uint32_t csa,
                                          uint32_t rowb, int rsw) {
-  float2 v[16];
+  float2 X[8], Y[8];
 #pragma unroll
-  for (int e = 0; e < 16; ++e)
-    v[e] = mul2(make_float2(__uint_as_float(d[2 * e]), __uint_as_float(d[2 * e + 1])), k2);
+  for (int g = 0; g < 8; ++g) {
+    X[g] = mul2(make_float2(__uint_as_float(d[4 * g]), __uint_as_float(d[4 * g + 1])), k2);
+    Y[g] = mul2(make_float2(__uint_as_float(d[4 * g + 2]), __uint_as_float(d[4 * g + 3])), k2);
+  }
   if (ROPE) {
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      const float4 t = lds128f(csa + (8 * q + jj) * (kSlots * 16));
-#pragma unroll
-      for (int ww = 0; ww < 2; ++ww) {
-        const float c = ww ? t.z : t.x, s = ww ? t.w : t.y;
-        const float2 P = v[2 * jj + ww];
-        const float2 Q = mul2(P, make_float2(s, s));
-        v[2 * jj + ww] = make_float2(__fmaf_rn(P.x, c, -Q.y), __fmaf_rn(P.y, c, Q.x));
-      }
+    for (int g = 0; g < 8; ++g) {
+      const float4 t = lds128f(csa + (8 * q + g) * (kSlots * 16));
+      const float2 C = make_float2(t.x, t.y), S = make_float2(t.z, t.w);
+      const float2 T = mul2(Y[g], S), U = mul2(X[g], S);
+      X[g] = fma2(X[g], C, make_float2(-T.x, -T.y));
+      Y[g] = fma2(Y[g], C, U);
     }
   }
 #pragma unroll
@@ -1022,9 +1031,8 @@ __device__ __forceinline__ void tc_chunk(const uint32_t (&d)[32], int q, float2 
     uint32_t A[4], B[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      const int e = 8 * h8 + 2 * t;
-      const __nv_bfloat162 pa = __floats2bfloat162_rn(v[e].x, v[e + 1].x);
-      const __nv_bfloat162 pb = __floats2bfloat162_rn(v[e].y, v[e + 1].y);
+      const __nv_bfloat162 pa = __floats2bfloat162_rn(X[4 * h8 + t].x, X[4 * h8 + t].y);
+      const __nv_bfloat162 pb = __floats2bfloat162_rn(Y[4 * h8 + t].x, Y[4 * h8 + t].y);
       A[t] = *reinterpret_cast<const uint32_t*>(&pa);
       B[t] = *reinterpret_cast<const uint32_t*>(&pb);
     }
@@ -1179,11 +1187,11 @@ __global__ void __launch_bounds__(128 * NWG, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (rvalid[x]) {
+          if (rvalid[x]) {  // (c_2j, c_2j+1, s_2j, s_2j+1)
             const float4 A = ra[x][u], B = rbw[x][u];
             v.x = __fmaf_rn(A.x, B.x, -__fmul_rn(A.y, B.y));
-            v.y = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
-            v.z = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
+            v.z = __fmaf_rn(A.y, B.x, __fmul_rn(A.x, B.y));
+            v.y = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
             v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
           }
           sts128(cs + x * kCsBytes + (((t >> 4) + 8 * u) * kSlots + slot) * 16,
