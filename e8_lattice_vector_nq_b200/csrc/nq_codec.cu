@@ -1200,10 +1200,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
         }
       }
     }
-    if (k + 1 < my_tiles) {
-      load_row(first + (k + 1) * step, w, meta);
-      if (ROPE) fetch_rope(first + (k + 1) * step);
-    }
+    if (k + 1 < my_tiles) load_row(first + (k + 1) * step, w, meta);
     // the MMAs are done (A has been read: its rows become the staging) and, by
     // the same barrier, every thread's part of the RoPE tables is written
     bool done = false;
@@ -1237,6 +1234,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
       }
       bulk_commit();
     }
+    if (ROPE && k + 1 < my_tiles) fetch_rope(first + (k + 1) * step);
   }
   if (lane == 0) bulk_wait_all();
   tc_fence_before();
