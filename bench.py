@@ -1079,9 +1079,10 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     """Same metric through the public API with HOST buffers: pinned H2D of the
     inputs, the four calls, D2H of the reconstructed cache, every step, as
     nq.HostRoundTrip pipelines them (chunks of layers on three streams).  When
-    the host cannot pin the whole cache, the leading layers that it can pin
-    are timed (the rate is per byte of bf16 KV in, so it stays comparable) and
-    the line says how many."""
+    the host cannot pin the whole cache, the layers it can pin serve as a ring
+    that every layer of the cache passes through (values copied); with values
+    read in place (eviction) the leading layers it can pin are timed instead.
+    The line says which."""
     from e8_lattice_vector_nq_b200 import nq
 
     units = K.shape[0]
@@ -1091,8 +1092,11 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     Kh, Vh, Koh, Voh = bufs
     Kh.copy_(K[:use])
     Vh.copy_(V[:use])
-    rt = nq.HostRoundTrip(codec, K, V, Kd, Vd, chunk_units=args.e2e_chunk, units=use)
-    sub_in = in_bytes * use // units
+    ring = use < units and not codec.evict and use % args.e2e_chunk == 0
+    rt = nq.HostRoundTrip(codec, K, V, Kd, Vd, chunk_units=args.e2e_chunk,
+                          units=None if ring else use)
+    timed = units if ring else use
+    sub_in = in_bytes * timed // units
 
     def step():
         rt.run(Kh, Vh, Koh, Voh)
@@ -1112,11 +1116,15 @@ def e2e(args, K, V, Kd, Vd, codec, stream, world, in_bytes):
     value = world * sub_in / (ms * 1e-3) / 1e9
     out = {"value": value, "unit": "GB/s",
            "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": Koh.numel() * 2 + Voh.numel() * 2,
+           "d2h_bytes_per_step": rt.d2h_bytes(Koh, Voh),
            "ms_per_step": ms, "steps": args.e2e_steps, "chunk_layers": args.e2e_chunk,
            "values_read_in_place": rt.values_in_place, "link": link,
            "h2d_bound_gbs": world * bound, "frac_of_h2d_bound": value / (world * bound)}
-    if use < units:
+    if ring:
+        out["host_ring_layers"] = use
+        out["note"] = (f"the host pinned only {use} of {units} layers: they serve as a ring that "
+                       f"all {units} layers pass through, both ways, every step")
+    elif use < units:
         out["layers_timed"] = use
         out["note"] = (f"the host pinned only {use} of {units} layers; the step is those layers "
                        f"(the rate is per byte of bf16 KV in)")

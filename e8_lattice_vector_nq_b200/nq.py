@@ -595,7 +595,12 @@ class HostRoundTrip:
     device-to-host copy of chunk c-1 run at the same time (the two copy
     directions share nothing on a full-duplex link).  The device tensors are
     the codec's working copies; every run() is asynchronous on the caller's
-    current stream, which afterwards waits for the last copy."""
+    current stream, which afterwards waits for the last copy.
+
+    Host tensors with fewer units than the run (R of them) act as a ring: unit
+    u is copied from and to host slot u % R, every unit still crossing the bus
+    both ways (for hosts that cannot pin a whole cache; values must then be
+    copied, not read in place, and R must be a multiple of the chunk)."""
 
     def __init__(self, codec: Codec, K: torch.Tensor, V: torch.Tensor, K_out: torch.Tensor,
                  V_out: torch.Tensor, chunk_units: int = 1, values_in_place: bool | None = None,
@@ -616,13 +621,30 @@ class HostRoundTrip:
 
     def h2d_bytes(self, Kh: torch.Tensor, Vh: torch.Tensor) -> int:
         """Bytes that cross the bus host-to-device per run."""
+        per_unit = lambda t: t[0].numel() * t.element_size()  # noqa: E731
         if not self.values_in_place:
-            return Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size()
+            return self.units * (per_unit(Kh) + per_unit(Vh))
         c = self.codec
-        return Kh.numel() * Kh.element_size() + self.units * c.heads * c.n * 128 * Vh.element_size()
+        return self.units * (per_unit(Kh) + c.heads * c.n * 128 * Vh.element_size())
+
+    def d2h_bytes(self, K_out_h: torch.Tensor, V_out_h: torch.Tensor) -> int:
+        """Bytes that cross the bus device-to-host per run."""
+        return self.units * (K_out_h[0].numel() * K_out_h.element_size()
+                             + V_out_h[0].numel() * V_out_h.element_size())
 
     def run(self, Kh: torch.Tensor, Vh: torch.Tensor, K_out_h: torch.Tensor,
             V_out_h: torch.Tensor):
+        R = Kh.shape[0]
+        if R < self.units:
+            step = self.chunks[0].stop - self.chunks[0].start
+            if self.values_in_place or R % step or min(Vh.shape[0], K_out_h.shape[0],
+                                                       V_out_h.shape[0]) < R:
+                raise ValueError("a host ring needs copied values, equal ring sizes and a "
+                                 "multiple of the chunk")
+
+        def host(u: slice) -> slice:  # the host slot of a chunk
+            return u if R >= self.units else slice(u.start % R, u.start % R + u.stop - u.start)
+
         caller = torch.cuda.current_stream(self.K.device)
         start = torch.cuda.Event()
         start.record(caller)
@@ -632,9 +654,9 @@ class HostRoundTrip:
             with torch.cuda.stream(self.h2d):
                 if self.ran:  # the previous run's kernels are done reading this chunk
                     self.h2d.wait_event(self.comp_done[c])
-                self.K[u].copy_(Kh[u], non_blocking=True)
+                self.K[u].copy_(Kh[host(u)], non_blocking=True)
                 if not self.values_in_place:
-                    self.V[u].copy_(Vh[u], non_blocking=True)
+                    self.V[u].copy_(Vh[host(u)], non_blocking=True)
                 self.in_ready[c].record(self.h2d)
             self.comp.wait_event(self.in_ready[c])
             if self.ran:  # the previous run's copy-out of this chunk is done
@@ -644,8 +666,8 @@ class HostRoundTrip:
             self.comp_done[c].record(self.comp)
             with torch.cuda.stream(self.d2h):
                 self.d2h.wait_event(self.comp_done[c])
-                K_out_h[u].copy_(self.K_out[u], non_blocking=True)
-                V_out_h[u].copy_(self.V_out[u], non_blocking=True)
+                K_out_h[host(u)].copy_(self.K_out[u], non_blocking=True)
+                V_out_h[host(u)].copy_(self.V_out[u], non_blocking=True)
                 self.out_done[c].record(self.d2h)
         caller.wait_event(self.out_done[-1])
         self.ran = True

@@ -49,3 +49,39 @@ def test_host_round_trip_equals_device_path(nq, chunk, in_place):
         assert torch.equal(Koh, Kr.cpu()) and torch.equal(Voh, Vr.cpu()), run
         assert torch.equal(codec.kept.cpu(), ref.kept.cpu())
     assert nq.device_error() == 0
+
+
+@pytest.mark.parametrize("chunk", [1, 2])
+def test_host_ring_passes_every_unit_through(nq, chunk):
+    """Host buffers of R < units units act as a ring (unit u uses slot u % R):
+    with equal inputs in every unit mapped to a slot (no eviction), each slot
+    ends holding the reconstruction of its input, and a ring that does not fit
+    the chunk, or values read in place, is refused."""
+    wl = synth.WORKLOADS["llama3_8b_128k"]
+    L, R, H, T = 8, 4, 8, 700
+    ring_in = [synth.gen_layer(wl, l, "cuda", tokens=T) for l in range(R)]
+    Kr_in = torch.stack([k for k, _ in ring_in])
+    Vr_in = torch.stack([v for _, v in ring_in])
+    # reference: the R ring layers through the device calls
+    ref = nq.Codec(R, H, T, wl.theta, 3, 2, wl.window, 0)
+    ref.encode(Kr_in, Vr_in)
+    Kref = torch.empty(R, H, ref.n, 128, dtype=torch.bfloat16, device="cuda")
+    Vref = torch.empty_like(Kref)
+    ref.decode(Kref, Vref)
+    codec = nq.Codec(L, H, T, wl.theta, 3, 2, wl.window, 0)
+    Kd = torch.empty(L, H, T, 128, dtype=torch.bfloat16, device="cuda")
+    Vd = torch.empty_like(Kd)
+    Ko = torch.empty(L, H, codec.n, 128, dtype=torch.bfloat16, device="cuda")
+    Vo = torch.empty_like(Ko)
+    rt = nq.HostRoundTrip(codec, Kd, Vd, Ko, Vo, chunk_units=chunk)
+    Kh, Vh = Kr_in.cpu().pin_memory(), Vr_in.cpu().pin_memory()
+    Koh = torch.zeros((R,) + tuple(Ko.shape[1:]), dtype=Ko.dtype).pin_memory()
+    Voh = torch.zeros_like(Koh).pin_memory()
+    rt.run(Kh, Vh, Koh, Voh)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(Koh, Kref.cpu()) and torch.equal(Voh, Vref.cpu())
+    assert rt.h2d_bytes(Kh, Vh) == L * 2 * H * T * 128 * 2
+    assert rt.d2h_bytes(Koh, Voh) == L * 2 * H * codec.n * 128 * 2
+    assert nq.device_error() == 0
+    with pytest.raises(ValueError):
+        nq.HostRoundTrip(codec, Kd, Vd, Ko, Vo, chunk_units=3).run(Kh, Vh, Koh, Voh)
