@@ -876,13 +876,22 @@ constexpr int kTcBx = 8192;    // B extra: coset and constant slots, four 2 KB c
 constexpr int kTcOnes = 4096;  // A constant slots (1.0), shared by the warpgroups
 constexpr int kTcTab = 1024;   // setup: slot table (code, shift) and per-row constants
 constexpr int kTcShared = kTcB + kTcBx + kTcOnes + kTcTab;
+// RoPE table of one slot tile: entry (j, slot) = (c_2j, c_2j+1, s_2j, s_2j+1) of
+// the slot's position at j * kTcCsPitch + slot * 16.  The pitch is 17 chunks of
+// 16 bytes, so both access patterns are free of bank conflicts: a quarter warp
+// writing eight consecutive j of one slot, and one reading entry j of eight
+// consecutive slots.
+constexpr int kTcCsPitch = 17 * 16;
+constexpr int kTcCsBytes = 32 * kTcCsPitch;
 constexpr uint32_t kTcIdesc = idesc_f16_f32(128, 128);
 constexpr uint32_t kTcWaitLimit = 1u << 20;
 constexpr uint32_t kErrMmaTimeout = 2u;
 
+// A warpgroup's A tile, coset slots and tables, rounded up to 1024 bytes so
+// that every warpgroup's A tile keeps the swizzle atom's 1024-byte alignment.
 template <int TABLES>
 __host__ __device__ constexpr int tc_wg_bytes() {
-  return kTcA + kTcAx + TABLES * kCsBytes;
+  return (kTcA + kTcAx + TABLES * kTcCsBytes + 1023) / 1024 * 1024;
 }
 template <int NWG, int TABLES>
 __host__ __device__ constexpr int tc_smem_bytes() {
@@ -1019,7 +1028,7 @@ __device__ __forceinline__ void tc_chunk(const uint32_t (&d)[32], int q, float2 
   if (ROPE) {
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
-      const float4 t = lds128f(csa + (8 * q + g) * (kSlots * 16));
+      const float4 t = lds128f(csa + (8 * q + g) * kTcCsPitch);
       const float2 C = make_float2(t.x, t.y), S = make_float2(t.z, t.w);
       const float2 T = mul2(Y[g], S), U = mul2(X[g], S);
       X[g] = fma2(X[g], C, make_float2(-T.x, -T.y));
@@ -1075,6 +1084,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
   constexpr uint32_t kWg = static_cast<uint32_t>(tc_wg_bytes<TABLES>());
   constexpr uint32_t kCols = NWG <= 2 ? 256u : 512u;
   static_assert(128 * NWG <= 512, "one accumulator of 128 columns per warpgroup");
+  static_assert(kTcShared % 1024 == 0 && kWg % 1024 == 0, "A tiles on 1024-byte boundaries");
   const uint32_t b_main = base, b_x = base + kTcB, ones = b_x + kTcBx, tab = ones + kTcOnes;
   const uint32_t a_main = base + kTcShared + wg * kWg, a_x = a_main + kTcA, cs = a_x + kTcAx;
   const uint32_t bars = base + kTcShared + NWG * kWg;
@@ -1126,8 +1136,10 @@ __global__ void __launch_bounds__(128 * NWG, 1)
   uint32_t meta = 0u;
 #pragma unroll
   for (int i = 0; i < 4 * BITS; ++i) w[i] = 0u;
-  // RoPE table rows of this thread's four cs entries (slot, j = t/16 + 8u) of
-  // each table of the next tile, fetched a tile ahead.
+  // RoPE table rows of this thread's four table entries (fslot, j = fj + 8u)
+  // of each table of the next tile, fetched a tile ahead: eight lanes read one
+  // 128-byte run of a slot's two table rows.
+  const int fslot = t >> 3, fj = t & 7;
   constexpr int kT = TABLES > 0 ? TABLES : 1;
   float4 ra[kT][4], rbw[kT][4];
   bool rvalid[kT];
@@ -1140,7 +1152,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
 #pragma unroll
     for (int x = 0; x < kT; ++x) {
       const int32_t src = HG8 || stile0 + x < a.slot_tiles
-                              ? slot_src_at(a, unit, stile0 + x, slot) : -1;
+                              ? slot_src_at(a, unit, stile0 + x, fslot) : -1;
       rvalid[x] = src >= 0;
       if (rvalid[x]) {
         const int64_t pos = a.pos_base + src;
@@ -1150,8 +1162,8 @@ __global__ void __launch_bounds__(128 * NWG, 1)
         const float4* tb = reinterpret_cast<const float4*>(a.tab + (a.n_a + (pos & 255)) * kHalf);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          ra[x][u] = __ldg(ta + (t >> 4) + 8 * u);
-          rbw[x][u] = __ldg(tb + (t >> 4) + 8 * u);
+          ra[x][u] = __ldg(ta + fj + 8 * u);
+          rbw[x][u] = __ldg(tb + fj + 8 * u);
         }
       }
     }
@@ -1194,7 +1206,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
             v.y = __fmaf_rn(A.z, B.z, -__fmul_rn(A.w, B.w));
             v.w = __fmaf_rn(A.w, B.z, __fmul_rn(A.z, B.w));
           }
-          sts128(cs + x * kCsBytes + (((t >> 4) + 8 * u) * kSlots + slot) * 16,
+          sts128(cs + x * kTcCsBytes + (fj + 8 * u) * kTcCsPitch + fslot * 16,
                  make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
                             __float_as_uint(v.w)));
         }
@@ -1211,7 +1223,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
       break;
     }
     tc_fence_after();
-    tc_epilogue<ROPE>(t_row, mk, a_main, cs + (ROPE ? mi : 0) * kCsBytes + slot * 16, t);
+    tc_epilogue<ROPE>(t_row, mk, a_main, cs + (ROPE ? mi : 0) * kTcCsBytes + slot * 16, t);
     tc_fence_before();
     fence_proxy_async_smem();
     __syncwarp();
