@@ -1111,10 +1111,16 @@ __global__ void __launch_bounds__(128 * NWG, 1)
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
   // Row t of a tile: row block rb = t / 16 is slot tile mi of the tile (rb / hg)
   // for head rb % hg of the head group, slot t % 16; blocks past m * hg idle.
+  // Keys in head groups of 8 pair their rows instead: lanes 2i and 2i+1 of
+  // warp w hold slot i of heads 2w and 2w+1, so the two lanes that read one
+  // RoPE table entry sit in the same quarter warp (one shared-memory access
+  // serves both), and a warp's 32 rows are one box of 2 heads x 16 tokens.
+  constexpr bool PAIRS = ROPE && HG8;
   const int hg = HG8 ? 8 : a.hg, m = HG8 ? 1 : a.tc_m;
-  const int rb = t >> 4, slot = t & 15;
-  const bool rb_used = rb < m * hg;
-  const int mi = rb_used ? rb / hg : 0, hrel = rb_used ? rb % hg : 0;
+  const int rb = t >> 4, slot = PAIRS ? (lane >> 1) : (t & 15);
+  const bool rb_used = PAIRS || rb < m * hg;
+  const int mi = PAIRS || !rb_used ? 0 : rb / hg;
+  const int hrel = PAIRS ? 2 * wl + (lane & 1) : (rb_used ? rb % hg : 0);
   // A tile index -> (head group, unit, first slot tile).
   auto tile_at = [&](int64_t t64, int& group, int& unit, int64_t& stile0) {
     const uint32_t tt = static_cast<uint32_t>(t64);
@@ -1232,8 +1238,14 @@ __global__ void __launch_bounds__(128 * NWG, 1)
       int group, unit;
       int64_t stile0;
       tile_at(first + k * step, group, unit, stile0);
+      if (PAIRS) {  // rows 32 wl .. 32 wl + 31: heads 2 wl, 2 wl + 1 of 16 tokens
+        const int y = static_cast<int>(stile0 * kSlots), h = group * 8 + 2 * wl;
+        const uint32_t src = a_main + wl * 4096;
+        tma_store_4d(&out_map, src, 0, h, y, unit);
+        tma_store_4d(&out_map, src + 16384, 64, h, y, unit);
+      }
 #pragma unroll
-      for (int b2 = 0; b2 < 2; ++b2) {
+      for (int b2 = 0; b2 < (PAIRS ? 0 : 2); ++b2) {
         const int rbi = 2 * wl + b2;
         if (rbi >= m * hg) continue;
         const int64_t st = stile0 + rbi / hg;
@@ -1281,8 +1293,11 @@ static EncodeTiledFn encode_tiled_fn() {
 
 // 4-D map of a bf16 [units][heads][n][128] output: boxes of 64 coordinates x
 // 16 tokens, 128-byte swizzle.  Strides in bytes; a unit dimension of extent
-// 1 may carry any stride, so it is given a valid one.
-static cudaError_t make_out_map(CUtensorMap* m, const CodecArgs& a, int units) {
+// 1 may carry any stride, so it is given a valid one.  head_pairs: the head
+// dimension is listed before the token one, with boxes of 64 coordinates x 2
+// heads x 16 tokens (shared-memory rows token-major: row 2 * token + head).
+static cudaError_t make_out_map(CUtensorMap* m, const CodecArgs& a, int units,
+                                bool head_pairs = false) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return cudaErrorNotSupported;
   const uint64_t st = static_cast<uint64_t>(a.st) * 2;
@@ -1293,6 +1308,14 @@ static cudaError_t make_out_map(CUtensorMap* m, const CodecArgs& a, int units) {
                         static_cast<cuuint64_t>(units)};
   cuuint64_t strides[3] = {st, sh, su};
   cuuint32_t box[4] = {64, kSlots, 1, 1};
+  if (head_pairs) {
+    dims[1] = static_cast<cuuint64_t>(a.heads);
+    dims[2] = static_cast<cuuint64_t>(a.n);
+    strides[0] = sh;
+    strides[1] = st;
+    box[1] = 2;
+    box[2] = kSlots;
+  }
   cuuint32_t es[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(a.kv), dims,
                   strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1331,8 +1354,8 @@ static cudaError_t launch_decode_tc_on(const CodecArgs& a, const CUtensorMap& ma
 // Runs the tensor-core decode when the engine setting and the call allow it
 // (*used = true), else leaves the call to the CUDA-core kernel.
 template <int BITS, bool ROPE, bool EXACT>
-static cudaError_t launch_decode_tc(CodecArgs a, const CUtensorMap& map, cudaStream_t stream,
-                                    bool* used) {
+static cudaError_t launch_decode_tc(CodecArgs a, const CUtensorMap& map, int units,
+                                    cudaStream_t stream, bool* used) {
   *used = false;
   const int engine = decode_engine();
   const int m = tc_slot_tiles_per_tile(a.hg, ROPE);
@@ -1352,7 +1375,12 @@ static cudaError_t launch_decode_tc(CodecArgs a, const CUtensorMap& map, cudaStr
     return cudaSuccess;
   *used = true;
   constexpr int T1 = ROPE ? 1 : 0;
-  if (a.hg == 8) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, T1, true>(a, map, sms, stream);
+  if (a.hg == 8) {
+    if (!ROPE) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, T1, true>(a, map, sms, stream);
+    CUtensorMap pairs;  // keys: rows in head pairs (see decode_tc_kernel)
+    if ((err = make_out_map(&pairs, a, units, true)) != cudaSuccess) return err;
+    return launch_decode_tc_on<BITS, ROPE, EXACT, 4, T1, true>(a, pairs, sms, stream);
+  }
   if constexpr (!ROPE) {
     return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, false>(a, map, sms, stream);
   } else {
@@ -1388,7 +1416,8 @@ static cudaError_t launch_one(bool decode, CodecArgs a, int units, cudaStream_t 
     cudaError_t e = make_out_map(&map, a, units);
     if (e != cudaSuccess) return e;
     bool used = false;
-    if ((e = launch_decode_tc<BITS, ROPE, EXACT>(a, map, stream, &used)) != cudaSuccess || used)
+    if ((e = launch_decode_tc<BITS, ROPE, EXACT>(a, map, units, stream, &used)) != cudaSuccess ||
+        used)
       return e;
     smem = 1024 + static_cast<size_t>(threads / 32) * kOutTileBytes +
            (ROPE ? 2 * kCsBytes + 2 * kRawBytes : 0);
