@@ -1071,9 +1071,9 @@ __device__ __forceinline__ void tc_epilogue(uint32_t taddr, uint32_t meta, uint3
 }
 
 // TABLES: RoPE tables per warpgroup (one per slot tile of a tile; 0 for
-// values).  HG8: head groups of 8, one slot tile per tile (the tiling then
-// folds to constants).
-template <int BITS, bool ROPE, bool EXACT, int NWG, int TABLES, bool HG8>
+// values).  HG: the head-group size when it is 8 (one slot tile per tile) or
+// 4 (two), which folds the tiling to constants; 0: taken from the arguments.
+template <int BITS, bool ROPE, bool EXACT, int NWG, int TABLES, int HG>
 __global__ void __launch_bounds__(128 * NWG, 1)
     decode_tc_kernel(const CodecArgs a, const __grid_constant__ CUtensorMap out_map) {
   static_assert(ROPE == (TABLES > 0), "keys carry one table per slot tile, values none");
@@ -1111,16 +1111,18 @@ __global__ void __launch_bounds__(128 * NWG, 1)
   const int64_t my_tiles = first < a.num_tiles ? (a.num_tiles - 1 - first) / step + 1 : 0;
   // Row t of a tile: row block rb = t / 16 is slot tile mi of the tile (rb / hg)
   // for head rb % hg of the head group, slot t % 16; blocks past m * hg idle.
-  // Keys in head groups of 8 pair their rows instead: lanes 2i and 2i+1 of
-  // warp w hold slot i of heads 2w and 2w+1, so the two lanes that read one
+  // Keys in head groups of 8 or 4 pair their rows instead: warp w serves slot
+  // tile mi = w / (hg / 2) and heads hp, hp + 1 of it (hp = 2 (w % (hg / 2))),
+  // lanes 2i and 2i+1 slot i of the two heads, so the two lanes that read one
   // RoPE table entry sit in the same quarter warp (one shared-memory access
   // serves both), and a warp's 32 rows are one box of 2 heads x 16 tokens.
-  constexpr bool PAIRS = ROPE && HG8;
-  const int hg = HG8 ? 8 : a.hg, m = HG8 ? 1 : a.tc_m;
+  constexpr bool PAIRS = ROPE && (HG == 8 || HG == 4);
+  const int hg = HG ? HG : a.hg, m = HG ? 8 / HG : a.tc_m;
   const int rb = t >> 4, slot = PAIRS ? (lane >> 1) : (t & 15);
   const bool rb_used = PAIRS || rb < m * hg;
-  const int mi = PAIRS || !rb_used ? 0 : rb / hg;
-  const int hrel = PAIRS ? 2 * wl + (lane & 1) : (rb_used ? rb % hg : 0);
+  const int mi = PAIRS ? wl / (hg / 2) : (rb_used ? rb / hg : 0);
+  const int hp = PAIRS ? 2 * (wl % (hg / 2)) : 0;
+  const int hrel = PAIRS ? hp + (lane & 1) : (rb_used ? rb % hg : 0);
   // A tile index -> (head group, unit, first slot tile).
   auto tile_at = [&](int64_t t64, int& group, int& unit, int64_t& stile0) {
     const uint32_t tt = static_cast<uint32_t>(t64);
@@ -1135,7 +1137,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
     int64_t stile0;
     tile_at(t64, group, unit, stile0);
     const int64_t st = stile0 + mi;
-    if (HG8 || (rb_used && st < a.slot_tiles))
+    if (HG == 8 || (rb_used && st < a.slot_tiles))
       load_codes_at<BITS, EXACT>(a, unit, group * hg + hrel, st, slot, wr, mr);
   };
   uint32_t w[4 * BITS];
@@ -1157,7 +1159,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
     tile_at(t64, group, unit, stile0);
 #pragma unroll
     for (int x = 0; x < kT; ++x) {
-      const int32_t src = HG8 || stile0 + x < a.slot_tiles
+      const int32_t src = HG == 8 || stile0 + x < a.slot_tiles
                               ? slot_src_at(a, unit, stile0 + x, fslot) : -1;
       rvalid[x] = src >= 0;
       if (rvalid[x]) {
@@ -1238,8 +1240,9 @@ __global__ void __launch_bounds__(128 * NWG, 1)
       int group, unit;
       int64_t stile0;
       tile_at(first + k * step, group, unit, stile0);
-      if (PAIRS) {  // rows 32 wl .. 32 wl + 31: heads 2 wl, 2 wl + 1 of 16 tokens
-        const int y = static_cast<int>(stile0 * kSlots), h = group * 8 + 2 * wl;
+      if (PAIRS && (HG == 8 || stile0 + mi < a.slot_tiles)) {
+        // rows 32 wl .. 32 wl + 31: heads hp, hp + 1 of the 16 tokens of slot tile mi
+        const int y = static_cast<int>((stile0 + mi) * kSlots), h = group * hg + hp;
         const uint32_t src = a_main + wl * 4096;
         tma_store_4d(&out_map, src, 0, h, y, unit);
         tma_store_4d(&out_map, src + 16384, 64, h, y, unit);
@@ -1249,7 +1252,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
         const int rbi = 2 * wl + b2;
         if (rbi >= m * hg) continue;
         const int64_t st = stile0 + rbi / hg;
-        if (!HG8 && st >= a.slot_tiles) continue;
+        if (HG != 8 && st >= a.slot_tiles) continue;
         const int y = static_cast<int>(st * kSlots);
         const int h = group * hg + rbi % hg;
         const uint32_t src = a_main + rbi * 2048;
@@ -1336,17 +1339,17 @@ static int tc_slot_tiles_per_tile(int hg, bool rope) {
   return rope && m > 2 ? 0 : m;
 }
 
-template <int BITS, bool ROPE, bool EXACT, int NWG, int TABLES, bool HG8>
+template <int BITS, bool ROPE, bool EXACT, int NWG, int TABLES, int HG>
 static cudaError_t launch_decode_tc_on(const CodecArgs& a, const CUtensorMap& map, int sms,
                                        cudaStream_t stream) {
   const void* fn =
-      reinterpret_cast<const void*>(decode_tc_kernel<BITS, ROPE, EXACT, NWG, TABLES, HG8>);
+      reinterpret_cast<const void*>(decode_tc_kernel<BITS, ROPE, EXACT, NWG, TABLES, HG>);
   constexpr int smem = tc_smem_bytes<NWG, TABLES>();
   static_assert(smem <= 232448, "one CTA per SM within 227 KB");
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   const int64_t grid = min64((a.num_tiles + NWG - 1) / NWG, static_cast<int64_t>(sms));
-  decode_tc_kernel<BITS, ROPE, EXACT, NWG, TABLES, HG8>
+  decode_tc_kernel<BITS, ROPE, EXACT, NWG, TABLES, HG>
       <<<static_cast<unsigned>(grid), 128 * NWG, smem, stream>>>(a, map);
   return cudaGetLastError();
 }
@@ -1374,18 +1377,18 @@ static cudaError_t launch_decode_tc(CodecArgs a, const CUtensorMap& map, int uni
   if (engine == NQ_DECODE_AUTO && a.num_tiles < static_cast<int64_t>(2) * nwg * sms)
     return cudaSuccess;
   *used = true;
-  constexpr int T1 = ROPE ? 1 : 0;
-  if (a.hg == 8) {
-    if (!ROPE) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, T1, true>(a, map, sms, stream);
-    CUtensorMap pairs;  // keys: rows in head pairs (see decode_tc_kernel)
-    if ((err = make_out_map(&pairs, a, units, true)) != cudaSuccess) return err;
-    return launch_decode_tc_on<BITS, ROPE, EXACT, 4, T1, true>(a, pairs, sms, stream);
-  }
   if constexpr (!ROPE) {
-    return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, false>(a, map, sms, stream);
+    if (a.hg == 8) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, 8>(a, map, sms, stream);
+    return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, 0>(a, map, sms, stream);
   } else {
-    if (m == 1) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 1, false>(a, map, sms, stream);
-    return launch_decode_tc_on<BITS, ROPE, EXACT, 3, 2, false>(a, map, sms, stream);
+    if (a.hg == 8 || a.hg == 4) {
+      CUtensorMap pairs;  // keys: rows in head pairs (see decode_tc_kernel)
+      if ((err = make_out_map(&pairs, a, units, true)) != cudaSuccess) return err;
+      if (a.hg == 8) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 1, 8>(a, pairs, sms, stream);
+      return launch_decode_tc_on<BITS, ROPE, EXACT, 3, 2, 4>(a, pairs, sms, stream);
+    }
+    if (m == 1) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 1, 0>(a, map, sms, stream);
+    return launch_decode_tc_on<BITS, ROPE, EXACT, 3, 2, 0>(a, map, sms, stream);
   }
 }
 
