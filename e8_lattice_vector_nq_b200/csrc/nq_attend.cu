@@ -198,16 +198,19 @@ __global__ void __launch_bounds__(256, GT == 8 ? 1 : 2) attend_partial_kernel(co
     // ---- keys and scores (a token past the chunk has kappa 0 and score -inf)
     float sc[GT];
     {
-      // only this half's code words are read (the other half's stay zero and
-      // are not used by the reconstruction)
+      // only this half's code words are read, and each is placed in both
+      // halves' positions, so that every index into wc is a constant (a
+      // runtime index would put the array in local memory)
       uint32_t wc[4 * BK];
       const uint32_t kt = kcb + (k & 1) * (kSlots * kKStride) + slot_l * kKStride;
 #pragma unroll
-      for (int c = 0; c < 4 * BK; ++c) wc[c] = 0u;
-#pragma unroll
       for (int c = 0; c < BK; ++c) {
-        wc[BK * half + c] = lds32(kt + 4 * (BK * half + c));
-        wc[2 * BK + BK * half + c] = lds32(kt + 4 * (2 * BK + BK * half + c));
+        const uint32_t wa = lds32(kt + 4 * (BK * half + c));
+        const uint32_t wb = lds32(kt + 4 * (2 * BK + BK * half + c));
+        wc[c] = wa;
+        wc[BK + c] = wa;
+        wc[2 * BK + c] = wb;
+        wc[3 * BK + c] = wb;
       }
       float2 v[32];
       reconstruct_half<BK>(wc, kmc, half, v);
