@@ -1379,6 +1379,7 @@ static cudaError_t launch_decode_tc(CodecArgs a, const CUtensorMap& map, int uni
   *used = true;
   if constexpr (!ROPE) {
     if (a.hg == 8) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, 8>(a, map, sms, stream);
+    if (a.hg == 4) return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, 4>(a, map, sms, stream);
     return launch_decode_tc_on<BITS, ROPE, EXACT, 4, 0, 0>(a, map, sms, stream);
   } else {
     if (a.hg == 8 || a.hg == 4) {
