@@ -702,29 +702,30 @@ __device__ __forceinline__ void decode_half(const uint32_t (&w)[4 * BITS], uint3
 // the words and returns the regular meta word (coset mask | sigma << 16).
 template <int BITS>
 __device__ __forceinline__ uint32_t unfold_exact(uint32_t (&w)[4 * BITS], uint32_t sig16) {
+  constexpr int kGB = 8 * BITS;                                 // bits per group
+  constexpr uint32_t kLsb8 = BITS == 3 ? 0x249249u : 0x5555u;  // low bits of codes 0..7
   uint32_t mask = 0u;
 #pragma unroll
   for (int g = 0; g < 16; ++g) {
-    constexpr int kGB = 8 * BITS;  // bits per group
-    const int p = kGB * g;
-    const int wi = p >> 5, off = p & 31;
-    const int wn = wi + 1 < 4 * BITS ? wi + 1 : wi;
-    const uint32_t G = (off + kGB <= 32 ? (w[wi] >> off) : __funnelshift_r(w[wi], w[wn], off)) &
-                       ((1u << kGB) - 1u);
-    // low bits of codes 0..6: 0x49249 (3-bit fields), 0x1555 (2-bit fields)
-    constexpr uint32_t kLsb = BITS == 3 ? 0x49249u : 0x1555u;
-    const uint32_t h = (G >> (7 * BITS)) & 1u;
-    const uint32_t par = __popc(G & kLsb) & 1u;
-    const int q = p + 7 * BITS;
-    w[q >> 5] ^= (h ^ par) << (q & 31);
-    mask |= h << g;
+    // the parity of the low bits of codes 0..7 (the stored coset bit included)
+    // is the coset bit xor the true low bit of code 7, so xor-ing it into the
+    // stored bit restores that bit; groups cross a word boundary only for 3
+    // bits, and never past the last word
+    const int p = kGB * g, wi = p >> 5, off = p & 31;
+    uint32_t x = w[wi] & (kLsb8 << off);
+    if (off + kGB > 32) x ^= w[wi + 1] & (kLsb8 >> (32 - off));
+    const int q = p + 7 * BITS, qw = q >> 5, qb = q & 31;
+    mask |= ((w[qw] >> qb) & 1u) << g;
+    w[qw] ^= (static_cast<uint32_t>(__popc(x)) & 1u) << qb;
   }
   return mask | (sig16 << 16);
 }
 
 // Codes and meta of the vector (unit, head h, slot stile * 16 + slot_l), if
-// that slot is below n (registers, loaded one tile ahead).
-template <int BITS, bool EXACT>
+// that slot is below n (registers, loaded one tile ahead).  RAW (exact layout
+// only): meta is the raw fp16 scale and the words stay folded, for the caller
+// to unfold when it uses them (so that the loads are not waited for here).
+template <int BITS, bool EXACT, bool RAW = false>
 __device__ __forceinline__ void load_codes_at(const CodecArgs& a, int unit, int h, int64_t stile,
                                               int slot_l, uint32_t (&w)[4 * BITS],
                                               uint32_t& meta) {
@@ -740,7 +741,9 @@ __device__ __forceinline__ void load_codes_at(const CodecArgs& a, int unit, int 
       w[4 * c + 2] = q.z;
       w[4 * c + 3] = q.w;
     }
-    if (EXACT)
+    if (EXACT && RAW)
+      meta = __ldg(reinterpret_cast<const unsigned short*>(a.meta) + vec);
+    else if (EXACT)
       meta = unfold_exact<BITS>(w, __ldg(reinterpret_cast<const unsigned short*>(a.meta) + vec));
     else
       meta = __ldg(a.meta + vec);
@@ -1138,7 +1141,7 @@ __global__ void __launch_bounds__(128 * NWG, 1)
     tile_at(t64, group, unit, stile0);
     const int64_t st = stile0 + mi;
     if (HG == 8 || (rb_used && st < a.slot_tiles))
-      load_codes_at<BITS, EXACT>(a, unit, group * hg + hrel, st, slot, wr, mr);
+      load_codes_at<BITS, EXACT, !ROPE>(a, unit, group * hg + hrel, st, slot, wr, mr);
   };
   uint32_t w[4 * BITS];
   uint32_t meta = 0u;
@@ -1185,6 +1188,9 @@ __global__ void __launch_bounds__(128 * NWG, 1)
     // this warp's rows of A are its output staging: its last stores must have read them
     if (lane == 0) bulk_wait_read_all();
     __syncwarp();
+    // exact-layout values were loaded raw a tile ago (keys unfold at the load:
+    // deferred, their kernel spills)
+    if (EXACT && !ROPE) meta = unfold_exact<BITS>(w, meta & 0xFFFFu);
     tc_write_a<BITS>(w, meta, a_main, a_x, t);
     const uint32_t mk = meta;
     fence_proxy_async_smem();
