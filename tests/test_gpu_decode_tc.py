@@ -11,7 +11,8 @@ words, every coset mask, scales from zero and subnormal to the largest fp16),
 ragged slot counts on both sides of the 16-slot tile, every head-group size
 1..8 (with idle rows for 3, 5, 6 and 7), several head groups (16 and 24
 heads), kept-list positions with one and two RoPE tables per tile, output
-views with padding, slot and position offsets, and the exact layout.  Every
+views with padding and token-major output views, slot and position offsets,
+and the exact layout.  Every
 decoded bf16 element must equal the oracle's decode of the same store.
 """
 import numpy as np
@@ -122,6 +123,37 @@ def test_kept_positions_views_and_offsets(nq, oq, heads):
         assert torch.count_nonzero(o[:, heads]) == 0
         assert torch.count_nonzero(o[:, :, :10]) == 0 and torch.count_nonzero(o[:, :, 310:]) == 0
     assert torch.count_nonzero(out_k[..., :16]) == 0 and torch.count_nonzero(out_v[..., 128:]) == 0
+
+
+@pytest.mark.parametrize("engine", ["tensor", "cuda"])
+@pytest.mark.parametrize("heads", [8, 4, 3])
+def test_token_major_output_views(nq, oq, heads, engine):
+    """Outputs held token-major ([units][tokens][heads][128], passed as a permuted
+    view, so the head stride is below the token stride): the paired key rows
+    (8 and 4 heads) store boxes of 2 heads x 16 tokens through a map that lists
+    heads before tokens, which must land on the same elements."""
+    units, n, theta = 2, 277, 1e6
+    ks = random_store(nq, units, heads, 300, 3, 21)
+    vs = random_store(nq, units, heads, 300, 2, 22)
+    max_pos = 4096
+    rope = nq.rope_tables(theta, max_pos)
+    out_k = torch.zeros(units, n + 9, heads, 128, dtype=torch.bfloat16, device="cuda")
+    out_v = torch.zeros_like(out_k)
+    Ko, Vo = out_k[:, 4:4 + n].permute(0, 2, 1, 3), out_v[:, 4:4 + n].permute(0, 2, 1, 3)
+    if engine == "cuda":
+        nq.set_decode_engine(nq.DECODE_CUDA_CORES)
+    try:
+        nq.nq_decode(ks, vs, n, Ko, Vo, rope, max_pos)
+        torch.cuda.synchronize()
+    finally:
+        nq.set_decode_engine(nq.DECODE_TENSOR_CORES)
+    assert nq.device_error() == 0
+    for u in range(units):
+        Kr = oracle_decode(oq, ks, u, 0, n, 3, True, theta, np.arange(n, dtype=np.int64))
+        Vr = oracle_decode(oq, vs, u, 0, n, 2, False, theta, None)
+        assert np.array_equal(u16(Ko[u]), Kr) and np.array_equal(u16(Vo[u]), Vr)
+    for o in (out_k, out_v):  # nothing outside the views was written
+        assert torch.count_nonzero(o[:, :4]) == 0 and torch.count_nonzero(o[:, 4 + n:]) == 0
 
 
 @pytest.mark.parametrize("name", ["tiny", "decode_append", "qwen25_7b_64k", "mistral7b_32k"])
