@@ -21,7 +21,7 @@ full against the CPU oracle on all host cores (oracle/parity.py):
 The exact (24/16-bit) layout is checked the same way on every layer of the
 Mistral- and Llama-shaped caches (no mismatch is excused there).
 
-Parity rule (the benchmark spec): kept sets and codes bit-exact except where the
+Parity rule: kept sets and codes bit-exact except where the
 oracle's value lies within 1e-5 relative of a decision boundary; those are
 counted, reported and must stay below 1e-6 of the elements; decoded bf16
 identical.  Counts are printed (pytest -s) and appended as JSON lines to the
